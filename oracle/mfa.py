@@ -1,0 +1,223 @@
+"""One decode step of Step-3's MFA attention layer, float64 (test infrastructure only).
+
+Source passages (Step-3 pages):
+
+* bud-325 summary, "Key claims" and "Method": hidden size 7168; the query is produced by a
+  low-rank factorization -- down-projected from 7168 to rank 2048, normalized, then
+  up-projected to 64 heads x 256; one K head and one V head (head dim 256) are shared by
+  all 64 query heads, so the KV cache holds one K and one V vector per token; per-token
+  decode attention cost is max(attention compute, KV memory access).
+* redeep.blog post, "What's New" (same factorization: 7168 -> 2048 -> norm -> 64 x 256) and
+  the architecture table (hidden 7168, low-rank query dimension 2048, 64 query heads,
+  head dimension 256, max context 65,536).
+
+Readings where the pages are silent (each one is listed with its reason in the design
+notes of the repository):
+
+* the "normalization" is RMSNorm over the 2048-wide vector, eps = 1e-6 inside the square
+  root, elementwise gain gamma, no bias;
+* no positional encoding; q, k, v are used as projected;
+* k = x W_k and v = x W_v, each [7168, 256], straight from the hidden state;
+* softmax scale 1/sqrt(256) = 1/16;
+* weights are row-major [in, out]; head h of the up-projection is output columns
+  [256 h, 256 h + 256);
+* ``seq_lens[b]`` counts the positions attended *after* the new token is appended; the new
+  token's K/V row is written at row ``seq_lens[b] - 1`` and attended to;
+* the FP8 KV cache stores e4m3(value / scale) with one float32 scale per tensor for K and
+  one for V; bf16 caches store bf16(value); every rounding is to nearest, ties to even.
+
+The method reaches exactly (up to rounding order) the plain definition of attention, so
+the oracle is that definition: scores, a max-subtracted softmax and a weighted sum, with
+numpy's float64 matmul as the only library step.
+"""
+
+import numpy as np
+
+from . import codecs
+
+# Layer dimensions stated on the pages (bud-325 "Key claims"; redeep architecture table).
+HIDDEN = 7168
+Q_RANK = 2048
+N_HEADS = 64
+HEAD_DIM = 256
+MAX_CONTEXT = 65536
+
+# Readings for what the pages leave open.
+RMS_EPS = 1e-6
+SOFTMAX_SCALE = 1.0 / 16.0  # 1 / sqrt(HEAD_DIM)
+
+KV_BF16 = "bf16"
+KV_FP8 = "fp8_e4m3"
+
+
+# ----------------------------------------------------------------------------------------
+# query path: x -> down-projection -> normalization -> up-projection -> 64 heads
+# ----------------------------------------------------------------------------------------
+
+
+def q_down(x, w_qdown):
+    """c = x W_qdown: the low-rank query down-projection (7168 -> 2048).
+
+    x [B, D], w_qdown [D, R] (float64 values) -> c [B, R].
+    Pinned by: small-integer inputs whose sums are exact, compared with exact Python
+    integer sums (tests/test_oracle_mfa.py)."""
+    return np.asarray(x, np.float64) @ np.asarray(w_qdown, np.float64)
+
+
+def rms_norm(c, gamma, eps=RMS_EPS):
+    """c_hat = c / sqrt(mean(c^2) + eps) * gamma over the last axis (the "normalized" step,
+    read as RMSNorm).
+
+    Pinned by: the closed form mean(c_hat^2) = m / (m + eps) for gamma = 1 (m = mean(c^2)),
+    sign preservation, scale invariance and a hand-worked vector."""
+    c = np.asarray(c, np.float64)
+    ms = np.mean(c * c, axis=-1, keepdims=True)
+    return c / np.sqrt(ms + eps) * np.asarray(gamma, np.float64)
+
+
+def q_up(c_hat, w_qup, n_heads=N_HEADS):
+    """q = c_hat W_qup reshaped to [B, n_heads, head_dim]; head h is output columns
+    [h * head_dim, (h + 1) * head_dim).
+
+    Pinned by: exact small-integer sums and a one-hot weight that routes a chosen input
+    element to a chosen (head, dim) slot."""
+    q = np.asarray(c_hat, np.float64) @ np.asarray(w_qup, np.float64)
+    b, n = q.shape
+    return q.reshape(b, n_heads, n // n_heads)
+
+
+def query_proj(x, w_qdown, gamma, w_qup, eps=RMS_EPS, n_heads=N_HEADS, emulate=True):
+    """The MFA query path. Returns (c_hat, q).
+
+    With ``emulate`` the two results that the CUDA path stores as bf16 buffers (the
+    normalized low-rank query that feeds the up-projection, and q itself) are rounded to
+    bf16 here as well, so the end-to-end comparison measures the kernels' arithmetic
+    rather than those two storage roundings. ``emulate=False`` keeps pure float64."""
+    c_hat = rms_norm(q_down(x, w_qdown), gamma, eps)
+    if emulate:
+        c_hat = codecs.bf16_round(c_hat)
+    q = q_up(c_hat, w_qup, n_heads)
+    if emulate:
+        q = codecs.bf16_round(q)
+    return c_hat, q
+
+
+# ----------------------------------------------------------------------------------------
+# the shared K/V head and its cache
+# ----------------------------------------------------------------------------------------
+
+
+def kv_project(x, w_k, w_v):
+    """k = x W_k, v = x W_v: the single shared K head and V head of the new token.
+
+    Pinned by: one-hot weights (k equals a chosen element of x exactly)."""
+    x = np.asarray(x, np.float64)
+    return x @ np.asarray(w_k, np.float64), x @ np.asarray(w_v, np.float64)
+
+
+def kv_store(values, kv_dtype, scale=1.0):
+    """Values -> the codes a cache of ``kv_dtype`` holds: bf16 bits (uint16), or
+    e4m3(value / scale) codes (uint8)."""
+    if kv_dtype == KV_BF16:
+        return codecs.bf16_encode(values)
+    if kv_dtype == KV_FP8:
+        return codecs.e4m3_encode(np.asarray(values, np.float64) / float(scale))
+    raise ValueError(f"unknown kv dtype {kv_dtype!r}")
+
+
+def kv_load(codes, kv_dtype, scale=1.0):
+    """Cache codes -> float64 values (e4m3 codes are multiplied by their scale)."""
+    if kv_dtype == KV_BF16:
+        return codecs.bf16_decode(codes)
+    if kv_dtype == KV_FP8:
+        return codecs.e4m3_decode(codes) * float(scale)
+    raise ValueError(f"unknown kv dtype {kv_dtype!r}")
+
+
+def kv_append(k_cache, v_cache, pos, k_codes, v_codes):
+    """Write the new token's K/V codes at row ``pos[b]`` of sequence b's cache.
+
+    k_cache, v_cache: lists of per-sequence code arrays [cap_b, head_dim]. Returns new
+    lists; every other row is left as it was. Pinned by: exact byte comparison of every
+    row (tests/test_oracle_mfa.py)."""
+    k_out, v_out = [], []
+    for b in range(len(k_cache)):
+        kc = np.array(k_cache[b], copy=True)
+        vc = np.array(v_cache[b], copy=True)
+        p = int(pos[b])
+        if not 0 <= p < kc.shape[0]:
+            raise IndexError(f"sequence {b}: row {p} outside capacity {kc.shape[0]}")
+        kc[p] = k_codes[b]
+        vc[p] = v_codes[b]
+        k_out.append(kc)
+        v_out.append(vc)
+    return k_out, v_out
+
+
+# ----------------------------------------------------------------------------------------
+# attention of the 64 query heads over the shared K/V head
+# ----------------------------------------------------------------------------------------
+
+
+def attention_weights(q_b, keys, scale=SOFTMAX_SCALE):
+    """Softmax weights of one sequence: w[h, j] = exp(s[h, j]) / sum_j exp(s[h, j]) with
+    s[h, j] = scale * q_b[h] . keys[j]. q_b [H, d], keys [L, d] -> [H, L].
+
+    The maximum over j is subtracted before exp, which leaves the weights unchanged.
+    Pinned by: two-token closed form (logistic of the score difference), weights summing
+    to 1, permutation invariance, and pure-Python brute force."""
+    s = (np.asarray(q_b, np.float64) @ np.asarray(keys, np.float64).T) * scale
+    s = s - np.max(s, axis=1, keepdims=True)
+    e = np.exp(s)
+    return e / np.sum(e, axis=1, keepdims=True)
+
+
+def decode_attn_seq(q_b, keys, values, scale=SOFTMAX_SCALE):
+    """out[h] = sum_j w[h, j] values[j] for one sequence. q_b [H, d], keys/values [L, d]
+    (float64, L >= 1) -> [H, d].
+
+    Pinned by: L = 1 gives out = v; identical keys, or q = 0, give the mean of V;
+    brute force at tiny sizes."""
+    if keys.shape[0] < 1:
+        raise ValueError("attention needs at least one cached position")
+    return attention_weights(q_b, keys, scale) @ np.asarray(values, np.float64)
+
+
+def decode_attn(q, k_cache, v_cache, seq_lens, kv_dtype=KV_BF16, k_scale=1.0, v_scale=1.0,
+                scale=SOFTMAX_SCALE, seqs=None):
+    """Attention of every sequence (or of the sequences listed in ``seqs``) over rows
+    [0, seq_lens[b]) of its cache codes. q [B, H, d] float64 -> out [len(seqs), H, d]."""
+    seqs = range(len(k_cache)) if seqs is None else seqs
+    out = []
+    for b in seqs:
+        n = int(seq_lens[b])
+        keys = kv_load(k_cache[b][:n], kv_dtype, k_scale)
+        vals = kv_load(v_cache[b][:n], kv_dtype, v_scale)
+        out.append(decode_attn_seq(q[b], keys, vals, scale))
+    return np.stack(out)
+
+
+# ----------------------------------------------------------------------------------------
+# the whole decode step
+# ----------------------------------------------------------------------------------------
+
+
+def decode_layer(x, w_qdown, gamma, w_qup, w_k, w_v, k_cache, v_cache, seq_lens,
+                 kv_dtype=KV_BF16, k_scale=1.0, v_scale=1.0, eps=RMS_EPS,
+                 scale=SOFTMAX_SCALE, n_heads=N_HEADS, emulate=True, seqs=None):
+    """One MFA decode step, in the order the pages state it: the query path, then the new
+    token's K/V appended to its sequence's cache at row seq_lens[b] - 1, then attention of
+    all heads over rows [0, seq_lens[b]).
+
+    Returns a dict with c_hat, q, k_codes, v_codes (the appended rows), k_cache, v_cache
+    (after the append) and out [B or len(seqs), H, d]."""
+    c_hat, q = query_proj(x, w_qdown, gamma, w_qup, eps, n_heads, emulate)
+    k_new, v_new = kv_project(x, w_k, w_v)
+    k_codes = kv_store(k_new, kv_dtype, k_scale)
+    v_codes = kv_store(v_new, kv_dtype, v_scale)
+    pos = [int(n) - 1 for n in seq_lens]
+    k_cache2, v_cache2 = kv_append(k_cache, v_cache, pos, k_codes, v_codes)
+    out = decode_attn(q, k_cache2, v_cache2, seq_lens, kv_dtype, k_scale, v_scale, scale,
+                      seqs)
+    return dict(c_hat=c_hat, q=q, k_codes=k_codes, v_codes=v_codes, k_cache=k_cache2,
+                v_cache=v_cache2, out=out)

@@ -1,0 +1,331 @@
+"""Pins of the float64 oracle of the MFA decode step against things other than itself:
+exact integer arithmetic, closed forms, invariants the definition fixes, pure-Python brute
+force at tiny sizes, the page-stated dimensions, and planted mistakes that must be caught."""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import codecs
+from oracle import mfa
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def test_constants_match_page_dimensions():
+    with open(os.path.join(GOLDEN, "page_dims.json")) as f:
+        dims = json.load(f)
+    assert mfa.HIDDEN == dims["hidden"]
+    assert mfa.Q_RANK == dims["q_rank"]
+    assert mfa.N_HEADS == dims["n_heads"]
+    assert mfa.HEAD_DIM == dims["head_dim"]
+    assert mfa.MAX_CONTEXT == dims["max_context"]
+    assert mfa.SOFTMAX_SCALE == 1.0 / math.sqrt(dims["head_dim"])
+
+
+# ----------------------------------------------------------------------------------------
+# projections: exact small-integer arithmetic against Python integers
+# ----------------------------------------------------------------------------------------
+
+
+def _int_matmul(a, b):
+    return [[sum(int(a[i][k]) * int(b[k][j]) for k in range(len(b))) for j in range(len(b[0]))]
+            for i in range(len(a))]
+
+
+@pytest.mark.parametrize("bsz,din,dout", [(1, 7, 5), (3, 16, 12), (2, 33, 8)])
+def test_projections_exact_on_small_integers(bsz, din, dout):
+    rng = np.random.default_rng(din)
+    x = rng.integers(-3, 4, (bsz, din))
+    w = rng.integers(-2, 3, (din, dout))
+    want = np.array(_int_matmul(x.tolist(), w.tolist()), dtype=np.float64)
+    assert np.array_equal(mfa.q_down(x, w), want)
+    k, v = mfa.kv_project(x, w, -w)
+    assert np.array_equal(k, want) and np.array_equal(v, -want)
+    q = mfa.q_up(x, w, n_heads=1)
+    assert np.array_equal(q.reshape(bsz, dout), want)
+
+
+def test_q_up_head_ordering_one_hot():
+    # W routes input element i to output column 256 h + j: head h, dim j
+    r, heads, d = 6, 4, 8
+    rng = np.random.default_rng(0)
+    for _ in range(10):
+        i, h, j = rng.integers(r), rng.integers(heads), rng.integers(d)
+        w = np.zeros((r, heads * d))
+        w[i, h * d + j] = 1.0
+        c = rng.standard_normal((2, r))
+        q = mfa.q_up(c, w, n_heads=heads)
+        expect = np.zeros((2, heads, d))
+        expect[:, h, j] = c[:, i]
+        assert np.array_equal(q, expect)
+
+
+# ----------------------------------------------------------------------------------------
+# normalization
+# ----------------------------------------------------------------------------------------
+
+
+def test_rms_norm_hand_worked():
+    # c = (3, 4): mean square 12.5; with eps = 0 the result is c / sqrt(12.5)
+    out = mfa.rms_norm(np.array([[3.0, 4.0]]), np.ones(2), eps=0.0)
+    assert np.allclose(out, [[3 / math.sqrt(12.5), 4 / math.sqrt(12.5)]], rtol=0, atol=1e-15)
+    out = mfa.rms_norm(np.array([[3.0, 4.0]]), np.array([2.0, -1.0]), eps=0.0)
+    assert np.allclose(out, [[6 / math.sqrt(12.5), -4 / math.sqrt(12.5)]], rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("scale", [1e-4, 1e-2, 1.0, 37.0])
+def test_rms_norm_closed_form_mean_square(scale):
+    rng = np.random.default_rng(1)
+    c = rng.standard_normal((5, 2048)) * scale
+    eps = 1e-6
+    out = mfa.rms_norm(c, np.ones(2048), eps)
+    m = np.mean(c * c, axis=-1)
+    assert np.allclose(np.mean(out * out, axis=-1), m / (m + eps), rtol=1e-12, atol=0)
+    assert np.array_equal(np.sign(out), np.sign(c))
+
+
+# ----------------------------------------------------------------------------------------
+# attention: closed forms, invariants, brute force
+# ----------------------------------------------------------------------------------------
+
+
+def test_attention_single_position_returns_v():
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((64, 256)) * 5
+    k = rng.standard_normal((1, 256))
+    v = rng.standard_normal((1, 256))
+    out = mfa.decode_attn_seq(q, k, v)
+    assert np.array_equal(out, np.repeat(v, 64, axis=0))
+
+
+def test_attention_two_positions_closed_form_ln3():
+    # q . k0 / 16 = ln 3 and q . k1 = 0  =>  weights 3/4 and 1/4 exactly (logistic)
+    d = 256
+    q = np.zeros((1, d))
+    q[0, 0] = 16.0
+    k = np.zeros((2, d))
+    k[0, 0] = math.log(3.0)
+    v = np.stack([np.full(d, 1.0), np.full(d, 5.0)])
+    out = mfa.decode_attn_seq(q, k, v)
+    assert np.allclose(out, 0.75 * v[0] + 0.25 * v[1], rtol=0, atol=1e-14)
+    w = mfa.attention_weights(q, k)
+    assert np.allclose(w, [[0.75, 0.25]], rtol=0, atol=1e-15)
+
+
+def test_attention_logistic_for_random_pairs():
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        q = rng.standard_normal((3, 256))
+        k = rng.standard_normal((2, 256)) * 3
+        w = mfa.attention_weights(q, k)
+        s = q @ k.T / 16.0
+        w0 = 1.0 / (1.0 + np.exp(s[:, 1] - s[:, 0]))
+        assert np.allclose(w[:, 0], w0, rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("L", [1, 2, 5, 64, 129])
+def test_attention_identical_keys_or_zero_query_give_mean_of_v(L):
+    rng = np.random.default_rng(L)
+    q = rng.standard_normal((64, 256)) * 4
+    v = rng.standard_normal((L, 256))
+    k_same = np.repeat(rng.standard_normal((1, 256)), L, axis=0)
+    mean_v = np.mean(v, axis=0)
+    assert np.allclose(mfa.decode_attn_seq(q, k_same, v), mean_v, rtol=0, atol=1e-13)
+    k = rng.standard_normal((L, 256))
+    assert np.allclose(mfa.decode_attn_seq(np.zeros((64, 256)), k, v), mean_v, rtol=0,
+                       atol=1e-13)
+
+
+def test_attention_weights_sum_to_one_and_permutation_invariance():
+    rng = np.random.default_rng(4)
+    q = rng.standard_normal((64, 256)) * 2
+    k = rng.standard_normal((300, 256)) * 2
+    v = rng.standard_normal((300, 256))
+    w = mfa.attention_weights(q, k)
+    assert np.allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-13)
+    assert (w >= 0).all()
+    perm = rng.permutation(300)
+    assert np.allclose(mfa.decode_attn_seq(q, k, v), mfa.decode_attn_seq(q, k[perm], v[perm]),
+                       rtol=1e-12, atol=1e-14)
+    # heads are independent: identical query rows give identical output rows
+    q2 = np.repeat(q[:1], 64, axis=0)
+    o = mfa.decode_attn_seq(q2, k, v)
+    assert np.allclose(o, np.repeat(o[:1], 64, axis=0), rtol=0, atol=0)
+
+
+def _brute_layer(x, wd, gamma, wu, wk, wv, caches_k, caches_v, lens, heads, eps, scale):
+    """Pure-Python loops (math.fsum / math.exp / math.sqrt) of the whole step, no numpy."""
+    bsz, dim = len(x), len(x[0])
+    rank, hd = len(wd[0]), len(wk[0])
+    hdim = len(wu[0]) // heads
+    outs = []
+    for b in range(bsz):
+        c = [math.fsum(x[b][i] * wd[i][r] for i in range(dim)) for r in range(rank)]
+        ms = math.fsum(t * t for t in c) / rank
+        ch = [c[r] / math.sqrt(ms + eps) * gamma[r] for r in range(rank)]
+        q = [math.fsum(ch[r] * wu[r][j] for r in range(rank)) for j in range(heads * hdim)]
+        kn = [math.fsum(x[b][i] * wk[i][j] for i in range(dim)) for j in range(hd)]
+        vn = [math.fsum(x[b][i] * wv[i][j] for i in range(dim)) for j in range(hd)]
+        n = lens[b]
+        # caches_* already hold the new row, rounded to bf16 by the cache, at row n - 1;
+        # it must lie within half a bf16 ulp (<= 2**-8 relative) of the exact projection
+        for new, row in ((kn, caches_k[b][n - 1]), (vn, caches_v[b][n - 1])):
+            for a, r in zip(new, row):
+                assert abs(a - r) <= abs(a) * 2.0 ** -8
+        ks = [list(r) for r in caches_k[b][:n]]
+        vs = [list(r) for r in caches_v[b][:n]]
+        head_out = []
+        for h in range(heads):
+            qh = q[h * hdim:(h + 1) * hdim]
+            s = [scale * math.fsum(qh[j] * ks[t][j] for j in range(hd)) for t in range(n)]
+            m = max(s)
+            e = [math.exp(si - m) for si in s]
+            z = math.fsum(e)
+            head_out.append([math.fsum(e[t] * vs[t][j] for t in range(n)) / z
+                             for j in range(hd)])
+        outs.append(head_out)
+    return np.array(outs)
+
+
+@pytest.mark.parametrize("lens", [[1], [3, 1, 7], [9, 4]])
+def test_decode_layer_matches_pure_python_brute_force(lens):
+    rng = np.random.default_rng(sum(lens))
+    dim, rank, heads, hd = 12, 8, 4, 6
+    bsz = len(lens)
+    x = rng.standard_normal((bsz, dim))
+    wd = rng.standard_normal((dim, rank)) / math.sqrt(dim)
+    gamma = rng.uniform(0.5, 1.5, rank)
+    wu = rng.standard_normal((rank, heads * hd)) / math.sqrt(rank)
+    wk = rng.standard_normal((dim, hd)) / math.sqrt(dim)
+    wv = rng.standard_normal((dim, hd)) / math.sqrt(dim)
+    ck = [rng.standard_normal((n, hd)) for n in lens]
+    cv = [rng.standard_normal((n, hd)) for n in lens]
+    eps, scale = 1e-6, 1.0 / math.sqrt(hd)
+    # the oracle works on stored codes; use bf16-exact values so the codes are lossless
+    ck = [codecs.bf16_round(t) for t in ck]
+    cv = [codecs.bf16_round(t) for t in cv]
+    kc = [codecs.bf16_encode(t) for t in ck]
+    vc = [codecs.bf16_encode(t) for t in cv]
+    res = mfa.decode_layer(x, wd, gamma, wu, wk, wv, kc, vc, lens, eps=eps, scale=scale,
+                           n_heads=heads, emulate=False)
+    # the appended row is rounded to bf16 by the cache; feed brute force the same row
+    k_new, v_new = mfa.kv_project(x, wk, wv)
+    ck2 = [np.vstack([ck[b][:lens[b] - 1], codecs.bf16_round(k_new[b])[None]])
+           for b in range(bsz)]
+    cv2 = [np.vstack([cv[b][:lens[b] - 1], codecs.bf16_round(v_new[b])[None]])
+           for b in range(bsz)]
+    want = _brute_layer(x.tolist(), wd.tolist(), gamma.tolist(), wu.tolist(), wk.tolist(),
+                        wv.tolist(), [t.tolist() for t in ck2], [t.tolist() for t in cv2],
+                        lens, heads, eps, scale)
+    assert np.allclose(res["out"], want, rtol=1e-12, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------------------
+# KV append: bytes
+# ----------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("kv_dtype", [mfa.KV_BF16, mfa.KV_FP8])
+def test_kv_append_writes_exactly_one_row(kv_dtype):
+    rng = np.random.default_rng(9)
+    caps = [5, 1, 8]
+    dt = np.uint16 if kv_dtype == mfa.KV_BF16 else np.uint8
+    kc = [rng.integers(0, 120, (c, 16)).astype(dt) for c in caps]
+    vc = [rng.integers(0, 120, (c, 16)).astype(dt) for c in caps]
+    pos = [4, 0, 3]
+    newk = rng.integers(0, 120, (3, 16)).astype(dt)
+    newv = rng.integers(0, 120, (3, 16)).astype(dt)
+    k2, v2 = mfa.kv_append(kc, vc, pos, newk, newv)
+    for b, p in enumerate(pos):
+        for r in range(caps[b]):
+            wk = newk[b] if r == p else kc[b][r]
+            wv = newv[b] if r == p else vc[b][r]
+            assert np.array_equal(k2[b][r], wk) and np.array_equal(v2[b][r], wv)
+        assert np.array_equal(kc[b], kc[b])  # inputs untouched
+    with pytest.raises(IndexError):
+        mfa.kv_append(kc, vc, [5, 0, 0], newk, newv)
+
+
+def test_kv_store_fp8_power_of_two_scale_is_exact():
+    # one-hot projection -> k equals a chosen element of x; values on the e4m3 grid times a
+    # power-of-two scale are stored and loaded back exactly
+    grid = codecs.e4m3_decode(np.arange(0, 0x7F))
+    rng = np.random.default_rng(12)
+    vals = rng.choice(grid, 64) * 0.125 * rng.choice([-1, 1], 64)
+    x = vals[None, :]
+    w = np.eye(64)
+    k, v = mfa.kv_project(x, w, 2 * w)
+    codes = mfa.kv_store(k, mfa.KV_FP8, 0.125)
+    assert np.array_equal(mfa.kv_load(codes, mfa.KV_FP8, 0.125), vals[None, :])
+    codes = mfa.kv_store(v, mfa.KV_FP8, 0.25)
+    assert np.array_equal(mfa.kv_load(codes, mfa.KV_FP8, 0.25), 2 * vals[None, :])
+
+
+def test_decode_layer_appends_at_len_minus_one_and_attends_to_it():
+    # L = 1: the only attended row is the new token's v (rounded to bf16), for every head
+    rng = np.random.default_rng(13)
+    dim, rank, heads, hd = 10, 4, 3, 5
+    x = rng.standard_normal((2, dim))
+    wd, wu = rng.standard_normal((dim, rank)), rng.standard_normal((rank, heads * hd))
+    wk, wv = rng.standard_normal((dim, hd)), rng.standard_normal((dim, hd))
+    kc = [codecs.bf16_encode(rng.standard_normal((4, hd))) for _ in range(2)]
+    vc = [codecs.bf16_encode(rng.standard_normal((4, hd))) for _ in range(2)]
+    res = mfa.decode_layer(x, wd, np.ones(rank), wu, wk, wv, kc, vc, [1, 3], n_heads=heads,
+                           scale=0.3)
+    v_new = codecs.bf16_round(x @ wv)
+    assert np.array_equal(res["out"][0], np.repeat(v_new[0][None], heads, axis=0))
+    assert np.array_equal(res["v_cache"][1][2], codecs.bf16_encode(v_new[1]))
+    assert np.array_equal(res["v_cache"][1][3], vc[1][3])  # row past the length untouched
+
+
+# ----------------------------------------------------------------------------------------
+# planted mistakes: each must be caught by one of the pins above
+# ----------------------------------------------------------------------------------------
+
+
+def _ln3_pin(attn_seq):
+    d = 256
+    q = np.zeros((1, d))
+    q[0, 0] = 16.0
+    k = np.zeros((2, d))
+    k[0, 0] = math.log(3.0)
+    v = np.stack([np.full(d, 1.0), np.full(d, 5.0)])
+    return np.allclose(attn_seq(q, k, v), 0.75 * v[0] + 0.25 * v[1], rtol=0, atol=1e-12)
+
+
+def test_planted_wrong_scale_is_caught():
+    assert _ln3_pin(mfa.decode_attn_seq)
+    assert not _ln3_pin(lambda q, k, v: mfa.decode_attn_seq(q, k, v, scale=1 / math.sqrt(255)))
+
+
+def test_planted_transposed_value_product_is_caught():
+    def wrong(q, k, v):  # weights applied to the wrong cache rows (reversed order of v)
+        return mfa.attention_weights(q, k) @ v[::-1]
+    assert not _ln3_pin(wrong)
+
+
+def test_planted_eps_outside_sqrt_is_caught():
+    c = np.random.default_rng(1).standard_normal((3, 2048)) * 1e-3
+    m = np.mean(c * c, axis=-1)
+    eps = 1e-6
+
+    def wrong(c, g, e):
+        return c / (np.sqrt(np.mean(c * c, axis=-1, keepdims=True)) + e) * g
+    good = mfa.rms_norm(c, np.ones(2048), eps)
+    bad = wrong(c, np.ones(2048), eps)
+    assert np.allclose(np.mean(good ** 2, -1), m / (m + eps), rtol=1e-12)
+    assert not np.allclose(np.mean(bad ** 2, -1), m / (m + eps), rtol=1e-9)
+
+
+def test_planted_off_by_one_append_row_is_caught():
+    rng = np.random.default_rng(21)
+    kc = [rng.integers(0, 9, (4, 3)).astype(np.uint16)]
+    new = np.full((1, 3), 77, np.uint16)
+    k2, _ = mfa.kv_append(kc, kc, [2], new, new)
+    assert np.array_equal(k2[0][2], new[0]) and np.array_equal(k2[0][3], kc[0][3])
+    k_bad, _ = mfa.kv_append(kc, kc, [3], new, new)
+    assert not np.array_equal(k_bad[0][2], new[0])
