@@ -1,0 +1,424 @@
+"""Benchmark of one MFA decode step (Step-3's Multi-Matrix Factorization Attention layer).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME|INDEX]
+
+A step is one whole decode step of the layer on one batch of synthetic inputs: hidden-state
+projections (query down-projection + RMSNorm + up-projection, K/V projection + cache
+append) and attention of the 64 heads over each sequence's shared K/V cache. The default
+workload is batch 32 at uniform context 4096 with a bf16 KV cache.
+
+Prints ONE JSON line (rank 0). `value` is whole-job decode throughput in tokens/s (one
+token per sequence per step, summed over ranks, divided by the slowest rank's device time)
+with every input already resident in HBM; `e2e` is the same metric through the public call
+with the step's inputs copied from pinned host memory and its output copied back inside
+the timed region. Between timed steps the inputs rotate over several device copies whose
+combined footprint is far above the 126 MB L2, so no step reads the previous step's bytes
+from L2. Multi-GPU runs (torchrun) shard sequences over ranks (weak scaling, no data-path
+collective: the decode step of one sequence needs nothing from another).
+
+`--impl reference` times the float64 CPU oracle on this host's cores on a bounded sample
+of the same workload (the baseline of this build; there is no runnable reference code).
+"""
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MFA decode-layer tokens/s at 4K/8K ctx; KV-stream HBM GB/s vs B200 peak"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "mfa_decode_b32_l4096_bf16"
+L2_BYTES = 126 * 1024 * 1024
+WEIGHT_BYTES = 2 * (7168 * 2048 + 2048 * 16384 + 2 * 7168 * 256)
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region (NVML in a thread; read-only queries)
+# ---------------------------------------------------------------------------------------
+
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - NVML missing
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                try:
+                    r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.reasons |= int(r)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU baseline: the float64 oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------------------
+
+
+def oracle_sample_throughput(inp, n_seq: int):
+    """Time the oracle's whole decode step for the first n_seq sequences; tokens/s."""
+    import numpy as np
+    from oracle import codecs
+    from oracle import mfa as omfa
+
+    def f64(t):
+        import torch
+        return codecs.bf16_decode(t.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+    def codes(t):
+        import torch
+        t = t.contiguous()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16)
+        return t.view(torch.uint8).numpy()
+
+    od = omfa.KV_BF16 if inp.kv_dtype == "bf16" else omfa.KV_FP8
+    w = [f64(inp.w_qdown), f64(inp.gamma), f64(inp.w_qup), f64(inp.w_k), f64(inp.w_v)]
+    x = f64(inp.x)[:n_seq]
+    kc = [codes(inp.k_cache[b]) for b in range(n_seq)]
+    vc = [codes(inp.v_cache[b]) for b in range(n_seq)]
+    lens = inp.seq_lens.tolist()[:n_seq]
+    t0 = time.perf_counter()
+    omfa.decode_layer(x, *w, kc, vc, lens, od, inp.k_scale, inp.v_scale)
+    dt = time.perf_counter() - t0
+    return n_seq / dt, dt
+
+
+def cpu_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------------------
+
+
+def attention_bytes(inp) -> int:
+    """Algorithmic HBM bytes of one attention launch: every attended K and V row once, q
+    read once and out written once per sequence."""
+    row = 256 * (2 if inp.kv_dtype == "bf16" else 1)
+    kv = 2 * row * int(inp.seq_lens.sum())
+    qo = 2 * inp.batch * 64 * 256 * 2
+    return kv + qo
+
+
+def kv_bytes(inp) -> int:
+    row = 256 * (2 if inp.kv_dtype == "bf16" else 1)
+    return 2 * row * int(inp.seq_lens.sum())
+
+
+def run_ours(args, wl, rank, world, local):
+    import torch
+    from decode_attention_10_b200 import build, mfa
+    from decode_attention_10_b200 import workloads as W
+
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    inp = W.generate_workload(wl, seed=1000 + wl.index + 7919 * rank)
+    bsz = inp.batch
+    step_bytes = WEIGHT_BYTES + kv_bytes(inp)
+    copies = max(2, math.ceil(3 * L2_BYTES / step_bytes))
+
+    class Copy:
+        pass
+
+    sets = []
+    for _ in range(copies):
+        c = Copy()
+        c.x = inp.x.to(dev)
+        c.w = [t.to(dev) for t in (inp.w_qdown, inp.gamma, inp.w_qup, inp.w_k, inp.w_v)]
+        if inp.k_buffer is not None:
+            kb, vb = inp.k_buffer.to(dev), inp.v_buffer.to(dev)
+            c.k, c.v = [kb[b] for b in range(bsz)], [vb[b] for b in range(bsz)]
+            c.keep = (kb, vb)
+        else:
+            c.k = [t.to(dev) for t in inp.k_cache]
+            c.v = [t.to(dev) for t in inp.v_cache]
+        c.cache = mfa.KVCache(c.k, c.v, inp.k_scale, inp.v_scale)
+        c.q = torch.empty(bsz, 64, 256, dtype=torch.bfloat16, device=dev)
+        c.out = torch.empty(bsz, 64, 256, dtype=torch.bfloat16, device=dev)
+        sets.append(c)
+    lens = inp.seq_lens.to(dev)
+    ws = mfa.Workspace(bsz, dev)
+
+    def layer(c):
+        mfa.decode_layer(c.x, *c.w, c.cache, lens, q_out=c.q, out=c.out, ws=ws)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for i in range(args.warmup):
+        layer(sets[i % copies])
+    torch.cuda.synchronize()
+    if mfa.get_error(ws) != 0:
+        raise RuntimeError("device error flag set during warm-up")
+    if not torch.isfinite(sets[0].out.float()).all():
+        raise RuntimeError("non-finite output")
+
+    # 1) the timed region: K whole decode steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record()
+        for i in range(args.steps):
+            layer(sets[i % copies])
+        e1.record()
+        torch.cuda.synchronize()
+    barrier()
+    t_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([t_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_ms = float(t.item())
+    ms_per_step = t_ms / args.steps
+    value = world * bsz * args.steps / (t_ms / 1e3)
+
+    # 2) the attention kernel alone: the same steps through the separate calls, with CUDA
+    #    events around every attention launch (on the launching stream)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    pos = lens - 1
+    for i in range(args.steps):
+        c = sets[i % copies]
+        mfa.query_proj(c.x, c.w[0], c.w[1], c.w[2], q_out=c.q, ws=ws)
+        mfa.kv_append(c.x, c.w[3], c.w[4], c.cache, pos, ws=ws)
+        evs[i][0].record()
+        mfa.decode_attn(c.q, c.cache, lens, out=c.out, ws=ws)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+    # 3) end to end through the public call with host buffers
+    x_host = [inp.x.pin_memory() for _ in range(copies)]
+    out_host = torch.empty(bsz, 64, 256, dtype=torch.bfloat16).pin_memory()
+    lens_host = inp.seq_lens.pin_memory()
+    barrier()
+    torch.cuda.synchronize()
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record()
+    for i in range(args.steps):
+        c = sets[i % copies]
+        c.x.copy_(x_host[i % copies], non_blocking=True)
+        lens.copy_(lens_host, non_blocking=True)
+        layer(c)
+        out_host.copy_(c.out, non_blocking=True)
+    e3.record()
+    torch.cuda.synchronize()
+    barrier()
+    t_e2e = e2.elapsed_time(e3)
+    if world > 1:
+        t = torch.tensor([t_e2e], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_e2e = float(t.item())
+    e2e_value = world * bsz * args.steps / (t_e2e / 1e3)
+
+    peak, peak_kind = measured_peaks()
+    a_bytes = attention_bytes(inp)
+    achieved = a_bytes / (attn_ms / 1e3) / 1e9
+    traffic = profiled_traffic(wl.name)
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if inp.kv_dtype == "bf16" else "bf16+fp8kv", "data": "synthetic",
+        "config": {"workload": wl.name, "batch_per_gpu": bsz, "global_batch": bsz * world,
+                   "context": wl.context, "kv_dtype": inp.kv_dtype,
+                   "heads": 64, "head_dim": 256, "hidden": 7168, "q_rank": 2048,
+                   "l2": f"inputs rotate over {copies} device copies "
+                         f"({step_bytes / 1e6:.0f} MB each, > 126 MB L2)",
+                   "parallelism": f"dp{world} (sequences sharded, weights replicated)"},
+        "kv_gbs": kv_bytes(inp) / (attn_ms / 1e3) / 1e9,
+        "attn_ms": attn_ms,
+        "roofline": {"kernel": "mfa decode attention (plan + split-K + merge, one launch)",
+                     "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": peak_kind,
+                     "bytes_per_launch": a_bytes, "traffic": traffic},
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": UNIT,
+                "h2d_bytes_per_step": bsz * 7168 * 2 + bsz * 4,
+                "d2h_bytes_per_step": bsz * 64 * 256 * 2},
+        "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_seq = min(bsz, 8)
+        tps, dt = oracle_sample_throughput(inp, n_seq)
+        result["cpu_baseline"] = {"value": tps, "unit": UNIT, "cores": cpu_cores(),
+                                  "kind": "oracle",
+                                  "sample": f"one whole decode step of {n_seq} of the "
+                                            f"{bsz} sequences (float64 numpy), {dt:.1f} s"}
+    return result
+
+
+LAUNCHES_PER_LAYER = 4  # x-projection, split-K finish (+RMSNorm, append), q_up, attention
+
+
+def profiled_traffic(workload_name):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
+    the current attention source; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        import hashlib
+        h = hashlib.sha256()
+        for name in d.get("sources", []):
+            with open(os.path.join(ROOT, name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != d.get("source_sha256"):
+            return None
+        entry = d.get("per_launch", {}).get(workload_name)
+        return None if entry is None else float(entry)
+    except Exception:
+        return None
+
+
+def run_reference(args, wl, rank, world):
+    """The oracle on host cores, on the same workload: each step is one whole decode step
+    of a bounded sample of the batch."""
+    from decode_attention_10_b200 import workloads as W
+    inp = W.generate_workload(wl)
+    n_seq = min(inp.batch, 2)
+    for _ in range(args.warmup):
+        oracle_sample_throughput(inp, n_seq)
+    times = []
+    for _ in range(args.steps):
+        _, dt = oracle_sample_throughput(inp, n_seq)
+        times.append(dt)
+    total = sum(times)
+    value = n_seq * len(times) / total
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch_per_gpu": inp.batch, "context": wl.context,
+                   "kv_dtype": inp.kv_dtype, "sample_sequences_per_step": n_seq},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"{n_seq} of {inp.batch} sequences per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    from decode_attention_10_b200 import workloads as W
+    try:
+        wl = W.workload(int(args.workload))
+    except ValueError:
+        wl = W.workload(args.workload)
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, wl, rank, world)), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, wl, rank, world)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,356 @@
+// extern "C" entry points of libmfa: argument checks, the device KV table, the workspace,
+// and the kernel sequence of each call. Declarations and the contract are in include/mfa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <vector>
+
+#include "mfa_internal.cuh"
+
+namespace mfa {
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool device_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  static int cached[64] = {0};
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) {
+    *sms = cached[dev];
+    return true;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return false;
+  if (dev >= 0 && dev < 64) cached[dev] = n;
+  *sms = n;
+  return true;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn != nullptr) return fn;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || p == nullptr)
+    return nullptr;
+  fn = reinterpret_cast<EncodeTiledFn>(p);
+  return fn;
+}
+
+// Tensor map over one sequence's cache rows: [rows, 256] elements, boxes of
+// (128 bytes of a row) x kTile rows, 128-byte swizzle -- the canonical K-major /
+// MN-major shared-memory layout of the tensor-core operands.
+bool encode_rows(EncodeTiledFn enc, CUtensorMap* m, void* base, int rows, int dtype) {
+  const bool fp8 = dtype == MFA_KV_FP8_E4M3;
+  const cuuint64_t elem = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {kHeadDim * elem};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / elem), (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r =
+      enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
+          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+mfa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MFA_OK : MFA_ERR_CUDA; }
+
+mfa_status check_kv(const mfa_kv_cache* kv) {
+  if (kv == nullptr || kv->table == nullptr) return MFA_ERR_INVALID_ARG;
+  if (kv->batch < 1 || kv->batch > kMaxBatch) return MFA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(kv->table) & 127u) != 0) return MFA_ERR_INVALID_ARG;
+  if (kv->dtype != MFA_KV_BF16 && kv->dtype != MFA_KV_FP8_E4M3) return MFA_ERR_UNSUPPORTED;
+  if (kv->dtype == MFA_KV_FP8_E4M3 && !(kv->k_scale > 0.f && kv->v_scale > 0.f))
+    return MFA_ERR_INVALID_ARG;
+  return MFA_OK;
+}
+
+mfa_status check_ws(void* ws, size_t ws_bytes, int batch, WsLayout* L) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MFA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (!device_sms(&sms)) return MFA_ERR_CUDA;
+  *L = ws_layout(batch, sms);
+  if (ws_bytes < L->total) return MFA_ERR_WORKSPACE;
+  return MFA_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
+                          const void* w_qup, float eps, void* q_out, int batch, void* ws,
+                          const WsLayout& L, cudaStream_t s) {
+  XProjArgs xa{};
+  xa.x = static_cast<const uint16_t*>(x);
+  xa.w[0] = static_cast<const uint16_t*>(w_qdown);
+  xa.w[1] = xa.w[2] = nullptr;
+  xa.batch = batch;
+  xa.tile_begin = 0;
+  xa.tile_end = kRank / 128;
+  xa.part = at<float>(ws, L.xproj_part);
+  cudaError_t e = launch_xproj(xa, s);
+  if (e != cudaSuccess) return MFA_ERR_CUDA;
+  FinishArgs fa{};
+  fa.part = xa.part;
+  fa.batch = batch;
+  fa.gamma = static_cast<const uint16_t*>(gamma);
+  fa.eps = eps;
+  fa.c_hat = at<uint16_t>(ws, L.c_hat);
+  fa.err = at<uint32_t>(ws, L.err);
+  e = launch_xproj_finish(fa, s);
+  if (e != cudaSuccess) return MFA_ERR_CUDA;
+  QUpArgs qa{};
+  qa.c_hat = fa.c_hat;
+  qa.w_qup = static_cast<const uint16_t*>(w_qup);
+  qa.batch = batch;
+  qa.q = static_cast<uint16_t*>(q_out);
+  return cuda_status(launch_q_up(qa, s));
+}
+
+}  // namespace
+}  // namespace mfa
+
+using namespace mfa;
+
+extern "C" {
+
+int32_t mfa_version(void) { return 100; }
+
+const char* mfa_status_str(int32_t status) {
+  switch (status) {
+    case MFA_OK: return "MFA_OK";
+    case MFA_ERR_INVALID_ARG: return "MFA_ERR_INVALID_ARG";
+    case MFA_ERR_UNSUPPORTED: return "MFA_ERR_UNSUPPORTED";
+    case MFA_ERR_CAPACITY: return "MFA_ERR_CAPACITY";
+    case MFA_ERR_WORKSPACE: return "MFA_ERR_WORKSPACE";
+    case MFA_ERR_CUDA: return "MFA_ERR_CUDA";
+    case MFA_ERR_EMPTY: return "MFA_ERR_EMPTY";
+    case MFA_ERR_TIMEOUT: return "MFA_ERR_TIMEOUT";
+    default: return "MFA_ERR_UNKNOWN";
+  }
+}
+
+size_t mfa_kv_table_bytes(int32_t batch) {
+  if (batch < 1 || batch > kMaxBatch) return 0;
+  return sizeof(KvSeq) * (size_t)batch;
+}
+
+mfa_status mfa_kv_table_init(void* table, size_t table_bytes, int32_t batch, int32_t dtype,
+                             void* const* k_ptrs, void* const* v_ptrs,
+                             const int32_t* capacity, void* stream) {
+  if (batch < 1 || batch > kMaxBatch) return MFA_ERR_INVALID_ARG;
+  if (table == nullptr || k_ptrs == nullptr || v_ptrs == nullptr || capacity == nullptr)
+    return MFA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(table) & 127u) != 0) return MFA_ERR_INVALID_ARG;
+  if (dtype != MFA_KV_BF16 && dtype != MFA_KV_FP8_E4M3) return MFA_ERR_UNSUPPORTED;
+  if (table_bytes < mfa_kv_table_bytes(batch)) return MFA_ERR_WORKSPACE;
+  for (int b = 0; b < batch; ++b) {
+    if (k_ptrs[b] == nullptr || v_ptrs[b] == nullptr) return MFA_ERR_INVALID_ARG;
+    if (!aligned16(k_ptrs[b]) || !aligned16(v_ptrs[b])) return MFA_ERR_INVALID_ARG;
+    if (capacity[b] < 1 || capacity[b] > MFA_MAX_CONTEXT) return MFA_ERR_INVALID_ARG;
+  }
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (enc == nullptr) return MFA_ERR_CUDA;
+  std::vector<KvSeq> host(batch);
+  std::memset(host.data(), 0, sizeof(KvSeq) * batch);
+  for (int b = 0; b < batch; ++b) {
+    if (!encode_rows(enc, &host[b].tmap_k, k_ptrs[b], capacity[b], dtype) ||
+        !encode_rows(enc, &host[b].tmap_v, v_ptrs[b], capacity[b], dtype))
+      return MFA_ERR_INVALID_ARG;
+    host[b].k = k_ptrs[b];
+    host[b].v = v_ptrs[b];
+    host[b].capacity = capacity[b];
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(table, host.data(), sizeof(KvSeq) * batch,
+                                  cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+size_t mfa_workspace_bytes(int32_t batch) {
+  if (batch < 1 || batch > kMaxBatch) return 0;
+  int sms = 0;
+  if (!device_sms(&sms)) return 0;
+  return ws_layout(batch, sms).total;
+}
+
+mfa_status mfa_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return MFA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, ws_bytes, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
+mfa_status mfa_get_error(void* ws, void* stream) {
+  if (ws == nullptr) return MFA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MFA_ERR_CUDA;
+  uint32_t bits = 0;
+  if (cudaMemcpy(&bits, ws, sizeof(bits), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  if (bits == 0) return MFA_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(bits), s) != cudaSuccess) return MFA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MFA_ERR_CUDA;
+  if (bits & kErrCapacity) return MFA_ERR_CAPACITY;
+  if (bits & kErrEmpty) return MFA_ERR_EMPTY;
+  return MFA_ERR_TIMEOUT;
+}
+
+mfa_status mfa_query_proj(const void* x, const void* w_qdown, const void* gamma,
+                          const void* w_qup, float eps, void* q_out, int32_t batch,
+                          void* ws, size_t ws_bytes, void* stream) {
+  if (batch < 1 || batch > kMaxBatch) return MFA_ERR_INVALID_ARG;
+  if (!(eps > 0.f)) return MFA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_qdown, gamma, w_qup, q_out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  mfa_status st = check_ws(ws, ws_bytes, batch, &L);
+  if (st != MFA_OK) return st;
+  return run_query_proj(x, w_qdown, gamma, w_qup, eps, q_out, batch, ws, L,
+                        static_cast<cudaStream_t>(stream));
+}
+
+mfa_status mfa_kv_append(const void* x, const void* w_k, const void* w_v,
+                         const mfa_kv_cache* kv, const int32_t* pos, void* ws,
+                         size_t ws_bytes, void* stream) {
+  mfa_status st = check_kv(kv);
+  if (st != MFA_OK) return st;
+  const void* ptrs[] = {x, w_k, w_v, pos};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  st = check_ws(ws, ws_bytes, kv->batch, &L);
+  if (st != MFA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  XProjArgs xa{};
+  xa.x = static_cast<const uint16_t*>(x);
+  xa.w[0] = nullptr;
+  xa.w[1] = static_cast<const uint16_t*>(w_k);
+  xa.w[2] = static_cast<const uint16_t*>(w_v);
+  xa.batch = kv->batch;
+  xa.tile_begin = kRank / 128;
+  xa.tile_end = kXProjCols / 128;
+  xa.part = at<float>(ws, L.xproj_part);
+  if (launch_xproj(xa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  FinishArgs fa{};
+  fa.part = xa.part;
+  fa.batch = kv->batch;
+  fa.kv = static_cast<const KvSeq*>(kv->table);
+  fa.kv_dtype = kv->dtype;
+  fa.k_scale = kv->k_scale;
+  fa.v_scale = kv->v_scale;
+  fa.pos = pos;
+  fa.pos_from_len = 0;
+  fa.err = at<uint32_t>(ws, L.err);
+  return cuda_status(launch_xproj_finish(fa, s));
+}
+
+mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t* seq_lens,
+                           float scale, void* out, void* ws, size_t ws_bytes, void* stream) {
+  mfa_status st = check_kv(kv);
+  if (st != MFA_OK) return st;
+  if (!(scale > 0.f)) return MFA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, seq_lens, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  st = check_ws(ws, ws_bytes, kv->batch, &L);
+  if (st != MFA_OK) return st;
+  AttnArgs aa{};
+  aa.q = static_cast<const uint16_t*>(q);
+  aa.kv = static_cast<const KvSeq*>(kv->table);
+  aa.kv_dtype = kv->dtype;
+  aa.k_scale = kv->k_scale;
+  aa.v_scale = kv->v_scale;
+  aa.seq_lens = seq_lens;
+  aa.scale = scale;
+  aa.out = static_cast<uint16_t*>(out);
+  aa.batch = kv->batch;
+  aa.partials = at<float>(ws, L.attn_part);
+  aa.counters = at<int32_t>(ws, L.counters);
+  aa.err = at<uint32_t>(ws, L.err);
+  aa.grid = L.attn_grid;
+  return cuda_status(launch_attention(aa, static_cast<cudaStream_t>(stream)));
+}
+
+mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamma,
+                            const void* w_qup, const void* w_k, const void* w_v, float eps,
+                            const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
+                            void* q_out, void* out, void* ws, size_t ws_bytes, void* stream) {
+  mfa_status st = check_kv(kv);
+  if (st != MFA_OK) return st;
+  if (!(eps > 0.f) || !(scale > 0.f)) return MFA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_qdown, gamma, w_qup, w_k, w_v, seq_lens, q_out, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  st = check_ws(ws, ws_bytes, kv->batch, &L);
+  if (st != MFA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int batch = kv->batch;
+  // one projection of x onto [W_qdown | W_k | W_v]
+  XProjArgs xa{};
+  xa.x = static_cast<const uint16_t*>(x);
+  xa.w[0] = static_cast<const uint16_t*>(w_qdown);
+  xa.w[1] = static_cast<const uint16_t*>(w_k);
+  xa.w[2] = static_cast<const uint16_t*>(w_v);
+  xa.batch = batch;
+  xa.tile_begin = 0;
+  xa.tile_end = kXProjCols / 128;
+  xa.part = at<float>(ws, L.xproj_part);
+  if (launch_xproj(xa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  // split-K sums, RMSNorm of the query half, K/V append at row seq_lens[b] - 1
+  FinishArgs fa{};
+  fa.part = xa.part;
+  fa.batch = batch;
+  fa.gamma = static_cast<const uint16_t*>(gamma);
+  fa.eps = eps;
+  fa.c_hat = at<uint16_t>(ws, L.c_hat);
+  fa.kv = static_cast<const KvSeq*>(kv->table);
+  fa.kv_dtype = kv->dtype;
+  fa.k_scale = kv->k_scale;
+  fa.v_scale = kv->v_scale;
+  fa.pos = seq_lens;
+  fa.pos_from_len = 1;
+  fa.err = at<uint32_t>(ws, L.err);
+  if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  QUpArgs qa{};
+  qa.c_hat = fa.c_hat;
+  qa.w_qup = static_cast<const uint16_t*>(w_qup);
+  qa.batch = batch;
+  qa.q = static_cast<uint16_t*>(q_out);
+  if (launch_q_up(qa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  AttnArgs aa{};
+  aa.q = qa.q;
+  aa.kv = fa.kv;
+  aa.kv_dtype = kv->dtype;
+  aa.k_scale = kv->k_scale;
+  aa.v_scale = kv->v_scale;
+  aa.seq_lens = seq_lens;
+  aa.scale = scale;
+  aa.out = static_cast<uint16_t*>(out);
+  aa.batch = batch;
+  aa.partials = at<float>(ws, L.attn_part);
+  aa.counters = at<int32_t>(ws, L.counters);
+  aa.err = fa.err;
+  aa.grid = L.attn_grid;
+  return cuda_status(launch_attention(aa, s));
+}
+
+}  // extern "C"

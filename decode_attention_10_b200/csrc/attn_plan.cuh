@@ -1,0 +1,163 @@
+// Length-aware split plan of the decode attention, computed on chip by every CTA.
+//
+// The cached positions of all sequences are cut into tiles of kTile positions and laid end
+// to end (sequence 0's tiles, then sequence 1's, ...). CTA g of a persistent grid of G CTAs
+// (G capped at the tile count NT, so that no CTA of the plan is empty)
+// takes the contiguous tile range [bound(g), bound(g + 1)), bound(g) = floor(g * NT / G),
+// so every CTA streams the same number of KV bytes (to within one tile) whatever the mix
+// of lengths. The part of one sequence that falls in one CTA's range is a work item. A
+// sequence covered by a single CTA is finished in place; a sequence split over n > 1 CTAs
+// gets n partial slots (m, l, acc), and the last CTA to finish one of them merges all n.
+#pragma once
+
+#include "mfa_internal.cuh"
+
+namespace mfa {
+
+struct PlanSmem {
+  int32_t tile_start[kMaxBatch + 1];  // exclusive prefix of tiles per sequence
+  int32_t slot_base[kMaxBatch];       // exclusive prefix of partial slots per sequence
+  int32_t len[kMaxBatch];             // attended positions (0 for rejected sequences)
+  int32_t scan_tmp[33];
+  int32_t grid;  // CTAs that get work: min(G, total tiles), so none of them is empty
+  int32_t flag;
+};
+
+__device__ __forceinline__ int plan_bound(int g, int G, int NT) {
+  return static_cast<int>(static_cast<int64_t>(g) * NT / G);
+}
+
+// CTA owning tile t: the largest g with plan_bound(g) <= t.
+__device__ __forceinline__ int plan_cta_of(int t, int G, int NT) {
+  return static_cast<int>((static_cast<int64_t>(t + 1) * G - 1) / NT);
+}
+
+// Block-wide exclusive scan of v[0, n) in place; returns the total. Every thread of the
+// block must call it (blockDim.x a multiple of 32).
+__device__ inline int block_exclusive_scan(int32_t* v, int n, int32_t* tmp) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (n + nt - 1) / nt;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  int local = 0;
+  for (int i = lo; i < hi; ++i) local += v[i];
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nwarps ? tmp[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    if (lane < nwarps) tmp[lane] = wi - w;  // exclusive warp offsets
+    if (lane == 31) tmp[32] = wi;          // total
+  }
+  __syncthreads();
+  int run = tmp[warp] + incl - local;
+  for (int i = lo; i < hi; ++i) {
+    const int x = v[i];
+    v[i] = run;
+    run += x;
+  }
+  const int total = tmp[32];
+  __syncthreads();
+  return total;
+}
+
+// Build the plan for `batch` sequences over a grid of G CTAs. Lengths outside
+// [1, capacity] are rejected (length 0; the output is zero-filled) and, if `report`, flagged.
+__device__ inline void plan_build(PlanSmem& P, const int32_t* __restrict__ seq_lens,
+                                  const KvSeq* __restrict__ kv, int batch, int G,
+                                  uint32_t* err, bool report) {
+  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+    const int L = seq_lens[b];
+    const int cap = kv[b].capacity;
+    int len = L;
+    if (L <= 0) {
+      len = 0;
+      if (report) atomicOr(err, kErrEmpty);
+    } else if (L > cap) {
+      len = 0;
+      if (report) atomicOr(err, kErrCapacity);
+    }
+    P.len[b] = len;
+    P.tile_start[b] = (len + kTile - 1) / kTile;
+  }
+  __syncthreads();
+  const int NT = block_exclusive_scan(P.tile_start, batch, P.scan_tmp);
+  const int Ge = min(G, NT);
+  if (threadIdx.x == 0) {
+    P.tile_start[batch] = NT;
+    P.grid = Ge;
+  }
+  __syncthreads();
+  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
+    int slots = 0;
+    if (te > ts) {
+      const int n = plan_cta_of(te - 1, Ge, NT) - plan_cta_of(ts, Ge, NT) + 1;
+      slots = n > 1 ? n : 0;
+    }
+    P.slot_base[b] = slots;
+  }
+  __syncthreads();
+  block_exclusive_scan(P.slot_base, batch, P.scan_tmp);
+}
+
+struct WorkItem {
+  int b;        // sequence
+  int tok0;     // first cached position of the item
+  int tok1;     // one past the last
+  int slot;     // partial slot, or -1 if the sequence is finished by this item alone
+  int nsplit;   // CTAs sharing the sequence
+};
+
+// Call f(item) for every work item of CTA g, in order.
+template <class F>
+__device__ inline void plan_for_each_item(const PlanSmem& P, int batch, int g, F&& f) {
+  const int NT = P.tile_start[batch];
+  const int G = P.grid;
+  if (NT == 0 || g >= G) return;
+  const int t0 = plan_bound(g, G, NT), t1 = plan_bound(g + 1, G, NT);
+  if (t0 >= t1) return;
+  // largest b with tile_start[b] <= t0 (that sequence contains tile t0)
+  int lo = 0, hi = batch - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (P.tile_start[mid] <= t0) lo = mid; else hi = mid - 1;
+  }
+  for (int b = lo; b < batch && P.tile_start[b] < t1; ++b) {
+    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
+    if (te <= t0 || te == ts) continue;
+    const int a0 = max(ts, t0), a1 = min(te, t1);
+    WorkItem it;
+    it.b = b;
+    it.tok0 = (a0 - ts) * kTile;
+    it.tok1 = min(P.len[b], (a1 - ts) * kTile);
+    const int gf = plan_cta_of(ts, G, NT);
+    it.nsplit = plan_cta_of(te - 1, G, NT) - gf + 1;
+    it.slot = it.nsplit > 1 ? P.slot_base[b] + (g - gf) : -1;
+    f(it);
+  }
+}
+
+// Partial slot views.
+__device__ __forceinline__ float* partial_m(float* base, int slot) {
+  return base + (size_t)slot * kPartialFloats;
+}
+__device__ __forceinline__ float* partial_l(float* base, int slot) {
+  return base + (size_t)slot * kPartialFloats + kHeads;
+}
+__device__ __forceinline__ float* partial_acc(float* base, int slot) {
+  return base + (size_t)slot * kPartialFloats + 2 * kHeads;
+}
+
+}  // namespace mfa

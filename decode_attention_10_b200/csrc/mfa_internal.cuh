@@ -1,0 +1,139 @@
+// Internal definitions shared by the kernels and the C-ABI layer of libmfa.
+#pragma once
+
+#include <cuda.h>  // CUtensorMap (type only; the driver is reached through the runtime)
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/mfa.h"
+
+namespace mfa {
+
+// Layer dimensions (Step-3 pages: bud-325 "Key claims"/"Method", redeep architecture table).
+constexpr int kHidden = MFA_HIDDEN;     // 7168
+constexpr int kRank = MFA_Q_RANK;       // 2048
+constexpr int kHeads = MFA_N_HEADS;     // 64
+constexpr int kHeadDim = MFA_HEAD_DIM;  // 256
+constexpr int kQWidth = kHeads * kHeadDim;  // 16384
+constexpr int kMaxBatch = MFA_MAX_BATCH;
+
+// Columns of the hidden-state projection x [W_qdown | W_k | W_v]: 2048 + 256 + 256.
+constexpr int kXProjCols = kRank + 2 * kHeadDim;  // 2560
+constexpr int kXProjSplits = 7;                   // split-K of the 7168-long reduction
+constexpr int kXProjKPerSplit = kHidden / kXProjSplits;  // 1024
+static_assert(kHidden % kXProjSplits == 0, "split-K must divide the hidden width");
+
+// Attention work unit: the plan hands out whole tiles of this many cached positions.
+constexpr int kTile = 128;
+
+// Device-side error bits kept in the workspace header.
+enum : uint32_t { kErrCapacity = 1u, kErrEmpty = 2u, kErrTimeout = 4u };
+
+// One entry of the device KV table: TMA tensor maps of the sequence's K and V rows
+// ([capacity, 256] elements, row-major) plus the raw pointers and capacity.
+struct alignas(128) KvSeq {
+  CUtensorMap tmap_k;
+  CUtensorMap tmap_v;
+  void* k;
+  void* v;
+  int32_t capacity;
+  int32_t reserved[27];
+};
+static_assert(sizeof(KvSeq) == 384, "KvSeq layout");
+
+// Split-K partial of one attention work item: running max m (log2 domain) and sum l per
+// head, and the unnormalized accumulator acc[head][dim], all fp32.
+constexpr int kPartialFloats = kHeads + kHeads + kHeads * kHeadDim;  // 16512
+constexpr size_t kPartialBytes = kPartialFloats * sizeof(float);     // 66048 = 258 * 256
+
+struct WsLayout {
+  size_t err;          // uint32 error bits
+  size_t counters;     // int32 [kMaxBatch] arrival counters of the split-K merge
+  size_t attn_part;    // partial slots
+  size_t xproj_part;   // fp32 [kXProjSplits][batch][kXProjCols]
+  size_t c_hat;        // bf16 [batch][kRank]
+  size_t total;
+  int attn_slots;
+  int attn_grid;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Persistent attention grid: one CTA per SM.
+inline int attn_grid_for(int num_sms) { return num_sms; }
+
+inline WsLayout ws_layout(int batch, int num_sms) {
+  WsLayout L{};
+  size_t off = 0;
+  L.err = off;
+  off += 256;
+  L.counters = off;
+  off = align_up(off + sizeof(int32_t) * kMaxBatch, 256);
+  L.attn_grid = attn_grid_for(num_sms);
+  L.attn_slots = L.attn_grid + batch;  // sum over sequences of their splits <= grid + batch
+  L.attn_part = off;
+  off = align_up(off + kPartialBytes * (size_t)L.attn_slots, 256);
+  L.xproj_part = off;
+  off = align_up(off + sizeof(float) * kXProjSplits * (size_t)batch * kXProjCols, 256);
+  L.c_hat = off;
+  off = align_up(off + sizeof(uint16_t) * (size_t)batch * kRank, 256);
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------------------------------
+// Kernel launchers (defined in the .cu files); all return cudaGetLastError().
+// ---------------------------------------------------------------------------------------
+
+struct XProjArgs {
+  const uint16_t* x;     // [batch, 7168] bf16
+  const uint16_t* w[3];  // W_qdown [7168, 2048], W_k [7168, 256], W_v [7168, 256]
+  int batch;
+  int tile_begin, tile_end;  // 128-column tiles of the 2560 concatenated columns
+  float* part;               // [kXProjSplits][batch][2560]
+};
+cudaError_t launch_xproj(const XProjArgs& a, cudaStream_t s);
+
+struct FinishArgs {
+  const float* part;  // x-projection partials
+  int batch;
+  // query half: c_hat = bf16(rmsnorm(c) * gamma)
+  const uint16_t* gamma;  // null = skip the query half
+  float eps;
+  uint16_t* c_hat;  // [batch, 2048]
+  // K/V half: append bf16 / e4m3 rows
+  const KvSeq* kv;  // null = skip the K/V half
+  int kv_dtype;
+  float k_scale, v_scale;
+  const int32_t* pos;      // device [batch]: row to write
+  int pos_from_len;        // 1: row = pos[b] - 1 (pos holds seq_lens)
+  uint32_t* err;
+};
+cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s);
+
+struct QUpArgs {
+  const uint16_t* c_hat;  // [batch, 2048]
+  const uint16_t* w_qup;  // [2048, 16384]
+  int batch;
+  uint16_t* q;  // [batch, 16384]
+};
+cudaError_t launch_q_up(const QUpArgs& a, cudaStream_t s);
+
+struct AttnArgs {
+  const uint16_t* q;        // [batch, 64, 256] bf16
+  const KvSeq* kv;          // device table
+  int kv_dtype;
+  float k_scale, v_scale;   // FP8 only
+  const int32_t* seq_lens;  // device [batch]
+  float scale;              // softmax scale
+  uint16_t* out;            // [batch, 64, 256] bf16
+  int batch;
+  float* partials;          // slots
+  int32_t* counters;        // [batch]
+  uint32_t* err;
+  int grid;
+};
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+
+}  // namespace mfa

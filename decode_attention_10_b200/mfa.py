@@ -1,0 +1,222 @@
+"""Thin ctypes binding of libmfa.so (include/mfa.h): argument marshalling only.
+
+Every step of the decode path runs in the library's CUDA kernels; this module only turns
+torch tensors into pointers, picks the current CUDA stream, and raises on error statuses.
+There is no fallback: if the library is missing, the first call raises.
+"""
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmfa.so")
+
+HIDDEN, Q_RANK, N_HEADS, HEAD_DIM = 7168, 2048, 64, 256
+MAX_CONTEXT, MAX_BATCH = 65536, 1024
+KV_BF16, KV_FP8_E4M3 = 0, 1
+
+STATUS = {0: "MFA_OK", 1: "MFA_ERR_INVALID_ARG", 2: "MFA_ERR_UNSUPPORTED",
+          3: "MFA_ERR_CAPACITY", 4: "MFA_ERR_WORKSPACE", 5: "MFA_ERR_CUDA",
+          6: "MFA_ERR_EMPTY", 7: "MFA_ERR_TIMEOUT"}
+
+# name -> (restype, argtypes), mirroring include/mfa.h
+_P = ctypes.c_void_p
+_SIGNATURES = {
+    "mfa_version": (ctypes.c_int32, []),
+    "mfa_status_str": (ctypes.c_char_p, [ctypes.c_int32]),
+    "mfa_kv_table_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
+    "mfa_kv_table_init": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int32,
+                                         _P, _P, _P, _P]),
+    "mfa_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
+    "mfa_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
+    "mfa_get_error": (ctypes.c_int, [_P, _P]),
+    "mfa_query_proj": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_float, _P, ctypes.c_int32, _P,
+                                      ctypes.c_size_t, _P]),
+    "mfa_kv_append": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "mfa_decode_attn": (ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _P, ctypes.c_size_t,
+                                       _P]),
+    "mfa_decode_layer": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
+                                        ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+}
+
+
+class KvCacheDesc(ctypes.Structure):
+    """mfa_kv_cache."""
+    _fields_ = [("batch", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
+                ("table", ctypes.c_void_p)]
+
+
+class MfaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmfa.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m decode_attention_10_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MfaError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    return t.data_ptr()
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KV_BF16
+    if t.dtype in (torch.float8_e4m3fn, torch.uint8):
+        return KV_FP8_E4M3
+    raise ValueError(f"unsupported KV dtype {t.dtype}")
+
+
+class KVCache:
+    """A KV cache described to the library: per-sequence K and V row buffers
+    ([capacity_b, 256] CUDA tensors of bf16 or float8_e4m3fn) plus the device table.
+    Keeps references to the buffers so they outlive the table."""
+
+    def __init__(self, k: Sequence[torch.Tensor], v: Sequence[torch.Tensor],
+                 k_scale: float = 1.0, v_scale: float = 1.0,
+                 stream: Optional[torch.cuda.Stream] = None):
+        lib = load()
+        if len(k) != len(v) or not k:
+            raise ValueError("need the same nonzero number of K and V buffers")
+        self.k, self.v = list(k), list(v)
+        self.batch = len(k)
+        self.dtype = _dtype_code(k[0])
+        caps = []
+        for kt, vt in zip(self.k, self.v):
+            if _dtype_code(kt) != self.dtype or _dtype_code(vt) != self.dtype:
+                raise ValueError("mixed KV dtypes")
+            if kt.dim() != 2 or kt.shape[1] != HEAD_DIM or kt.shape != vt.shape:
+                raise ValueError("each K/V buffer must be [capacity, 256]")
+            _ptr(kt), _ptr(vt)
+            caps.append(int(kt.shape[0]))
+        self.capacity = caps
+        self.k_scale, self.v_scale = float(k_scale), float(v_scale)
+        dev = self.k[0].device
+        nbytes = lib.mfa_kv_table_bytes(self.batch)
+        if nbytes == 0:
+            raise ValueError(f"batch {self.batch} out of range")
+        self.table = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        arr = ctypes.c_void_p * self.batch
+        kp = arr(*[t.data_ptr() for t in self.k])
+        vp = arr(*[t.data_ptr() for t in self.v])
+        cp = (ctypes.c_int32 * self.batch)(*caps)
+        _check(lib.mfa_kv_table_init(self.table.data_ptr(), nbytes, self.batch, self.dtype,
+                                     ctypes.cast(kp, _P), ctypes.cast(vp, _P),
+                                     ctypes.cast(cp, _P), _stream(stream)),
+               "mfa_kv_table_init")
+        self.desc = KvCacheDesc(self.batch, self.dtype, self.k_scale, self.v_scale,
+                                self.table.data_ptr())
+
+
+class Workspace:
+    """Device workspace for `batch` sequences (allocated by torch, zeroed by the library)."""
+
+    def __init__(self, batch: int, device=None, stream: Optional[torch.cuda.Stream] = None):
+        lib = load()
+        self.batch = int(batch)
+        self.nbytes = lib.mfa_workspace_bytes(self.batch)
+        if self.nbytes == 0:
+            raise ValueError(f"batch {batch} out of range (or no CUDA device)")
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8,
+                               device=device if device is not None else "cuda")
+        _check(lib.mfa_workspace_init(self.buf.data_ptr(), self.nbytes, _stream(stream)),
+               "mfa_workspace_init")
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+
+def get_error(ws: Workspace, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronize the stream and return (and clear) the workspace's device status."""
+    return load().mfa_get_error(ws.ptr, _stream(stream))
+
+
+def query_proj(x, w_qdown, gamma, w_qup, eps: float = 1e-6, q_out=None, ws=None,
+               stream=None) -> torch.Tensor:
+    lib = load()
+    bsz = int(x.shape[0])
+    if q_out is None:
+        q_out = torch.empty(bsz, N_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=x.device)
+    ws = ws if ws is not None else Workspace(bsz, x.device)
+    _check(lib.mfa_query_proj(_ptr(x), _ptr(w_qdown), _ptr(gamma), _ptr(w_qup), float(eps),
+                              _ptr(q_out), bsz, ws.ptr, ws.nbytes, _stream(stream)),
+           "mfa_query_proj")
+    return q_out
+
+
+def kv_append(x, w_k, w_v, cache: KVCache, pos: torch.Tensor, ws=None, stream=None):
+    lib = load()
+    ws = ws if ws is not None else Workspace(cache.batch, x.device)
+    _check(lib.mfa_kv_append(_ptr(x), _ptr(w_k), _ptr(w_v), ctypes.byref(cache.desc),
+                             _ptr(pos), ws.ptr, ws.nbytes, _stream(stream)),
+           "mfa_kv_append")
+
+
+def decode_attn(q, cache: KVCache, seq_lens: torch.Tensor, scale: float = 1.0 / 16.0,
+                out=None, ws=None, stream=None) -> torch.Tensor:
+    lib = load()
+    if out is None:
+        out = torch.empty(cache.batch, N_HEADS, HEAD_DIM, dtype=torch.bfloat16,
+                          device=q.device)
+    ws = ws if ws is not None else Workspace(cache.batch, q.device)
+    _check(lib.mfa_decode_attn(_ptr(q), ctypes.byref(cache.desc), _ptr(seq_lens),
+                               float(scale), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)),
+           "mfa_decode_attn")
+    return out
+
+
+def decode_layer(x, w_qdown, gamma, w_qup, w_k, w_v, cache: KVCache, seq_lens,
+                 eps: float = 1e-6, scale: float = 1.0 / 16.0, q_out=None, out=None,
+                 ws=None, stream=None):
+    """One MFA decode step; returns (q, out)."""
+    lib = load()
+    bsz = cache.batch
+    if q_out is None:
+        q_out = torch.empty(bsz, N_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=x.device)
+    if out is None:
+        out = torch.empty(bsz, N_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=x.device)
+    ws = ws if ws is not None else Workspace(bsz, x.device)
+    _check(lib.mfa_decode_layer(_ptr(x), _ptr(w_qdown), _ptr(gamma), _ptr(w_qup), _ptr(w_k),
+                                _ptr(w_v), float(eps), ctypes.byref(cache.desc),
+                                _ptr(seq_lens), float(scale), _ptr(q_out), _ptr(out), ws.ptr,
+                                ws.nbytes, _stream(stream)),
+           "mfa_decode_layer")
+    return q_out, out

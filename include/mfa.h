@@ -1,0 +1,182 @@
+/*
+ * mfa.h -- C ABI of the B200 (sm_100a) decode step of Step-3's MFA attention layer.
+ *
+ * The layer (Step-3 pages: bud-325 summary, "Key claims" and "Method"; redeep.blog,
+ * "What's New" and the architecture table): for each token, the hidden vector x (7168) is
+ * projected down to a low-rank query of width 2048, normalized, and projected up to 64
+ * query heads of dimension 256. All 64 heads attend over ONE shared K head and ONE shared
+ * V head (dimension 256) kept in a per-sequence KV cache, which holds one K and one V
+ * vector per token; the new token's K and V are projected from x and appended.
+ *
+ * Readings taken where the pages are silent (stated once here, used by every call):
+ *   - "normalized" = RMSNorm over the 2048 values: c_hat = c / sqrt(mean(c^2) + eps) * gamma;
+ *   - k = x W_k, v = x W_v with W_k, W_v of shape [7168, 256]; no positional encoding;
+ *   - softmax scale is an argument (1/sqrt(256) = 1/16 for the layer);
+ *   - weights are row-major [in, out]; head h of q is columns [256 h, 256 h + 256);
+ *   - seq_lens[b] counts the positions attended AFTER the append; the new token is
+ *     written at row seq_lens[b] - 1 and attended to;
+ *   - FP8 caches store e4m3(value / scale), one float scale per tensor for K and for V;
+ *   - every rounding (fp32 -> bf16, fp32 -> e4m3) is to nearest, ties to even; e4m3
+ *     saturates to +-448.
+ *
+ * Conventions for every call:
+ *   - "device" pointers are CUDA global-memory addresses on the current device; "host"
+ *     pointers are ordinary CPU memory. All buffers are owned by the caller; the library
+ *     keeps no pointer after a call returns.
+ *   - bf16 buffers hold raw bfloat16 bit patterns (uint16_t). Every device buffer must
+ *     be 16-byte aligned; rows are dense (no padding) unless stated.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Compute calls only
+ *     enqueue work on it: they neither allocate nor synchronize, and may be captured in
+ *     a CUDA graph. Setup calls (mfa_kv_table_init, mfa_workspace_init) may synchronize.
+ *   - Problems visible on the host (null pointer, bad size, misalignment, workspace too
+ *     small, unsupported dtype) return an error status before anything is enqueued.
+ *     Problems visible only on the device (a length above a sequence's capacity, an empty
+ *     sequence, a bounded wait that expired) set a flag in the workspace and the affected
+ *     sequences' outputs are zero-filled; mfa_get_error reports and clears it.
+ *   - No call aborts, throws or prints.
+ */
+#ifndef MFA_H_
+#define MFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MFA_API __attribute__((visibility("default")))
+#else
+#define MFA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layer dimensions stated on the pages (bud-325 "Key claims"; redeep architecture table). */
+#define MFA_HIDDEN 7168      /* hidden width of x */
+#define MFA_Q_RANK 2048      /* low-rank query width */
+#define MFA_N_HEADS 64       /* query heads */
+#define MFA_HEAD_DIM 256     /* dimension of every query head and of the shared K and V head */
+#define MFA_MAX_CONTEXT 65536 /* longest context the model takes (redeep architecture table) */
+/* Library limit: sequences per call (the attention kernel plans the batch on chip). */
+#define MFA_MAX_BATCH 1024
+
+typedef enum {
+  MFA_OK = 0,
+  MFA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, size out of range, eps <= 0, ... */
+  MFA_ERR_UNSUPPORTED = 2, /* unknown KV dtype, or no sm_100 device */
+  MFA_ERR_CAPACITY = 3,    /* device: a length/position outside a sequence's capacity */
+  MFA_ERR_WORKSPACE = 4,   /* workspace or table buffer too small */
+  MFA_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed (launch error, ...) */
+  MFA_ERR_EMPTY = 6,       /* device: a sequence with seq_lens[b] == 0 in mfa_decode_attn */
+  MFA_ERR_TIMEOUT = 7      /* device: a bounded wait inside a kernel expired */
+} mfa_status;
+
+typedef enum {
+  MFA_KV_BF16 = 0,     /* cache rows are 256 bfloat16 values (512 bytes) */
+  MFA_KV_FP8_E4M3 = 1  /* cache rows are 256 OCP e4m3 codes (256 bytes) */
+} mfa_kv_dtype;
+
+/* Description of a KV cache of `batch` sequences, passed by pointer to the compute calls.
+ * `table` is the device table written by mfa_kv_table_init for the same batch and dtype. */
+typedef struct {
+  int32_t batch;
+  int32_t dtype;       /* mfa_kv_dtype */
+  float k_scale;       /* FP8 only: K rows hold e4m3(k / k_scale); must be > 0 */
+  float v_scale;       /* FP8 only: V rows hold e4m3(v / v_scale); must be > 0 */
+  const void* table;   /* device */
+} mfa_kv_cache;
+
+/* ---------------------------------------------------------------------------------------
+ * Setup
+ * ------------------------------------------------------------------------------------- */
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+MFA_API int32_t mfa_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+MFA_API const char* mfa_status_str(int32_t status);
+
+/* Bytes of the device KV table for `batch` sequences (0 if batch is out of range). */
+MFA_API size_t mfa_kv_table_bytes(int32_t batch);
+
+/* Describe a KV cache to the library. For each sequence b: k_ptrs[b] and v_ptrs[b] are
+ * device base addresses of its K and V rows, each [capacity[b], 256] elements of `dtype`,
+ * row-major, 16-byte aligned (sequences may live in separate allocations or be slices of
+ * one [B, L, 256] buffer). k_ptrs, v_ptrs and capacity are HOST arrays of length `batch`;
+ * 1 <= capacity[b] <= MFA_MAX_CONTEXT.
+ * `table` is a DEVICE buffer of at least mfa_kv_table_bytes(batch) bytes, 128-byte
+ * aligned. The call encodes one TMA tensor map per K and V buffer on the host, copies the
+ * table to `table` on `stream` and waits for that copy. Call it again whenever a
+ * sequence's buffer moves or grows. Errors: INVALID_ARG, WORKSPACE (table too small),
+ * UNSUPPORTED (dtype), CUDA (no device / driver entry point / copy failure). */
+MFA_API mfa_status mfa_kv_table_init(void* table, size_t table_bytes, int32_t batch, int32_t dtype,
+                             void* const* k_ptrs, void* const* v_ptrs,
+                             const int32_t* capacity, void* stream);
+
+/* Bytes of the workspace the compute calls need for `batch` sequences on the current
+ * device (0 if batch is out of range). One workspace must not be used by two calls that
+ * can run at the same time. */
+MFA_API size_t mfa_workspace_bytes(int32_t batch);
+
+/* Zero a freshly allocated workspace (device buffer, 256-byte aligned) on `stream` and
+ * wait. Needed once per allocation: the compute calls leave it ready for the next call. */
+MFA_API mfa_status mfa_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Wait for `stream`, then report and clear the device-side error flags of `ws`:
+ * MFA_OK, MFA_ERR_CAPACITY, MFA_ERR_EMPTY or MFA_ERR_TIMEOUT (the first set, in that
+ * order), or MFA_ERR_CUDA if the stream reports an error. */
+MFA_API mfa_status mfa_get_error(void* ws, void* stream);
+
+/* ---------------------------------------------------------------------------------------
+ * Compute (asynchronous on `stream`)
+ * ------------------------------------------------------------------------------------- */
+
+/* MFA query path (pages: bud-325 "Method" -- down-projection 7168 -> 2048, normalization,
+ * up-projection to 64 heads x 256):
+ *   c = x W_qdown (fp32 accumulation); c_hat = bf16(c / sqrt(mean(c^2) + eps) * gamma);
+ *   q = bf16(c_hat W_qup), written as q_out[b][h][j] = q[b][256 h + j].
+ * x: device bf16 [batch, 7168]; w_qdown: device bf16 [7168, 2048]; gamma: device bf16
+ * [2048]; w_qup: device bf16 [2048, 16384]; q_out: device bf16 [batch, 64, 256].
+ * 1 <= batch <= MFA_MAX_BATCH; eps > 0 (1e-6 for the layer).
+ * ws: device workspace of mfa_workspace_bytes(batch) bytes (initialized once). */
+MFA_API mfa_status mfa_query_proj(const void* x, const void* w_qdown, const void* gamma,
+                          const void* w_qup, float eps, void* q_out, int32_t batch,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Shared K/V head projection and cache append (pages: bud-325 "Method" -- one K and one
+ * V per token, shared by all query heads):
+ *   k = x W_k, v = x W_v (fp32 accumulation), stored as bf16(k) / bf16(v), or as
+ *   e4m3(k / k_scale) / e4m3(v / v_scale), at row pos[b] of sequence b.
+ * x: device bf16 [kv->batch, 7168]; w_k, w_v: device bf16 [7168, 256]; pos: device int32
+ * [kv->batch]. A position outside [0, capacity[b]) writes nothing for that sequence and
+ * sets MFA_ERR_CAPACITY in the workspace. Only the row pos[b] of each cache is written. */
+MFA_API mfa_status mfa_kv_append(const void* x, const void* w_k, const void* w_v,
+                         const mfa_kv_cache* kv, const int32_t* pos, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/* Decode attention of the 64 query heads over the shared K/V head (pages: bud-325
+ * "Method"; the cost is max(attention compute, KV memory access)):
+ *   out[b][h] = sum_{j < L_b} softmax_j(scale * q[b][h] . K_b[j]) V_b[j],  L_b = seq_lens[b],
+ * with K_b, V_b the cache rows (e4m3 codes times their scale for FP8 caches).
+ * q: device bf16 [kv->batch, 64, 256]; seq_lens: device int32 [kv->batch]; out: device
+ * bf16 [kv->batch, 64, 256]; scale > 0 (1/16 for the layer). The work is split over the
+ * GPU's SMs by length (split-K over the cache, merged in the same kernel). A sequence with
+ * L_b == 0 or L_b > capacity[b] gets a zero output and sets MFA_ERR_EMPTY /
+ * MFA_ERR_CAPACITY in the workspace. */
+MFA_API mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t* seq_lens,
+                           float scale, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* One whole MFA decode step: mfa_query_proj, then mfa_kv_append at row seq_lens[b] - 1,
+ * then mfa_decode_attn over seq_lens[b] rows -- in that order, on `stream`.
+ * Arguments as in those calls; q_out (device bf16 [batch, 64, 256]) receives q.
+ * The library does not advance seq_lens: that is the caller's bookkeeping. */
+MFA_API mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamma,
+                            const void* w_qup, const void* w_k, const void* w_v, float eps,
+                            const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
+                            void* q_out, void* out, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MFA_H_ */

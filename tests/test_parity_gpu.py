@@ -1,0 +1,276 @@
+"""GPU parity of the CUDA path (called through the C ABI) against the float64 oracle on the
+same seeded inputs: per op (the oracle reads the GPU-visible inputs of that op) and end to
+end (the oracle's own chain), small cases spanning several tiles and ragged tails, edge
+lengths, forced split-K, device-side error paths, and the five named workloads (sampled
+sequences at full size)."""
+
+import numpy as np
+import pytest
+import torch
+
+from decode_attention_10_b200 import workloads as W
+from oracle import codecs
+from oracle import mfa as omfa
+
+from mfa_util import (GpuStep, assert_close, bf16_np, codes_np, max_abs, oracle_dtype,
+                      oracle_weights, rel_l2)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from decode_attention_10_b200 import build, mfa
+    build.build()
+    mfa.load()
+
+
+def _q_close(q_gpu, q_ref):
+    # q is stored as bf16 on both sides; allow two bf16 ulps of the reference value plus a
+    # small absolute slack for values whose normalized input rounded differently
+    ulp = np.ldexp(1.0, np.frexp(np.abs(q_ref))[1] - 8)
+    bad = np.abs(q_gpu - q_ref) > 2 * ulp + 1e-3
+    assert not bad.any(), f"{bad.sum()} q elements off, max {max_abs(q_gpu, q_ref):.3e}"
+    assert rel_l2(q_gpu, q_ref) <= 1e-3
+
+
+def _check_layer(inp: W.Inputs, sample=None, e2e=True):
+    step = GpuStep(inp)
+    k_before = [codes_np(t) for t in step.k]
+    v_before = [codes_np(t) for t in step.v]
+    q_gpu, out_gpu = step.layer()
+    torch.cuda.synchronize()
+    from decode_attention_10_b200 import mfa
+    assert mfa.get_error(step.ws) == 0
+    bsz = inp.batch
+    seqs = list(range(bsz)) if sample is None else sample
+    lens = inp.seq_lens.tolist()
+    od = oracle_dtype(inp.kv_dtype)
+    ow = oracle_weights(inp)
+    xs = ow["x"][seqs]
+    # query path
+    _, q_ref = omfa.query_proj(xs, ow["w_qdown"], ow["gamma"], ow["w_qup"])
+    q_np = bf16_np(q_gpu)[seqs]
+    _q_close(q_np, q_ref)
+    # appended rows: one code apart at most (fp32 vs float64 rounding decision); every
+    # other byte of the cache unchanged
+    k_new, v_new = omfa.kv_project(xs, ow["w_k"], ow["w_v"])
+    k_codes = omfa.kv_store(k_new, od, inp.k_scale)
+    v_codes = omfa.kv_store(v_new, od, inp.v_scale)
+    k_after = {b: codes_np(step.k[b]) for b in seqs}
+    v_after = {b: codes_np(step.v[b]) for b in seqs}
+    for i, b in enumerate(seqs):
+        row = lens[b] - 1
+        for after, before, want in ((k_after[b], k_before[b], k_codes[i]),
+                                    (v_after[b], v_before[b], v_codes[i])):
+            rest = np.ones(after.shape[0], bool)
+            rest[row] = False
+            assert np.array_equal(after[rest], before[rest]), f"seq {b}: other rows changed"
+            got = after[row].astype(np.int64)
+            diff = np.abs(got - want.astype(np.int64))
+            assert diff.max() <= 1, f"seq {b}: appended row differs by {diff.max()} codes"
+            assert (diff != 0).mean() < 0.01
+    # attention, per op: the oracle reads the GPU's q and the GPU's cache after the append
+    out_np = bf16_np(out_gpu)[seqs]
+    k_list = [k_after[b] for b in seqs]
+    v_list = [v_after[b] for b in seqs]
+    ref = omfa.decode_attn(q_np, k_list, v_list, [lens[b] for b in seqs], od, inp.k_scale,
+                           inp.v_scale)
+    res = assert_close(out_np, ref, inp.kv_dtype, "attention (per op)")
+    if e2e:
+        # end to end: the oracle's own chain from x, weights and the original cache
+        kc = [k_before[b] for b in seqs]
+        vc = [v_before[b] for b in seqs]
+        full = omfa.decode_layer(xs, ow["w_qdown"], ow["gamma"], ow["w_qup"], ow["w_k"],
+                                 ow["w_v"], kc, vc, [lens[b] for b in seqs], od, inp.k_scale,
+                                 inp.v_scale)
+        assert_close(out_np, full["out"], inp.kv_dtype, "layer (end to end)")
+    return res
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_layer_small_ragged(kv_dtype):
+    # lengths span one and several 128-position tiles with ragged tails
+    inp = W.generate([1, 130, 300, 129, 128, 2], kv_dtype, seed=11)
+    _check_layer(inp)
+
+
+def test_layer_per_sequence_buffers_with_spare_capacity():
+    lens = [77, 513, 1]
+    caps = [100, 600, 9]
+    inp = W.generate(lens, W.KV_BF16, seed=12, contiguous=False, capacity=caps)
+    _check_layer(inp)
+
+
+def _attn_case(lens, kv_dtype, seed, caps=None, nan_tail=False, q_scale=1.0):
+    from decode_attention_10_b200 import mfa
+    inp = W.generate(lens, kv_dtype, seed=seed, contiguous=False, capacity=caps)
+    g = torch.Generator().manual_seed(seed + 7)
+    q = (torch.randn(len(lens), 64, 256, generator=g) * q_scale).to(torch.bfloat16)
+    k = [t.clone() for t in inp.k_cache]
+    v = [t.clone() for t in inp.v_cache]
+    if nan_tail:  # rows past the length hold NaN patterns: they must not leak into out
+        for kt, vt, n in zip(k, v, lens):
+            kt.view(torch.uint8)[n:] = 0x7F if kv_dtype == W.KV_FP8 else 0xFF
+            vt.view(torch.uint8)[n:] = 0x7F if kv_dtype == W.KV_FP8 else 0xFF
+    kd = [t.cuda() for t in k]
+    vd = [t.cuda() for t in v]
+    cache = mfa.KVCache(kd, vd, inp.k_scale, inp.v_scale)
+    out = mfa.decode_attn(q.cuda(), cache, inp.seq_lens.cuda())
+    torch.cuda.synchronize()
+    ref = omfa.decode_attn(bf16_np(q), [codes_np(t) for t in k], [codes_np(t) for t in v],
+                           lens, oracle_dtype(kv_dtype), inp.k_scale, inp.v_scale)
+    return bf16_np(out), ref, cache
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_attention_edge_lengths(kv_dtype):
+    lens = [1, 2, 63, 64, 65, 127, 128, 129, 255, 256, 257, 1000]
+    out, ref, _ = _attn_case(lens, kv_dtype, seed=21)
+    assert_close(out, ref, kv_dtype, "edge lengths")
+    # L = 1: the output is exactly the single cached V row, for every head
+    assert np.array_equal(out[0], np.repeat(ref[0][:1], 64, axis=0))
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_attention_rows_past_length_are_ignored(kv_dtype):
+    lens = [5, 130, 300]
+    caps = [64, 256, 512]
+    out, ref, _ = _attn_case(lens, kv_dtype, seed=22, caps=caps, nan_tail=True)
+    assert np.isfinite(out).all()
+    assert_close(out, ref, kv_dtype, "NaN past length")
+
+
+def test_attention_long_sequence_split_over_many_ctas():
+    # one 40,000-position sequence spans ~313 tiles, more than one per SM: split-K + merge
+    out, ref, _ = _attn_case([40000], W.KV_BF16, seed=23)
+    assert_close(out, ref, W.KV_BF16, "long single sequence")
+    out, ref, _ = _attn_case([65536, 3, 20000], W.KV_BF16, seed=24)
+    assert_close(out, ref, W.KV_BF16, "mixed long")
+
+
+def test_attention_sharp_softmax():
+    # large scores: the running max changes often and by a lot
+    out, ref, _ = _attn_case([3000, 700], W.KV_BF16, seed=25, q_scale=12.0)
+    assert_close(out, ref, W.KV_BF16, "sharp softmax")
+
+
+def test_attention_split_invariance():
+    # the same sequence alone, and batched with others (so it is split differently),
+    # gives the same output up to fp32 rounding of the merge
+    from decode_attention_10_b200 import mfa
+    inp = W.generate([9000, 300, 20000], W.KV_BF16, seed=26, contiguous=False)
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(3, 64, 256, generator=g).to(torch.bfloat16).cuda()
+    kd = [t.cuda() for t in inp.k_cache]
+    vd = [t.cuda() for t in inp.v_cache]
+    full = mfa.decode_attn(q, mfa.KVCache(kd, vd), inp.seq_lens.cuda())
+    alone = mfa.decode_attn(q[:1].contiguous(), mfa.KVCache(kd[:1], vd[:1]),
+                            inp.seq_lens[:1].cuda())
+    a, b = bf16_np(full[:1]), bf16_np(alone)
+    assert rel_l2(a, b) < 2e-3 and max_abs(a, b) < 2e-3
+
+
+def test_device_errors_zero_fill_and_report():
+    from decode_attention_10_b200 import mfa
+    inp = W.generate([50, 60, 70], W.KV_BF16, seed=27, contiguous=False)
+    kd = [t.cuda() for t in inp.k_cache]
+    vd = [t.cuda() for t in inp.v_cache]
+    cache = mfa.KVCache(kd, vd)
+    ws = mfa.Workspace(3)
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(3, 64, 256, generator=g).to(torch.bfloat16).cuda()
+    lens = torch.tensor([50, 61, 70], dtype=torch.int32).cuda()  # 61 > capacity 60
+    out = mfa.decode_attn(q, cache, lens, ws=ws)
+    assert mfa.get_error(ws) == 3  # MFA_ERR_CAPACITY
+    assert mfa.get_error(ws) == 0  # cleared
+    assert (out[1].float() == 0).all()
+    ref = omfa.decode_attn(bf16_np(q), [codes_np(t) for t in inp.k_cache],
+                           [codes_np(t) for t in inp.v_cache], [50, 60, 70])
+    o = bf16_np(out)
+    assert_close(o[[0, 2]], ref[[0, 2]], what="healthy sequences")
+    lens = torch.tensor([50, 0, 70], dtype=torch.int32).cuda()
+    out = mfa.decode_attn(q, cache, lens, ws=ws)
+    assert mfa.get_error(ws) == 6  # MFA_ERR_EMPTY
+    assert (out[1].float() == 0).all()
+    # append at a row past the capacity: nothing written, flagged
+    before = [codes_np(t) for t in kd]
+    pos = torch.tensor([0, 60, 3], dtype=torch.int32).cuda()
+    mfa.kv_append(inp.x.cuda(), inp.w_k.cuda(), inp.w_v.cuda(), cache, pos, ws=ws)
+    assert mfa.get_error(ws) == 3
+    after = [codes_np(t) for t in kd]
+    assert np.array_equal(after[1], before[1])
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_kv_append_bit_exact(kv_dtype):
+    """One-hot W makes k and v exact copies of chosen elements of x; with values on the
+    cache grid (and a power-of-two FP8 scale) the stored bytes are known exactly."""
+    from decode_attention_10_b200 import mfa
+    bsz, caps = 5, [3, 8, 1, 130, 64]
+    rng = np.random.default_rng(3)
+    fp8 = kv_dtype == W.KV_FP8
+    k_scale, v_scale = (0.5, 0.25) if fp8 else (1.0, 1.0)
+    if fp8:
+        grid = codecs.e4m3_decode(np.arange(0, 0x7F))
+        xv = rng.choice(grid, (bsz, 7168)) * rng.choice([-1.0, 1.0], (bsz, 7168)) * 0.25
+    else:
+        xv = codecs.bf16_round(rng.standard_normal((bsz, 7168)))
+    x = torch.from_numpy(codecs.bf16_encode(xv).view(np.int16)).view(torch.bfloat16)
+    pk, pv = rng.permutation(7168)[:256], rng.permutation(7168)[:256]
+    wk = torch.zeros(7168, 256)
+    wv = torch.zeros(7168, 256)
+    wk[pk, np.arange(256)] = 1.0
+    wv[pv, np.arange(256)] = 2.0
+    dt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    k = [torch.zeros(c, 256).to(dt).cuda() for c in caps]
+    v = [torch.zeros(c, 256).to(dt).cuda() for c in caps]
+    for t in k + v:
+        t.view(torch.uint8).fill_(0x5A)  # canary bytes
+    cache = mfa.KVCache(k, v, k_scale, v_scale)
+    pos = [2, 7, 0, 129, 31]
+    mfa.kv_append(x.cuda(), wk.to(torch.bfloat16).cuda(), wv.to(torch.bfloat16).cuda(), cache,
+                  torch.tensor(pos, dtype=torch.int32).cuda())
+    torch.cuda.synchronize()
+    od = oracle_dtype(kv_dtype)
+    kexp = omfa.kv_store(xv[:, pk], od, k_scale)
+    vexp = omfa.kv_store(2.0 * xv[:, pv], od, v_scale)
+    for b in range(bsz):
+        kb, vb = codes_np(k[b]), codes_np(v[b])
+        assert np.array_equal(kb[pos[b]], kexp[b]) and np.array_equal(vb[pos[b]], vexp[b])
+        rest = np.ones(caps[b], bool)
+        rest[pos[b]] = False
+        canary = 0x5A5A if not fp8 else 0x5A
+        assert (kb[rest] == canary).all() and (vb[rest] == canary).all()
+
+
+def test_query_proj_matches_oracle():
+    from decode_attention_10_b200 import mfa
+    inp = W.generate([1] * 37, W.KV_BF16, seed=31)  # a batch that is not a tile multiple
+    q = mfa.query_proj(inp.x.cuda(), inp.w_qdown.cuda(), inp.gamma.cuda(), inp.w_qup.cuda())
+    torch.cuda.synchronize()
+    ow = oracle_weights(inp)
+    _, q_ref = omfa.query_proj(ow["x"], ow["w_qdown"], ow["gamma"], ow["w_qup"])
+    _q_close(bf16_np(q), q_ref)
+
+
+def test_query_proj_nonunit_gamma_and_scaled_input():
+    from decode_attention_10_b200 import mfa
+    inp = W.generate([1] * 3, W.KV_BF16, seed=32, x_scale=1e-3)
+    g = torch.Generator().manual_seed(1)
+    gamma = (0.5 + torch.rand(2048, generator=g)).to(torch.bfloat16)
+    q = mfa.query_proj(inp.x.cuda(), inp.w_qdown.cuda(), gamma.cuda(), inp.w_qup.cuda())
+    torch.cuda.synchronize()
+    ow = oracle_weights(inp)
+    _, q_ref = omfa.query_proj(ow["x"], ow["w_qdown"], bf16_np(gamma), ow["w_qup"])
+    _q_close(bf16_np(q), q_ref)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("index", [0, 1, 2, 3, 4])
+def test_named_workload_sampled(index):
+    w = W.workload(index)
+    inp = W.generate_workload(w)
+    b = inp.batch
+    sample = sorted(set([0, b // 3, b // 2, b - 1]))
+    _check_layer(inp, sample=sample, e2e=True)
