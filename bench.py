@@ -410,7 +410,7 @@ def main():
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        res = run_ours(args, wl, rank, world)
+        res = run_ours(args, wl, rank, world, local)
     finally:
         if world > 1:
             import torch

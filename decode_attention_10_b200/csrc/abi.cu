@@ -29,39 +29,12 @@ bool device_sms(int* sms) {
   return true;
 }
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn != nullptr) return fn;
-  void* p = nullptr;
-  cudaDriverEntryPointQueryResult q{};
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-          cudaSuccess ||
-      q != cudaDriverEntryPointSuccess || p == nullptr)
-    return nullptr;
-  fn = reinterpret_cast<EncodeTiledFn>(p);
-  return fn;
-}
-
 // Tensor map over one sequence's cache rows: [rows, 256] elements, boxes of
 // (128 bytes of a row) x kTile rows, 128-byte swizzle -- the canonical K-major /
 // MN-major shared-memory layout of the tensor-core operands.
-bool encode_rows(EncodeTiledFn enc, CUtensorMap* m, void* base, int rows, int dtype) {
-  const bool fp8 = dtype == MFA_KV_FP8_E4M3;
-  const cuuint64_t elem = fp8 ? 1 : 2;
-  cuuint64_t dims[2] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {kHeadDim * elem};
-  cuuint32_t box[2] = {(cuuint32_t)(128 / elem), (cuuint32_t)kTile};
-  cuuint32_t estr[2] = {1, 1};
-  const CUresult r =
-      enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base,
-          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+bool encode_rows(CUtensorMap* m, void* base, int rows, int dtype) {
+  const int elem = dtype == MFA_KV_FP8_E4M3 ? 1 : 2;
+  return encode_2d(m, base, (uint64_t)rows, kHeadDim, elem, 128 / elem, kTile);
 }
 
 mfa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MFA_OK : MFA_ERR_CUDA; }
@@ -121,6 +94,51 @@ mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
 }
 
 }  // namespace
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn != nullptr) return fn;
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || p == nullptr)
+    return nullptr;
+  fn = reinterpret_cast<EncodeTiledFn>(p);
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int elem_bytes,
+               uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(cols * elem_bytes)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(
+      m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+
+// The attention of one call: the tensor-core kernel for bf16 caches, the CUDA-core one
+// for FP8 caches.
+mfa_status run_attention(const AttnArgs& aa, cudaStream_t s) {
+  if (aa.kv_dtype == MFA_KV_BF16) {
+    CUtensorMap q_map;
+    if (!encode_2d(&q_map, aa.q, (uint64_t)aa.batch * kHeads, kHeadDim, 2, 64, 64))
+      return MFA_ERR_CUDA;
+    return cuda_status(launch_attention_tc(q_map, aa, s));
+  }
+  return cuda_status(launch_attention(aa, s));
+}
+
+}  // namespace
 }  // namespace mfa
 
 using namespace mfa;
@@ -162,13 +180,12 @@ mfa_status mfa_kv_table_init(void* table, size_t table_bytes, int32_t batch, int
     if (!aligned16(k_ptrs[b]) || !aligned16(v_ptrs[b])) return MFA_ERR_INVALID_ARG;
     if (capacity[b] < 1 || capacity[b] > MFA_MAX_CONTEXT) return MFA_ERR_INVALID_ARG;
   }
-  EncodeTiledFn enc = encode_tiled_fn();
-  if (enc == nullptr) return MFA_ERR_CUDA;
+  if (encode_tiled_fn() == nullptr) return MFA_ERR_CUDA;
   std::vector<KvSeq> host(batch);
   std::memset(host.data(), 0, sizeof(KvSeq) * batch);
   for (int b = 0; b < batch; ++b) {
-    if (!encode_rows(enc, &host[b].tmap_k, k_ptrs[b], capacity[b], dtype) ||
-        !encode_rows(enc, &host[b].tmap_v, v_ptrs[b], capacity[b], dtype))
+    if (!encode_rows(&host[b].tmap_k, k_ptrs[b], capacity[b], dtype) ||
+        !encode_rows(&host[b].tmap_v, v_ptrs[b], capacity[b], dtype))
       return MFA_ERR_INVALID_ARG;
     host[b].k = k_ptrs[b];
     host[b].v = v_ptrs[b];
@@ -286,7 +303,7 @@ mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t*
   aa.counters = at<int32_t>(ws, L.counters);
   aa.err = at<uint32_t>(ws, L.err);
   aa.grid = L.attn_grid;
-  return cuda_status(launch_attention(aa, static_cast<cudaStream_t>(stream)));
+  return run_attention(aa, static_cast<cudaStream_t>(stream));
 }
 
 mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamma,
@@ -350,7 +367,7 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   aa.counters = at<int32_t>(ws, L.counters);
   aa.err = fa.err;
   aa.grid = L.attn_grid;
-  return cuda_status(launch_attention(aa, s));
+  return run_attention(aa, s);
 }
 
 }  // extern "C"

