@@ -63,34 +63,67 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// x [batch, 7168] onto the 128-column tiles [tile_begin, tile_end) of [W_qdown | W_k | W_v]
+// (16 + 2 + 2 tiles), split-K partials into the workspace. Null weights are not read.
+mfa_status run_xproj(const void* x, const void* w_qdown, const void* w_k, const void* w_v,
+                     int batch, int tile_begin, int tile_end, float* part, uint32_t* err,
+                     cudaStream_t s) {
+  CUtensorMap wm[3];
+  std::memset(wm, 0, sizeof(wm));
+  if (w_qdown && !encode_2d(&wm[0], w_qdown, kHidden, kRank, 2, 64, 64)) return MFA_ERR_CUDA;
+  if (w_k && !encode_2d(&wm[1], w_k, kHidden, kHeadDim, 2, 64, 64)) return MFA_ERR_CUDA;
+  if (w_v && !encode_2d(&wm[2], w_v, kHidden, kHeadDim, 2, 64, 64)) return MFA_ERR_CUDA;
+  CUtensorMap xm;
+  if (!encode_2d(&xm, x, (uint64_t)batch, kHidden, 2, 64, wgemm_n_box(batch))) return MFA_ERR_CUDA;
+  WGemmArgs p{};
+  p.batch = batch;
+  p.tile_begin = tile_begin;
+  p.three_weights = 1;
+  p.w0_tiles = kRank / 128;
+  p.w1_tiles = kHeadDim / 128;
+  p.kblocks_per_cta = kXProjKPerSplit / 64;
+  p.out_f32 = part;
+  p.out_ld = kXProjCols;
+  p.err = err;
+  return cuda_status(launch_wgemm(wm, xm, p, tile_end - tile_begin, kXProjSplits, s));
+}
+
+// q = bf16(c_hat W_qup): c_hat [batch, 2048], W_qup [2048, 16384], q [batch, 16384].
+mfa_status run_q_up(const uint16_t* c_hat, const void* w_qup, void* q, int batch, uint32_t* err,
+                    cudaStream_t s) {
+  CUtensorMap wm[3];
+  std::memset(wm, 0, sizeof(wm));
+  if (!encode_2d(&wm[0], w_qup, kRank, kQWidth, 2, 64, 64)) return MFA_ERR_CUDA;
+  CUtensorMap xm;
+  if (!encode_2d(&xm, c_hat, (uint64_t)batch, kRank, 2, 64, wgemm_n_box(batch)))
+    return MFA_ERR_CUDA;
+  WGemmArgs p{};
+  p.batch = batch;
+  p.tile_begin = 0;
+  p.three_weights = 0;
+  p.kblocks_per_cta = kRank / 64;
+  p.out_bf16 = static_cast<uint16_t*>(q);
+  p.out_ld = kQWidth;
+  p.err = err;
+  return cuda_status(launch_wgemm(wm, xm, p, kQWidth / 128, 1, s));
+}
+
 mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
                           const void* w_qup, float eps, void* q_out, int batch, void* ws,
                           const WsLayout& L, cudaStream_t s) {
-  XProjArgs xa{};
-  xa.x = static_cast<const uint16_t*>(x);
-  xa.w[0] = static_cast<const uint16_t*>(w_qdown);
-  xa.w[1] = xa.w[2] = nullptr;
-  xa.batch = batch;
-  xa.tile_begin = 0;
-  xa.tile_end = kRank / 128;
-  xa.part = at<float>(ws, L.xproj_part);
-  cudaError_t e = launch_xproj(xa, s);
-  if (e != cudaSuccess) return MFA_ERR_CUDA;
+  float* part = at<float>(ws, L.xproj_part);
+  uint32_t* err = at<uint32_t>(ws, L.err);
+  mfa_status st = run_xproj(x, w_qdown, nullptr, nullptr, batch, 0, kRank / 128, part, err, s);
+  if (st != MFA_OK) return st;
   FinishArgs fa{};
-  fa.part = xa.part;
+  fa.part = part;
   fa.batch = batch;
   fa.gamma = static_cast<const uint16_t*>(gamma);
   fa.eps = eps;
   fa.c_hat = at<uint16_t>(ws, L.c_hat);
-  fa.err = at<uint32_t>(ws, L.err);
-  e = launch_xproj_finish(fa, s);
-  if (e != cudaSuccess) return MFA_ERR_CUDA;
-  QUpArgs qa{};
-  qa.c_hat = fa.c_hat;
-  qa.w_qup = static_cast<const uint16_t*>(w_qup);
-  qa.batch = batch;
-  qa.q = static_cast<uint16_t*>(q_out);
-  return cuda_status(launch_q_up(qa, s));
+  fa.err = err;
+  if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  return run_q_up(fa.c_hat, w_qup, q_out, batch, err, s);
 }
 
 }  // namespace
@@ -255,18 +288,12 @@ mfa_status mfa_kv_append(const void* x, const void* w_k, const void* w_v,
   st = check_ws(ws, ws_bytes, kv->batch, &L);
   if (st != MFA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  XProjArgs xa{};
-  xa.x = static_cast<const uint16_t*>(x);
-  xa.w[0] = nullptr;
-  xa.w[1] = static_cast<const uint16_t*>(w_k);
-  xa.w[2] = static_cast<const uint16_t*>(w_v);
-  xa.batch = kv->batch;
-  xa.tile_begin = kRank / 128;
-  xa.tile_end = kXProjCols / 128;
-  xa.part = at<float>(ws, L.xproj_part);
-  if (launch_xproj(xa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  float* part = at<float>(ws, L.xproj_part);
+  st = run_xproj(x, nullptr, w_k, w_v, kv->batch, kRank / 128, kXProjCols / 128, part,
+                 at<uint32_t>(ws, L.err), s);
+  if (st != MFA_OK) return st;
   FinishArgs fa{};
-  fa.part = xa.part;
+  fa.part = part;
   fa.batch = kv->batch;
   fa.kv = static_cast<const KvSeq*>(kv->table);
   fa.kv_dtype = kv->dtype;
@@ -322,19 +349,13 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int batch = kv->batch;
   // one projection of x onto [W_qdown | W_k | W_v]
-  XProjArgs xa{};
-  xa.x = static_cast<const uint16_t*>(x);
-  xa.w[0] = static_cast<const uint16_t*>(w_qdown);
-  xa.w[1] = static_cast<const uint16_t*>(w_k);
-  xa.w[2] = static_cast<const uint16_t*>(w_v);
-  xa.batch = batch;
-  xa.tile_begin = 0;
-  xa.tile_end = kXProjCols / 128;
-  xa.part = at<float>(ws, L.xproj_part);
-  if (launch_xproj(xa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  float* part = at<float>(ws, L.xproj_part);
+  st = run_xproj(x, w_qdown, w_k, w_v, batch, 0, kXProjCols / 128, part,
+                 at<uint32_t>(ws, L.err), s);
+  if (st != MFA_OK) return st;
   // split-K sums, RMSNorm of the query half, K/V append at row seq_lens[b] - 1
   FinishArgs fa{};
-  fa.part = xa.part;
+  fa.part = part;
   fa.batch = batch;
   fa.gamma = static_cast<const uint16_t*>(gamma);
   fa.eps = eps;
@@ -347,14 +368,10 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   fa.pos_from_len = 1;
   fa.err = at<uint32_t>(ws, L.err);
   if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
-  QUpArgs qa{};
-  qa.c_hat = fa.c_hat;
-  qa.w_qup = static_cast<const uint16_t*>(w_qup);
-  qa.batch = batch;
-  qa.q = static_cast<uint16_t*>(q_out);
-  if (launch_q_up(qa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  st = run_q_up(fa.c_hat, w_qup, q_out, batch, fa.err, s);
+  if (st != MFA_OK) return st;
   AttnArgs aa{};
-  aa.q = qa.q;
+  aa.q = static_cast<const uint16_t*>(q_out);
   aa.kv = fa.kv;
   aa.kv_dtype = kv->dtype;
   aa.k_scale = kv->k_scale;

@@ -1,0 +1,204 @@
+// Weight-streaming projections of the MFA decode step on the sm_100a tensor cores.
+//
+// Both hidden-state projections of the layer (Step-3 pages: bud-325 "Method" -- the query
+// is down-projected 7168 -> 2048, normalized and up-projected 2048 -> 64 x 256; the shared
+// K and V heads are projected 7168 -> 256 each) are skinny GEMMs: a few to a few hundred
+// token rows against large weight matrices. Each weight byte is used by every row, so the
+// weights are what streams from HBM. They are put on the M side of the MMA ("swap AB"):
+//     out^T[n, b] = sum_k W[k, n] * X[b, k]
+//   A = W^T tile [128 output features x 64 k] -- read straight from the row-major [in, out]
+//       weight by TMA as two [64 features x 64 k] boxes (MN-major, 128-byte swizzle);
+//   B = X tile   [N rows x 64 k] (K-major, 128-byte swizzle), N = batch rounded up to 16;
+//   D = TMEM accumulator [128 lanes x N columns] fp32.
+// One CTA computes one 128-feature tile over a range of k (split-K for the 7168-long
+// reduction of the x-projection), with warp 0 issuing TMA into a multi-stage ring, one
+// thread of warp 1 issuing the MMAs, and warps 2..5 draining the accumulator.
+#include <cuda_bf16.h>
+
+#include "mfa_internal.cuh"
+#include "sm100.cuh"
+
+namespace mfa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;
+constexpr int kBK = 64;                 // k per stage (one 128-byte swizzle row of X)
+constexpr int kATileBytes = 128 * kBK * 2;  // 16 KB: [64 k rows x 128 B] x 2 boxes
+constexpr int kABoxBytes = kATileBytes / 2;
+constexpr int kMaxStages = 12;
+constexpr int kSmemBudget = 220 * 1024;
+
+struct GemmCtl {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full;
+  uint32_t tmem_base;
+  int32_t abort_flag;
+};
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  __nv_bfloat16 h = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    wgemm_kernel(const __grid_constant__ CUtensorMap w0, const __grid_constant__ CUtensorMap w1,
+                 const __grid_constant__ CUtensorMap w2, const __grid_constant__ CUtensorMap xmap,
+                 WGemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int stages = p.stages;
+  const int b_bytes = p.n_box * 128;
+  uint8_t* a_ring = base;                                  // stages x 16 KB
+  uint8_t* b_ring = base + (size_t)stages * kATileBytes;   // stages x n_box * 128 B
+  GemmCtl& C = *reinterpret_cast<GemmCtl*>(b_ring + (size_t)stages * b_bytes);
+  volatile int* abort = &C.abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // which weight and which 128 output features
+  const int m_abs = p.tile_begin + blockIdx.x;
+  const CUtensorMap* wm = &w0;
+  int n0 = m_abs * 128;
+  if (p.three_weights) {
+    if (m_abs >= p.w0_tiles + p.w1_tiles) {
+      wm = &w2;
+      n0 = (m_abs - p.w0_tiles - p.w1_tiles) * 128;
+    } else if (m_abs >= p.w0_tiles) {
+      wm = &w1;
+      n0 = (m_abs - p.w0_tiles) * 128;
+    }
+  }
+  const int kb0 = blockIdx.y * p.kblocks_per_cta;
+  const int nkb = p.kblocks_per_cta;
+  const int b0 = blockIdx.z * 256;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < stages; ++i) {
+      mbar_init(&C.full[i], 1);
+      mbar_init(&C.empty[i], 1);
+    }
+    mbar_init(&C.acc_full, 1);
+    C.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&C.tmem_base, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = C.tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(wm);
+      prefetch_tensormap(&xmap);
+      const uint64_t evict_first = policy_evict_first();
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % stages, use = i / stages;
+        if (use > 0) mbar_wait(&C.empty[s], (use - 1) & 1, abort);
+        if (*abort) break;
+        mbar_arrive_expect_tx(&C.full[s], kATileBytes + b_bytes);
+        const int k = (kb0 + i) * kBK;
+        uint8_t* a = a_ring + (size_t)s * kATileBytes;
+        tma_load_2d_hint(a, wm, n0, k, &C.full[s], evict_first);
+        tma_load_2d_hint(a + kABoxBytes, wm, n0 + 64, k, &C.full[s], evict_first);
+        tma_load_2d(b_ring + (size_t)s * b_bytes, &xmap, k, b0, &C.full[s]);
+        issued = i + 1;
+      }
+      if (*abort)
+        for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i)
+          mbar_wait_drain(&C.full[i % stages], (i / stages) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_f16(128, p.n_box, true, true, false);
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % stages;
+        mbar_wait(&C.full[s], (i / stages) & 1, abort);
+        tc_fence_after();
+        if (*abort) break;
+        const uint32_t a = smem_u32(a_ring + (size_t)s * kATileBytes);
+        const uint32_t b = smem_u32(b_ring + (size_t)s * b_bytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(a + 2048 * kk, kABoxBytes, 1024);  // MN-major W^T
+          const uint64_t bd = sdesc_sw128(b + 32 * kk, 16, 1024);            // K-major X
+          umma_f16_ss(tmem, ad, bd, idesc, (i | kk) != 0);
+        }
+        umma_commit(&C.empty[s]);
+      }
+      umma_commit(&C.acc_full);
+      mbar_wait_drain(&C.acc_full, 0);
+    }
+  } else {
+    // epilogue: thread = TMEM lane = output feature n0 + row
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+    mbar_wait(&C.acc_full, 0, abort);
+    tc_fence_after();
+    const bool ok = !*abort;
+    const int n_abs = m_abs * 128 + row;  // column in the concatenated output
+    for (int c0 = 0; c0 < p.n_box; c0 += 16) {
+      uint32_t r[16];
+      tmem_ld_32x32b_x16(tmem + lane_addr + c0, r);
+      tmem_wait_ld();
+      if (!ok) continue;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int b = b0 + c0 + i;
+        if (b >= p.batch) break;
+        const float v = __uint_as_float(r[i]);
+        if (p.out_f32 != nullptr)
+          p.out_f32[((size_t)blockIdx.y * p.batch + b) * p.out_ld + n_abs] = v;
+        else
+          p.out_bf16[(size_t)b * p.out_ld + n_abs] = f32_to_bf16_bits(v);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0 && C.abort_flag && p.err != nullptr) atomicOr(p.err, kErrTimeout);
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, p.tmem_cols);
+  }
+}
+
+}  // namespace
+
+int wgemm_n_box(int batch) {
+  const int n = batch < 256 ? batch : 256;
+  return (n + 15) / 16 * 16;
+}
+
+cudaError_t launch_wgemm(const CUtensorMap* w, const CUtensorMap& xmap, WGemmArgs p,
+                         int m_tiles, int splits, cudaStream_t s) {
+  p.n_box = wgemm_n_box(p.batch);
+  const int stage_bytes = kATileBytes + p.n_box * 128;
+  int stages = kSmemBudget / stage_bytes;
+  if (stages > kMaxStages) stages = kMaxStages;
+  if (stages > p.kblocks_per_cta) stages = p.kblocks_per_cta;
+  if (stages < 2) stages = 2;
+  p.stages = stages;
+  int cols = 32;
+  while (cols < p.n_box) cols <<= 1;
+  p.tmem_cols = cols;
+  const size_t smem = 1024 + (size_t)stages * stage_bytes + sizeof(GemmCtl);
+  cudaError_t e =
+      cudaFuncSetAttribute(wgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(m_tiles, splits, (p.batch + 255) / 256);
+  wgemm_kernel<<<grid, kThreads, smem, s>>>(w[0], w[1], w[2], xmap, p);
+  return cudaGetLastError();
+}
+
+}  // namespace mfa

@@ -86,14 +86,26 @@ inline WsLayout ws_layout(int batch, int num_sms) {
 // Kernel launchers (defined in the .cu files); all return cudaGetLastError().
 // ---------------------------------------------------------------------------------------
 
-struct XProjArgs {
-  const uint16_t* x;     // [batch, 7168] bf16
-  const uint16_t* w[3];  // W_qdown [7168, 2048], W_k [7168, 256], W_v [7168, 256]
-  int batch;
-  int tile_begin, tile_end;  // 128-column tiles of the 2560 concatenated columns
-  float* part;               // [kXProjSplits][batch][2560]
+// Weight-streaming GEMM on the tensor cores: out^T[n, b] = sum_k W[k, n] X[b, k] for 128
+// output features per CTA (grid.x), a range of k per CTA (grid.y: split-K), and up to 256
+// rows of X per CTA (grid.z).
+struct WGemmArgs {
+  int batch;            // rows of X
+  int tile_begin;       // first 128-feature tile (of the concatenated outputs)
+  int three_weights;    // 1: tiles [0, w0_tiles) read w[0], then w1_tiles of w[1], then w[2]
+  int w0_tiles, w1_tiles;
+  int kblocks_per_cta;  // 64-wide k blocks per CTA
+  float* out_f32;       // fp32 split partials [grid.y][batch][out_ld], or null
+  uint16_t* out_bf16;   // bf16 [batch][out_ld] (when out_f32 is null)
+  int out_ld;
+  uint32_t* err;
+  int n_box, stages, tmem_cols;  // filled in by launch_wgemm
 };
-cudaError_t launch_xproj(const XProjArgs& a, cudaStream_t s);
+// w: 3 tensor maps over row-major [K, N_out] bf16 weights, boxes [64 x 64]; xmap over X
+// [batch, K] bf16, boxes [64 x wgemm_n_box(batch)]; all with 128-byte swizzle.
+cudaError_t launch_wgemm(const CUtensorMap* w, const CUtensorMap& xmap, WGemmArgs p,
+                         int m_tiles, int splits, cudaStream_t s);
+int wgemm_n_box(int batch);
 
 struct FinishArgs {
   const float* part;  // x-projection partials
@@ -112,13 +124,6 @@ struct FinishArgs {
 };
 cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s);
 
-struct QUpArgs {
-  const uint16_t* c_hat;  // [batch, 2048]
-  const uint16_t* w_qup;  // [2048, 16384]
-  int batch;
-  uint16_t* q;  // [batch, 16384]
-};
-cudaError_t launch_q_up(const QUpArgs& a, cudaStream_t s);
 
 struct AttnArgs {
   const uint16_t* q;        // [batch, 64, 256] bf16
