@@ -108,6 +108,9 @@ mfa_status run_q_up(const uint16_t* c_hat, const void* w_qup, void* q, int batch
   return cuda_status(launch_wgemm(wm, xm, p, kQWidth / 128, 1, s));
 }
 
+
+}  // namespace
+
 mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
                           const void* w_qup, float eps, void* q_out, int batch, void* ws,
                           const WsLayout& L, cudaStream_t s) {
@@ -125,8 +128,6 @@ mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
   if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
   return run_q_up(fa.c_hat, w_qup, q_out, batch, err, s);
 }
-
-}  // namespace
 
 EncodeTiledFn encode_tiled_fn() {
   static EncodeTiledFn fn = nullptr;

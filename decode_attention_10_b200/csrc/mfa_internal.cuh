@@ -145,6 +145,12 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);  // CUDA-core k
 cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s);
 size_t attention_tc_smem_bytes();
 
+// The query path (x-projection onto W_qdown, finish with RMSNorm, q_up) on `s`, using the
+// x-projection partials, c_hat and error word at the offsets of L inside `ws`.
+mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
+                          const void* w_qup, float eps, void* q_out, int batch, void* ws,
+                          const WsLayout& L, cudaStream_t s);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

@@ -40,7 +40,10 @@ _SIGNATURES = {
                                        _P]),
     "mfa_decode_layer": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
                                         ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+    "mfa_query_proj_noalloc": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_float, _P,
+                                              ctypes.c_int32, _P]),
 }
+NOALLOC_MAX_BATCH = 32
 
 
 class KvCacheDesc(ctypes.Structure):
@@ -220,3 +223,15 @@ def decode_layer(x, w_qdown, gamma, w_qup, w_k, w_v, cache: KVCache, seq_lens,
                                 ws.nbytes, _stream(stream)),
            "mfa_decode_layer")
     return q_out, out
+
+
+def query_proj_noalloc(x, w_qdown, gamma, w_qup, eps: float = 1e-6, q_out=None, stream=None):
+    """mfa_query_proj without a workspace: the library's built-in scratch (batch <= 32)."""
+    lib = load()
+    bsz = int(x.shape[0])
+    if q_out is None:
+        q_out = torch.empty(bsz, N_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=x.device)
+    _check(lib.mfa_query_proj_noalloc(_ptr(x), _ptr(w_qdown), _ptr(gamma), _ptr(w_qup),
+                                      float(eps), _ptr(q_out), bsz, _stream(stream)),
+           "mfa_query_proj_noalloc")
+    return q_out

@@ -175,6 +175,36 @@ MFA_API mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const vo
                             const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
                             void* q_out, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Without a caller-provided workspace
+ * ------------------------------------------------------------------------------------- */
+
+/* Largest batch mfa_query_proj_noalloc accepts. */
+#define MFA_NOALLOC_MAX_BATCH 32
+
+/* mfa_query_proj without the workspace, for callers that cannot allocate device memory:
+ * programs whose device memory is planned once, up front, by another component (a serving
+ * engine that gives all free HBM to its KV cache); loops that must not call the allocator
+ * once running, because cudaMalloc can synchronize the device and take unbounded time; and
+ * plugin interfaces that pass inputs and outputs but no workspace. The Step-3 pages have no
+ * counterpart to this call: it is a convenience of the library, not a step of the method.
+ * Arguments, results and rounding are those of mfa_query_proj without ws/ws_bytes.
+ *   - The scratch it needs (about 2.3 MiB: split-K partials, the normalized low-rank query,
+ *     an error word) is one fixed array inside the library, reserved on every GPU that loads
+ *     the library until the process exits. No call allocates or frees anything.
+ *   - batch > MFA_NOALLOC_MAX_BATCH returns MFA_ERR_WORKSPACE (the built-in scratch is too
+ *     small for it); batch < 1, eps <= 0 or a null/misaligned pointer return
+ *     MFA_ERR_INVALID_ARG. Nothing is enqueued in either case.
+ *   - The first call on a device looks up the array's device address on that device (it
+ *     must be the current device); make that first call before any stream capture.
+ *   - Every call on a device uses the same array, which keeps the last call's contents.
+ *     Calls that can run at the same time on the GPU (unordered streams, several host
+ *     threads) race on it and corrupt each other's results: order them on one stream.
+ *   - The device-side error word is cleared at the start of each call and not reported. */
+MFA_API mfa_status mfa_query_proj_noalloc(const void* x, const void* w_qdown, const void* gamma,
+                                          const void* w_qup, float eps, void* q_out,
+                                          int32_t batch, void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif
