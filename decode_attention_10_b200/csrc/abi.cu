@@ -160,16 +160,13 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, i
 
 namespace {
 
-// The attention of one call: the tensor-core kernel for bf16 caches, the CUDA-core one
-// for FP8 caches.
+// The attention of one call: the tensor-core kernel, then the merge of split sequences.
 mfa_status run_attention(const AttnArgs& aa, cudaStream_t s) {
-  if (aa.kv_dtype == MFA_KV_BF16) {
-    CUtensorMap q_map;
-    if (!encode_2d(&q_map, aa.q, (uint64_t)aa.batch * kHeads, kHeadDim, 2, 64, 64))
-      return MFA_ERR_CUDA;
-    return cuda_status(launch_attention_tc(q_map, aa, s));
-  }
-  return cuda_status(launch_attention(aa, s));
+  CUtensorMap q_map;
+  if (!encode_2d(&q_map, aa.q, (uint64_t)aa.batch * kHeads, kHeadDim, 2, 64, 64))
+    return MFA_ERR_CUDA;
+  if (launch_attention_tc(q_map, aa, s) != cudaSuccess) return MFA_ERR_CUDA;
+  return cuda_status(launch_attention_combine(aa, s));
 }
 
 }  // namespace
@@ -328,7 +325,7 @@ mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t*
   aa.out = static_cast<uint16_t*>(out);
   aa.batch = kv->batch;
   aa.partials = at<float>(ws, L.attn_part);
-  aa.counters = at<int32_t>(ws, L.counters);
+  aa.seq_info = at<int2>(ws, L.seq_info);
   aa.err = at<uint32_t>(ws, L.err);
   aa.grid = L.attn_grid;
   return run_attention(aa, static_cast<cudaStream_t>(stream));
@@ -382,7 +379,7 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   aa.out = static_cast<uint16_t*>(out);
   aa.batch = batch;
   aa.partials = at<float>(ws, L.attn_part);
-  aa.counters = at<int32_t>(ws, L.counters);
+  aa.seq_info = at<int2>(ws, L.seq_info);
   aa.err = fa.err;
   aa.grid = L.attn_grid;
   return run_attention(aa, s);

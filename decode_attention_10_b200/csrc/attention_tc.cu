@@ -1,5 +1,5 @@
 // Decode attention of the 64 query heads over the shared K/V head on the sm_100a tensor
-// cores (bf16 KV cache).
+// cores, for bf16 and FP8 (e4m3) KV caches.
 //
 // What it computes (Step-3 pages: bud-325 "Method" -- 64 query heads share ONE K head and
 // ONE V head of dimension 256; decode cost is max(attention compute, KV memory access)):
@@ -23,8 +23,18 @@
 //   Tiles are windows of 128 positions; the last window of a work item ends at the item's
 //   end (it may start before the item or at a negative position, which TMA zero-fills), so
 //   rows past a sequence's length are never read. Positions outside the item are masked.
+// FP8 caches: TMA brings raw e4m3 boxes of [128 positions x 128 dims] into a 4-slot ring;
+// the softmax warps convert them (e4m3 -> f16 is exact) into the same swizzled 16 KB chunks
+// the bf16 path uses (a 6-slot ring), and both products run with f16 operands: Q is
+// converted to f16 in place once per item (scaled by a power of two if its magnitude could
+// overflow f16), P is written as f16. The K and V scales fold into the softmax scale and
+// the output scale.
 // The split plan (which CTA streams which tiles) is computed on chip: see attn_plan.cuh.
+// A sequence covered by one CTA is finished in place; the items of a sequence split over
+// several CTAs leave (m, l, acc) partials that attention_combine_kernel merges.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "attn_plan.cuh"
 #include "mfa_internal.cuh"
@@ -37,8 +47,11 @@ using namespace sm100;
 
 constexpr int kThreads = 192;
 constexpr int kSoftmaxThreads = 128;
-constexpr int kSlots = 10;             // ring slots (even: a V half-tile's 2 chunks are adjacent)
-constexpr int kChunkBytes = 16384;     // [128 positions x 64 dims] bf16
+constexpr int kChunkBytes = 16384;     // [128 positions x 64 dims] 16-bit, 128-byte swizzle
+constexpr int kRingBytes = 10 * kChunkBytes;
+constexpr int kRawSlots = 4;           // FP8: raw e4m3 boxes [128 positions x 128 dims]
+constexpr int kRawBytes = 16384;
+constexpr int kMaxSlots = 10;
 constexpr int kQChunkBytes = 8192;     // [64 heads x 64 dims] bf16
 constexpr int kPBytes = 16384;         // P^T: [128 positions x 64 heads] bf16
 constexpr uint32_t kTmemCols = 256;
@@ -47,11 +60,21 @@ constexpr uint32_t kTmemO = 128;       // O^T halves: columns [128, 192) and [19
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-constexpr uint32_t kIdescS = idesc_f16(128, 64, true, false, false);  // K (K-major) x Q (K-major)
-constexpr uint32_t kIdescPV = idesc_f16(128, 64, true, true, true);   // V^T (MN) x P^T (MN)
+// Per cache type: the MMA operand ring (chunks of [128 positions x 64 dims], 16-bit), where
+// it sits in the ring area, the operand type, and the L2 prefetch distance.
+template <bool kFp8>
+struct Cfg {
+  static constexpr int kSlots = kFp8 ? 6 : 10;  // even: a V half-tile's 2 chunks are adjacent
+  static constexpr int kRingOff = kFp8 ? kRawSlots * kRawBytes : 0;
+  static constexpr bool kBf16 = !kFp8;           // operands: bf16, or f16 for FP8 caches
+  static constexpr int kPrefetchTiles = kFp8 ? 4 : 2;
+  static constexpr uint32_t kIdescS = idesc_f16(128, 64, kBf16, false, false);  // K x Q^T
+  static constexpr uint32_t kIdescPV = idesc_f16(128, 64, kBf16, true, true);   // V^T x P^T
+};
+static_assert(Cfg<true>::kRingOff + Cfg<true>::kSlots * kChunkBytes <= kRingBytes, "ring");
 
 struct __align__(1024) TcSmem {
-  uint8_t ring[kSlots][kChunkBytes];
+  uint8_t ring_area[kRingBytes];
   uint8_t q[4][kQChunkBytes];
   uint8_t p[kPBytes];
   PlanSmem plan;
@@ -59,17 +82,27 @@ struct __align__(1024) TcSmem {
   float alpha[kHeads];
   float red[4][kHeads];
   float lsum[kHeads];
-  uint64_t kv_full[kSlots];
-  uint64_t kv_empty[kSlots];
-  uint64_t q_full, q_empty;
+  uint64_t kv_full[kMaxSlots];
+  uint64_t kv_empty[kMaxSlots];
+  uint64_t raw_full[kRawSlots];
+  uint64_t raw_empty[kRawSlots];
+  uint64_t q_full, q_empty, q_ready;
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_free;
   uint64_t o_free;
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort_flag;
-  int32_t last_flag;
+  int32_t q_exp;  // FP8: Q was scaled by 2^-q_exp on conversion to f16
 };
+
+template <bool kFp8>
+__device__ __forceinline__ uint8_t* ring_chunk(TcSmem& S, uint32_t slot) {
+  return S.ring_area + Cfg<kFp8>::kRingOff + slot * kChunkBytes;
+}
+__device__ __forceinline__ uint8_t* raw_box(TcSmem& S, uint32_t slot) {
+  return S.ring_area + slot * kRawBytes;
+}
 
 __device__ __forceinline__ int num_tiles(const WorkItem& it) {
   return (it.tok1 - it.tok0 + kTile - 1) / kTile;
@@ -91,6 +124,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t w) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
+}
+__device__ __forceinline__ float f16_hi(uint32_t w) {
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+}
+
+// four e4m3 codes (one 32-bit word, lowest byte first) -> two f16x2 words, exact
+__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t w) {
+  const __half2_raw lo =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
+  const __half2_raw hi =
+      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  return make_uint2(static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16),
+                    static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16));
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -143,7 +199,9 @@ __device__ __forceinline__ void warp_transpose_sum64(float (&v)[64], int lane) {
 // ---------------------------------------------------------------------------------------
 // warp 0: TMA producer
 // ---------------------------------------------------------------------------------------
+template <bool kFp8>
 __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs& a, int g) {
+  using C = Cfg<kFp8>;
   volatile int* abort = &S.abort_flag;
   uint32_t chunk = 0, issued = 0;
   int item = 0, q_issued = 0;
@@ -159,31 +217,53 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
       q_issued = item + 1;
     }
     const int n = num_tiles(it);
+    // bf16: four [128 x 64] boxes per tile straight into the MMA ring; FP8: two raw
+    // [128 x 128] e4m3 boxes per tile into the raw ring
     auto load_tile = [&](const CUtensorMap* m, int t) {
       int y, a0, e0;
       tile_window(it, t, y, a0, e0);
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
-        if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);
+      constexpr int kBoxes = kFp8 ? 2 : 4;
+      constexpr uint32_t kN = kFp8 ? kRawSlots : C::kSlots;
+      for (int c = 0; c < kBoxes; ++c) {
+        const uint32_t slot = chunk % kN, use = chunk / kN;
+        uint64_t* empty = kFp8 ? &S.raw_empty[slot] : &S.kv_empty[slot];
+        uint64_t* full = kFp8 ? &S.raw_full[slot] : &S.kv_full[slot];
+        if (use > 0) mbar_wait(empty, (use - 1) & 1, abort);
         if (!*abort) {
-          mbar_arrive_expect_tx(&S.kv_full[slot], kChunkBytes);
-          tma_load_2d(S.ring[slot], m, 64 * c, y, &S.kv_full[slot]);
+          mbar_arrive_expect_tx(full, kChunkBytes);
+          uint8_t* dst = kFp8 ? raw_box(S, slot) : ring_chunk<kFp8>(S, slot);
+          tma_load_2d(dst, m, (kFp8 ? 128 : 64) * c, y, full);
           issued = chunk + 1;
         }
         ++chunk;
       }
     };
+    // L2 prefetch runs kPrefetchTiles ahead of the loads, so that the shared-memory ring
+    // only has to cover L2 latency
+    auto prefetch_tile = [&](int t) {
+      if (t >= n || *abort) return;
+      int y, a0, e0;
+      tile_window(it, t, y, a0, e0);
+      constexpr int kBoxes = kFp8 ? 2 : 4;
+      for (int c = 0; c < kBoxes; ++c) {
+        tma_prefetch_2d(km, (kFp8 ? 128 : 64) * c, y);
+        tma_prefetch_2d(vm, (kFp8 ? 128 : 64) * c, y);
+      }
+    };
+    for (int t = 0; t < C::kPrefetchTiles; ++t) prefetch_tile(t);
     load_tile(km, 0);
     for (int t = 0; t < n; ++t) {
       if (t + 1 < n) load_tile(km, t + 1);
       load_tile(vm, t);
+      prefetch_tile(t + C::kPrefetchTiles);
     }
     ++item;
   });
   // Before the CTA may exit, every copy it started must have landed.
   if (*abort) {
-    for (uint32_t c = (issued > kSlots ? issued - kSlots : 0); c < issued; ++c)
-      mbar_wait_drain(&S.kv_full[c % kSlots], (c / kSlots) & 1);
+    constexpr uint32_t kN = kFp8 ? kRawSlots : C::kSlots;
+    for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
+      mbar_wait_drain(kFp8 ? &S.raw_full[c % kN] : &S.kv_full[c % kN], (c / kN) & 1);
     if (q_issued > 0) mbar_wait_drain(&S.q_full, (q_issued - 1) & 1);
   }
 }
@@ -191,7 +271,10 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
 // ---------------------------------------------------------------------------------------
 // warp 1 (one thread): MMA issue
 // ---------------------------------------------------------------------------------------
+template <bool kFp8>
 __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
+  using C = Cfg<kFp8>;
+  constexpr uint32_t kSlots = C::kSlots;
   volatile int* abort = &S.abort_flag;
   uint32_t chunk = 0;
   uint32_t gt = 0;  // tiles issued so far by this CTA (all items)
@@ -199,7 +282,7 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
   const uint32_t q_base = smem_u32(S.q[0]);
   plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem& it) {
     const int n = num_tiles(it);
-    mbar_wait(&S.q_full, item & 1, abort);
+    mbar_wait(kFp8 ? &S.q_ready : &S.q_full, item & 1, abort);
     tc_fence_after();
 
     auto issue_s = [&](uint32_t tile) {
@@ -212,12 +295,12 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
         mbar_wait(&S.kv_full[slot], use & 1, abort);
         tc_fence_after();
         if (!*abort) {
-          const uint32_t a_base = smem_u32(S.ring[slot]);
+          const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, slot));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
             const uint64_t bd = sdesc_sw128(q_base + c * kQChunkBytes + 32 * kk, 16, 1024);
-            umma_f16_ss(d, ad, bd, kIdescS, (c | kk) != 0);
+            umma_f16_ss(d, ad, bd, C::kIdescS, (c | kk) != 0);
           }
           umma_commit(&S.kv_empty[slot]);
         }
@@ -239,12 +322,12 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
         tc_fence_after();
         if (!*abort) {
           const uint32_t d = tmem + kTmemO + 64 * h;
-          const uint32_t a_base = smem_u32(S.ring[s0]);
+          const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, s0));
 #pragma unroll
           for (int kt = 0; kt < kTile / 16; ++kt) {
             const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
             const uint64_t bd = sdesc_sw128(p_base + 2048 * kt, kPBytes, 1024);
-            umma_f16_ss(d, ad, bd, kIdescPV, !(first && kt == 0));
+            umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
           }
           umma_commit(&S.kv_empty[s0]);
           umma_commit(&S.kv_empty[s1]);
@@ -269,74 +352,86 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
 }
 
 // ---------------------------------------------------------------------------------------
-// split merge (run by the 128 softmax threads of the CTA that finished a sequence last):
-//   M[h] = max_i m_i[h],  L[h] = sum_i l_i[h] 2^(m_i[h] - M[h]),
-//   out[h][d] = v_mul / L[h] * sum_i 2^(m_i[h] - M[h]) acc_i[h][d].
-// The per-split weights are staged in shared memory (the P^T buffer, idle at this point),
-// so each thread keeps 2 x 32 independent loads in flight per split.
+// FP8 conversions, run by the 128 softmax threads
 // ---------------------------------------------------------------------------------------
-__device__ void merge_splits(TcSmem& S, const AttnArgs& a, const WorkItem& it, int tid,
-                             uint16_t* out, float v_mul) {
-  constexpr int kChunkSplits = kPBytes / (sizeof(float) * kHeads);  // 64 splits per pass
-  float* w = reinterpret_cast<float*>(S.p);
-  const int base = S.plan.slot_base[it.b];
-  const int ns = it.nsplit;
-  if (tid < kHeads) {
-    float M = -INFINITY;
-#pragma unroll 4
-    for (int i = 0; i < ns; ++i) M = fmaxf(M, __ldcg(partial_m(a.partials, base + i) + tid));
-    float L = 0.f;
-#pragma unroll 4
-    for (int i = 0; i < ns; ++i)
-      L += __ldcg(partial_l(a.partials, base + i) + tid) *
-           exp2f(__ldcg(partial_m(a.partials, base + i) + tid) - M);
-    S.alpha[tid] = M;          // reused as scratch: the merge max
-    S.lsum[tid] = v_mul / L;   // and the output scale
+
+// Raw box `rbox` (e4m3, [128 positions x 128 dims], 128-byte swizzle) -> MMA ring chunks
+// `chunk` and `chunk + 1` (f16, [128 positions x 64 dims] each, same swizzle).
+__device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int tid, int lane,
+                            volatile int* abort) {
+  constexpr uint32_t kSlots = Cfg<true>::kSlots;
+  const uint32_t rslot = rbox % kRawSlots;
+  mbar_wait(&S.raw_full[rslot], (rbox / kRawSlots) & 1, abort);
+  const uint8_t* raw = raw_box(S, rslot);
+#pragma unroll 1
+  for (int cc = 0; cc < 2; ++cc) {
+    const uint32_t ch = chunk + cc, fslot = ch % kSlots, fuse = ch / kSlots;
+    if (fuse > 0) mbar_wait(&S.kv_empty[fslot], (fuse - 1) & 1, abort);
+    uint8_t* dst = ring_chunk<true>(S, fslot);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int pc = tid + 128 * i;  // one 16-byte piece: 16 dims of one position
+      const int r = pc >> 2, jj = pc & 3, j = 4 * cc + jj, sw = r & 7;
+      const uint4 v = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
+      const uint2 h0 = e4m3x4_to_f16x4(v.x), h1 = e4m3x4_to_f16x4(v.y);
+      const uint2 h2 = e4m3x4_to_f16x4(v.z), h3 = e4m3x4_to_f16x4(v.w);
+      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj) ^ sw) << 4)) =
+          make_uint4(h0.x, h0.y, h1.x, h1.y);
+      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj + 1) ^ sw) << 4)) =
+          make_uint4(h2.x, h2.y, h3.x, h3.y);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.kv_full[fslot]);
   }
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&S.raw_empty[rslot]);
+}
+
+// Q of the current item (bf16, loaded by TMA) -> f16 in place, scaled by 2^-e where e >= 0
+// is the smallest exponent that keeps every |q| below 2^15. Returns e.
+__device__ int convert_q(TcSmem& S, int item, int tid, int warp, int lane, volatile int* abort) {
+  mbar_wait(&S.q_full, item & 1, abort);
+  uint4* q = reinterpret_cast<uint4*>(S.q[0]);
+  constexpr int kPieces = kHeads * kHeadDim / 8 / kSoftmaxThreads;  // 16 per thread
+  float mx = 0.f;
+#pragma unroll
+  for (int i = 0; i < kPieces; ++i) {
+    const uint4 v = q[tid + kSoftmaxThreads * i];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[k] << 16)),
+                           fabsf(__uint_as_float(w[k] & 0xFFFF0000u))));
+  }
+  mx = warp_max_f32(mx);
+  if (lane == 0) S.red[warp - 2][0] = mx;
   named_bar_sync(1, kSoftmaxThreads);
-#pragma unroll 1
-  for (int hg = 0; hg < 2; ++hg) {
-    float o0[32], o1[32];
+  const float m = fmaxf(fmaxf(S.red[0][0], S.red[1][0]), fmaxf(S.red[2][0], S.red[3][0]));
+  const int e = (m >= 32768.f && m <= 3.0e38f) ? ilogbf(m) - 14 : 0;
+  const float sc = ldexpf(1.f, -e);
 #pragma unroll
-    for (int h = 0; h < 32; ++h) o0[h] = o1[h] = 0.f;
-#pragma unroll 1
-    for (int i0 = 0; i0 < ns; i0 += kChunkSplits) {
-      const int cnt = min(kChunkSplits, ns - i0);
-      for (int e = tid; e < cnt * kHeads; e += kSoftmaxThreads) {
-        const int ii = e / kHeads, h = e % kHeads;
-        w[e] = exp2f(__ldcg(partial_m(a.partials, base + i0 + ii) + h) - S.alpha[h]);
-      }
-      named_bar_sync(1, kSoftmaxThreads);
-#pragma unroll 1
-      for (int ii = 0; ii < cnt; ++ii) {
-        const float* src = partial_acc(a.partials, base + i0 + ii) + (hg * 32) * kHeadDim;
-        const float* wi = w + ii * kHeads + hg * 32;
-        float x0[32], x1[32];
+  for (int i = 0; i < kPieces; ++i) {
+    uint4& ref = q[tid + kSoftmaxThreads * i];
+    const uint4 v = ref;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
 #pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          x0[h] = __ldcg(src + h * kHeadDim + tid);
-          x1[h] = __ldcg(src + h * kHeadDim + 128 + tid);
-        }
-#pragma unroll
-        for (int h = 0; h < 32; ++h) {
-          o0[h] = fmaf(wi[h], x0[h], o0[h]);
-          o1[h] = fmaf(wi[h], x1[h], o1[h]);
-        }
-      }
-      named_bar_sync(1, kSoftmaxThreads);
-    }
-#pragma unroll
-    for (int h = 0; h < 32; ++h) {
-      const int hh = hg * 32 + h;
-      out[hh * kHeadDim + tid] = f32_to_bf16_bits(o0[h] * S.lsum[hh]);
-      out[hh * kHeadDim + 128 + tid] = f32_to_bf16_bits(o1[h] * S.lsum[hh]);
-    }
+    for (int k = 0; k < 4; ++k)
+      o[k] = pack_f16x2(__uint_as_float(w[k] << 16) * sc, __uint_as_float(w[k] & 0xFFFF0000u) * sc);
+    ref = make_uint4(o[0], o[1], o[2], o[3]);
   }
+  fence_proxy_async_smem();
+  named_bar_sync(1, kSoftmaxThreads);  // every thread has read red before it is reused
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&S.q_ready);
+  return e;
 }
 
 // ---------------------------------------------------------------------------------------
-// warps 2..5: softmax, rescale, epilogue, split merge
+// warps 2..5: softmax, rescale, epilogue (and the FP8 conversions)
 // ---------------------------------------------------------------------------------------
+template <bool kFp8>
 __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
   volatile int* abort = &S.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -344,10 +439,10 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
   const int quad = warp & 3;               // TMEM lane quadrant this warp may access
   const int row = quad * 32 + lane;        // tile position / O^T row of this thread
   const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-  const bool fp8 = a.kv_dtype == MFA_KV_FP8_E4M3;
-  const float s_mul = a.scale * kLog2e * (fp8 ? a.k_scale : 1.f);
-  const float v_mul = fp8 ? a.v_scale : 1.f;
+  const float s_mul0 = a.scale * kLog2e * (kFp8 ? a.k_scale : 1.f);
+  const float v_mul = kFp8 ? a.v_scale : 1.f;
   uint32_t gt = 0;
+  uint32_t rbox = 0, fchunk = 0;  // FP8: raw boxes and MMA-ring chunks converted so far
   int item = 0;
   uint8_t* const p_row = S.p + row * 128;
 
@@ -355,8 +450,23 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     const int n = num_tiles(it);
     // this warp's running row sums of heads 2*lane and 2*lane + 1
     float l0 = 0.f, l1 = 0.f;
+    float s_mul = s_mul0;
+    auto convert_tile = [&]() {  // one K or V tile: two raw boxes -> four ring chunks
+      convert_box(S, rbox, fchunk, tid, lane, abort);
+      convert_box(S, rbox + 1, fchunk + 2, tid, lane, abort);
+      rbox += 2;
+      fchunk += 4;
+    };
+    if constexpr (kFp8) {
+      s_mul = s_mul0 * ldexpf(1.f, convert_q(S, item, tid, warp, lane, abort));
+      convert_tile();  // K(0)
+    }
 
     for (int t = 0; t < n; ++t) {
+      if constexpr (kFp8) {
+        if (t + 1 < n) convert_tile();  // K(t + 1), consumed by S(t + 1)
+        convert_tile();                 // V(t), consumed by PV(t)
+      }
       const uint32_t tile = gt + t, j = tile & 1, k = tile >> 1;
       int y, a0, e0;
       tile_window(it, t, y, a0, e0);
@@ -419,17 +529,24 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
         }
       }
 
-      // probabilities (rounded to bf16, the precision the tensor core reads), the P^T row of
-      // this position, and the row sums of the rounded values
+      // probabilities (rounded to the operand type the tensor core reads: bf16, or f16
+      // for FP8 caches), the P^T row of this position, and the row sums of the rounded values
       uint32_t pk[kHeads / 2];
 #pragma unroll
       for (int h = 0; h < kHeads; h += 2) {
         const float p0 = ex2(s[h] - S.m_used[h]);
         const float p1 = ex2(s[h + 1] - S.m_used[h + 1]);
-        const uint32_t w = pack_bf16x2(p0, p1);
-        pk[h / 2] = w;
-        s[h] = __uint_as_float(w << 16);
-        s[h + 1] = __uint_as_float(w & 0xFFFF0000u);
+        if constexpr (kFp8) {
+          const uint32_t w = pack_f16x2(p0, p1);
+          pk[h / 2] = w;
+          s[h] = f16_lo(w);
+          s[h + 1] = f16_hi(w);
+        } else {
+          const uint32_t w = pack_bf16x2(p0, p1);
+          pk[h / 2] = w;
+          s[h] = __uint_as_float(w << 16);
+          s[h + 1] = __uint_as_float(w & 0xFFFF0000u);
+        }
       }
       warp_transpose_sum64(s, lane);
       l0 += s[0];
@@ -482,32 +599,16 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.o_free);
 
-    if (it.slot >= 0 && ok) {
-      if (tid < kHeads) {
-        partial_m(a.partials, it.slot)[tid] = S.m_used[tid];
-        partial_l(a.partials, it.slot)[tid] = S.lsum[tid];
-      }
-      __threadfence();
-      named_bar_sync(1, kSoftmaxThreads);
-      if (tid == 0) {
-        const int old = atomicAdd(a.counters + it.b, 1);
-        const int last = old == it.nsplit - 1;
-        if (last) atomicExch(a.counters + it.b, 0);
-        S.last_flag = last;
-      }
-      named_bar_sync(1, kSoftmaxThreads);
-      if (S.last_flag) {
-        __threadfence();
-        merge_splits(S, a, it, tid, out, v_mul);
-      }
-      named_bar_sync(1, kSoftmaxThreads);
-    } else {
-      named_bar_sync(1, kSoftmaxThreads);
+    if (it.slot >= 0 && ok && tid < kHeads) {
+      partial_m(a.partials, it.slot)[tid] = S.m_used[tid];
+      partial_l(a.partials, it.slot)[tid] = S.lsum[tid];
     }
+    // m_used / lsum are rewritten by the next item only after its first barrier
     ++item;
   });
 }
 
+template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap q_map, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -517,12 +618,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = blockIdx.x;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSlots; ++i) {
-      mbar_init(&S.kv_full[i], 1);
+    for (int i = 0; i < Cfg<kFp8>::kSlots; ++i) {
+      mbar_init(&S.kv_full[i], kFp8 ? 4 : 1);  // FP8: the four converting warps arrive
       mbar_init(&S.kv_empty[i], 1);
+    }
+    for (int i = 0; i < kRawSlots; ++i) {
+      mbar_init(&S.raw_full[i], 1);
+      mbar_init(&S.raw_empty[i], 4);
     }
     mbar_init(&S.q_full, 1);
     mbar_init(&S.q_empty, 1);
+    mbar_init(&S.q_ready, 4);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_free[i], 4);
@@ -538,10 +644,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  pdl_launch_dependents();  // the combine kernel may start launching; it waits for us
   plan_build(S.plan, a.seq_lens, a.kv, a.batch, a.grid, a.err, g == 0);
-  for (int b = g; b < a.batch; b += gridDim.x) {
-    if (S.plan.len[b] != 0) continue;
-    for (int i = threadIdx.x; i < kQWidth; i += kThreads) a.out[(size_t)b * kQWidth + i] = 0;
+  if (g == 0) {
+    // per sequence: its first partial slot and its number of splits (0 = rejected), for
+    // the combine kernel
+    const int NT = S.plan.tile_start[a.batch], G = S.plan.grid;
+    for (int b = threadIdx.x; b < a.batch; b += kThreads) {
+      const int ts = S.plan.tile_start[b], te = S.plan.tile_start[b + 1];
+      const int ns = te > ts ? plan_cta_of(te - 1, G, NT) - plan_cta_of(ts, G, NT) + 1 : 0;
+      a.seq_info[b] = make_int2(S.plan.slot_base[b], ns);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -549,11 +662,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) run_producer(S, &q_map, a, g);
+    if (lane == 0) run_producer<kFp8>(S, &q_map, a, g);
   } else if (warp == 1) {
-    if (lane == 0) run_mma(S, a, g, tmem);
+    if (lane == 0) run_mma<kFp8>(S, a, g, tmem);
   } else {
-    run_softmax(S, a, g, tmem);
+    run_softmax<kFp8>(S, a, g, tmem);
   }
 
   tc_fence_before();
@@ -566,17 +679,92 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// combine: one block per (sequence, group of 4 heads); thread t owns dims 2t and 2t + 1.
+//   M[h] = max_i m_i[h],  L[h] = sum_i l_i[h] 2^(m_i[h] - M[h]),
+//   out[h][d] = v_mul / L[h] * sum_i 2^(m_i[h] - M[h]) acc_i[h][d].
+// Sequences finished by a single work item were written by the attention kernel; rejected
+// sequences (no split) get a zero output here.
+// ---------------------------------------------------------------------------------------
+constexpr int kCombineHeads = 4;
+
+__global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
+  pdl_wait();
+  const int b = blockIdx.x, h0 = blockIdx.y * kCombineHeads, tid = threadIdx.x;
+  const int2 info = a.seq_info[b];
+  const int base = info.x, ns = info.y;
+  uint32_t* out = reinterpret_cast<uint32_t*>(a.out + (size_t)b * kQWidth + h0 * kHeadDim);
+  if (ns == 0) {
+    for (int i = tid; i < kCombineHeads * kHeadDim / 2; i += 128) out[i] = 0u;
+    return;
+  }
+  if (ns == 1) return;
+  const float v_mul = a.kv_dtype == MFA_KV_FP8_E4M3 ? a.v_scale : 1.f;
+  float M[kCombineHeads];
+#pragma unroll
+  for (int h = 0; h < kCombineHeads; ++h) M[h] = -INFINITY;
+#pragma unroll 4
+  for (int i = 0; i < ns; ++i) {
+    const float4 m = __ldcg(reinterpret_cast<const float4*>(partial_m(a.partials, base + i) + h0));
+    M[0] = fmaxf(M[0], m.x), M[1] = fmaxf(M[1], m.y), M[2] = fmaxf(M[2], m.z),
+    M[3] = fmaxf(M[3], m.w);
+  }
+  float L[kCombineHeads] = {0.f, 0.f, 0.f, 0.f};
+  float2 o[kCombineHeads];
+#pragma unroll
+  for (int h = 0; h < kCombineHeads; ++h) o[h] = make_float2(0.f, 0.f);
+#pragma unroll 4
+  for (int i = 0; i < ns; ++i) {
+    const float4 m = __ldcg(reinterpret_cast<const float4*>(partial_m(a.partials, base + i) + h0));
+    const float4 l = __ldcg(reinterpret_cast<const float4*>(partial_l(a.partials, base + i) + h0));
+    const float* acc = partial_acc(a.partials, base + i) + h0 * kHeadDim + 2 * tid;
+    const float mm[4] = {m.x, m.y, m.z, m.w}, ll[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+    for (int h = 0; h < kCombineHeads; ++h) {
+      const float w = exp2f(mm[h] - M[h]);
+      const float2 x = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
+      L[h] = fmaf(ll[h], w, L[h]);
+      o[h].x = fmaf(w, x.x, o[h].x);
+      o[h].y = fmaf(w, x.y, o[h].y);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < kCombineHeads; ++h) {
+    const float inv = v_mul / L[h];
+    out[h * kHeadDim / 2 + tid] = pack_bf16x2(o[h].x * inv, o[h].y * inv);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.batch, kHeads / kCombineHeads, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attention_combine_kernel, a);
+}
 
 size_t attention_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
 
-cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s) {
+template <bool kFp8>
+static cudaError_t launch_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s) {
   const size_t smem = attention_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel,
+  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<kFp8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attention_tc_kernel<<<a.grid, kThreads, smem, s>>>(q_map, a);
+  attention_tc_kernel<kFp8><<<a.grid, kThreads, smem, s>>>(q_map, a);
   return cudaGetLastError();
+}
+
+cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s) {
+  return a.kv_dtype == MFA_KV_FP8_E4M3 ? launch_tc<true>(q_map, a, s) : launch_tc<false>(q_map, a, s);
 }
 
 }  // namespace mfa

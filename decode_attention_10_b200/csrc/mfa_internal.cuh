@@ -49,7 +49,7 @@ constexpr size_t kPartialBytes = kPartialFloats * sizeof(float);     // 66048 = 
 
 struct WsLayout {
   size_t err;          // uint32 error bits
-  size_t counters;     // int32 [kMaxBatch] arrival counters of the split-K merge
+  size_t seq_info;     // int2 [kMaxBatch]: (first partial slot, splits) per sequence
   size_t attn_part;    // partial slots
   size_t xproj_part;   // fp32 [kXProjSplits][batch][kXProjCols]
   size_t c_hat;        // bf16 [batch][kRank]
@@ -68,8 +68,8 @@ inline WsLayout ws_layout(int batch, int num_sms) {
   size_t off = 0;
   L.err = off;
   off += 256;
-  L.counters = off;
-  off = align_up(off + sizeof(int32_t) * kMaxBatch, 256);
+  L.seq_info = off;
+  off = align_up(off + 2 * sizeof(int32_t) * kMaxBatch, 256);
   L.attn_grid = attn_grid_for(num_sms);
   L.attn_slots = L.attn_grid + batch;  // sum over sequences of their splits <= grid + batch
   L.attn_part = off;
@@ -135,15 +135,18 @@ struct AttnArgs {
   uint16_t* out;            // [batch, 64, 256] bf16
   int batch;
   float* partials;          // slots
-  int32_t* counters;        // [batch]
+  int2* seq_info;           // [batch]: (first slot, splits), written for the combine kernel
   uint32_t* err;
   int grid;
 };
-cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s);  // CUDA-core kernel (FP8 KV)
-// Tensor-core kernel (bf16 KV); q_map covers q as [batch * 64 rows, 256] bf16, boxes of
-// [64 x 64] with 128-byte swizzle.
+// Tensor-core attention (bf16 or FP8 KV); q_map covers q as [batch * 64 rows, 256] bf16,
+// boxes of [64 x 64] with 128-byte swizzle.
 cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s);
 size_t attention_tc_smem_bytes();
+// Merge of the split-K partials of every split sequence (and zero output of rejected ones);
+// launched right after launch_attention_tc on the same stream, as its programmatic
+// dependent.
+cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s);
 
 // The query path (x-projection onto W_qdown, finish with RMSNorm, q_up) on `s`, using the
 // x-projection partials, c_hat and error word at the offsets of L inside `ws`.

@@ -235,3 +235,26 @@ def query_proj_noalloc(x, w_qdown, gamma, w_qup, eps: float = 1e-6, q_out=None, 
                                       float(eps), _ptr(q_out), bsz, _stream(stream)),
            "mfa_query_proj_noalloc")
     return q_out
+
+
+class DecodeStep:
+    """A decode step bound to fixed buffers, for serving loops: the ctypes arguments of
+    mfa_decode_layer are converted once, so each call costs one foreign call. The buffers
+    (x, weights, cache, seq_lens, q_out, out, workspace) must stay alive and in place; their
+    contents may change between calls (that is the point: new x, advanced seq_lens)."""
+
+    def __init__(self, x, w_qdown, gamma, w_qup, w_k, w_v, cache: KVCache, seq_lens,
+                 q_out, out, ws: Workspace, eps: float = 1e-6, scale: float = 1.0 / 16.0,
+                 stream=None):
+        self._lib = load()
+        self._keep = (x, w_qdown, gamma, w_qup, w_k, w_v, cache, seq_lens, q_out, out, ws)
+        self._args = (_P(_ptr(x)), _P(_ptr(w_qdown)), _P(_ptr(gamma)), _P(_ptr(w_qup)),
+                      _P(_ptr(w_k)), _P(_ptr(w_v)), ctypes.c_float(eps),
+                      ctypes.byref(cache.desc), _P(_ptr(seq_lens)), ctypes.c_float(scale),
+                      _P(_ptr(q_out)), _P(_ptr(out)), _P(ws.ptr), ctypes.c_size_t(ws.nbytes),
+                      _P(_stream(stream)))
+
+    def __call__(self):
+        st = self._lib.mfa_decode_layer(*self._args)
+        if st != 0:
+            raise MfaError(st, "mfa_decode_layer")
