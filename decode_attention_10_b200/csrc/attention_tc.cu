@@ -7,7 +7,7 @@
 // Because every head reads the same K/V rows, one pass over a sequence's cache serves all
 // 64 heads: each cached byte is read from HBM once and used 64 times on chip.
 //
-// Design (one persistent CTA per SM, warp-specialized):
+// Design (one persistent CTA per SM, warp-specialized, 320 threads):
 //   warp 0      TMA producer: Q of the current work item (4 boxes of [64 heads x 64 dims]),
 //               then K and V tiles of 128 positions as 16 KB boxes of [128 positions x 64
 //               dims] into a 10-slot shared-memory ring (128-byte swizzle).
@@ -15,17 +15,20 @@
 //                 S^T(t)[128 pos x 64 heads] = K(t)[128 x 256] . Q^T        (M=128, N=64)
 //                 O^T[256 dims x 64 heads] += V(t)^T[256 x 128] . P^T(t)    (2 x M=128, N=64)
 //               S^T is double-buffered in TMEM, so S(t+1) runs while the softmax of t does.
-//   warps 2..5  softmax, rescale and epilogue; thread = TMEM lane = one position of the tile
-//               (S^T) or one dimension of a half of O^T. Scores live in the log2 domain.
-//               The running max m per head is only raised when a tile's max exceeds it by
-//               more than 8 (a factor 256); otherwise exponents stay bounded and O needs no
-//               rescaling. P^T(t) is written to shared memory as bf16 (MN-major, swizzled).
+//   warps 2..9  softmax, rescale and epilogue, in two groups of four warps: group 0 owns
+//               heads 0..31, group 1 heads 32..63, of the same tile. Thread = TMEM lane =
+//               one position of the tile (S^T) or one dimension of a half of O^T. Scores
+//               live in the log2 domain. The running max m per head is only raised when a
+//               tile's max exceeds it by more than 8 (a factor 256); otherwise exponents stay
+//               bounded and O needs no rescaling. Each group writes its heads' half of the
+//               P^T(t) row (16-bit, MN-major, swizzled). The groups share no state, so
+//               neither waits for the other except through the MMA barriers.
 //   Tiles are windows of 128 positions; the last window of a work item ends at the item's
 //   end (it may start before the item or at a negative position, which TMA zero-fills), so
 //   rows past a sequence's length are never read. Positions outside the item are masked.
 // FP8 caches: TMA brings raw e4m3 boxes of [128 positions x 128 dims] into a 4-slot ring;
-// the softmax warps convert them (e4m3 -> f16 is exact) into the same swizzled 16 KB chunks
-// the bf16 path uses (a 6-slot ring), and both products run with f16 operands: Q is
+// the eight softmax warps convert them (e4m3 -> f16 is exact) into the same swizzled 16 KB
+// chunks the bf16 path uses (a 6-slot ring), and both products run with f16 operands: Q is
 // converted to f16 in place once per item (scaled by a power of two if its magnitude could
 // overflow f16), P is written as f16. The K and V scales fold into the softmax scale and
 // the output scale.
@@ -45,29 +48,32 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kChunkBytes = 16384;     // [128 positions x 64 dims] 16-bit, 128-byte swizzle
+constexpr int kThreads = 320;
+constexpr int kSoftmaxWarps = 8;        // warps 2..9
+constexpr int kGroupThreads = 128;      // one softmax group = four warps = the 128 lanes
+constexpr int kGroupHeads = 32;         // heads per group
+constexpr int kChunkBytes = 16384;      // [128 positions x 64 dims] 16-bit, 128-byte swizzle
 constexpr int kRingBytes = 10 * kChunkBytes;
-constexpr int kRawSlots = 4;           // FP8: raw e4m3 boxes [128 positions x 128 dims]
+constexpr int kRawSlots = 4;            // FP8: raw e4m3 boxes [128 positions x 128 dims]
 constexpr int kRawBytes = 16384;
 constexpr int kMaxSlots = 10;
-constexpr int kQChunkBytes = 8192;     // [64 heads x 64 dims] bf16
-constexpr int kPBytes = 16384;         // P^T: [128 positions x 64 heads] bf16
+constexpr int kQChunkBytes = 8192;      // [64 heads x 64 dims] 16-bit
+constexpr int kPBytes = 16384;          // P^T: [128 positions x 64 heads] 16-bit
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kTmemS = 0;         // S^T buffers: columns [0, 64) and [64, 128)
-constexpr uint32_t kTmemO = 128;       // O^T halves: columns [128, 192) and [192, 256)
+constexpr uint32_t kTmemS = 0;          // S^T buffers: columns [0, 64) and [64, 128)
+constexpr uint32_t kTmemO = 128;        // O^T halves: columns [128, 192) and [192, 256)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// named barriers: 1 + group among one softmax group, 3 among all eight softmax warps
+constexpr uint32_t kBarAllSoftmax = 3;
 
 // Per cache type: the MMA operand ring (chunks of [128 positions x 64 dims], 16-bit), where
-// it sits in the ring area, the operand type, and the L2 prefetch distance.
+// it sits in the ring area, and the operand type.
 template <bool kFp8>
 struct Cfg {
   static constexpr int kSlots = kFp8 ? 6 : 10;  // even: a V half-tile's 2 chunks are adjacent
   static constexpr int kRingOff = kFp8 ? kRawSlots * kRawBytes : 0;
   static constexpr bool kBf16 = !kFp8;           // operands: bf16, or f16 for FP8 caches
-  static constexpr int kPrefetchTiles = kFp8 ? 4 : 2;
   static constexpr uint32_t kIdescS = idesc_f16(128, 64, kBf16, false, false);  // K x Q^T
   static constexpr uint32_t kIdescPV = idesc_f16(128, 64, kBf16, true, true);   // V^T x P^T
 };
@@ -82,6 +88,7 @@ struct __align__(1024) TcSmem {
   float alpha[kHeads];
   float red[4][kHeads];
   float lsum[kHeads];
+  float qmax[kSoftmaxWarps];
   uint64_t kv_full[kMaxSlots];
   uint64_t kv_empty[kMaxSlots];
   uint64_t raw_full[kRawSlots];
@@ -93,7 +100,6 @@ struct __align__(1024) TcSmem {
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort_flag;
-  int32_t q_exp;  // FP8: Q was scaled by 2^-q_exp on conversion to f16
 };
 
 template <bool kFp8>
@@ -155,45 +161,42 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Sum 64 per-lane values over the 32 lanes of the warp: afterwards lane l holds the sums of
-// entries 2l (in v[0]) and 2l + 1 (in v[1]). Each step exchanges half of the live entries
-// with the partner lane (bit 4, 3, 2, 1, 0 of the lane id) and keeps the half it owns.
-__device__ __forceinline__ void warp_transpose_sum64(float (&v)[64], int lane) {
+// Sum 32 per-lane values over the 32 lanes of the warp: afterwards lane l holds the sum of
+// entry l in v[0]. Each step exchanges half of the live entries with the partner lane (bit
+// 4, 3, 2, 1, 0 of the lane id) and keeps the half it owns.
+__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
+  for (int i = 0; i < 16; ++i) {
     const bool up = lane & 16;
-    const float send = up ? v[i] : v[i + 32];
-    const float keep = up ? v[i + 32] : v[i];
+    const float send = up ? v[i] : v[i + 16];
+    const float keep = up ? v[i + 16] : v[i];
     v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
   }
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const bool up = lane & 8;
-    const float send = up ? v[i] : v[i + 16];
-    const float keep = up ? v[i + 16] : v[i];
+    const float send = up ? v[i] : v[i + 8];
+    const float keep = up ? v[i + 8] : v[i];
     v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < 4; ++i) {
     const bool up = lane & 4;
-    const float send = up ? v[i] : v[i + 8];
-    const float keep = up ? v[i + 8] : v[i];
+    const float send = up ? v[i] : v[i + 4];
+    const float keep = up ? v[i + 4] : v[i];
     v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const bool up = lane & 2;
-    const float send = up ? v[i] : v[i + 4];
-    const float keep = up ? v[i + 4] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-  }
-#pragma unroll
   for (int i = 0; i < 2; ++i) {
-    const bool up = lane & 1;
+    const bool up = lane & 2;
     const float send = up ? v[i] : v[i + 2];
     const float keep = up ? v[i + 2] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
   }
+  const bool up = lane & 1;
+  const float send = up ? v[0] : v[1];
+  const float keep = up ? v[1] : v[0];
+  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -202,11 +205,29 @@ __device__ __forceinline__ void warp_transpose_sum64(float (&v)[64], int lane) {
 template <bool kFp8>
 __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs& a, int g) {
   using C = Cfg<kFp8>;
+  constexpr int kBoxes = kFp8 ? 2 : 4;      // boxes per K or V tile
+  constexpr int kBoxX = kFp8 ? 128 : 64;    // elements per box row
+  constexpr uint32_t kN = kFp8 ? kRawSlots : C::kSlots;
   volatile int* abort = &S.abort_flag;
   uint32_t chunk = 0, issued = 0;
   int item = 0, q_issued = 0;
   prefetch_tensormap(q_map);
-  plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem& it) {
+
+  // the current work item and the next one, whose tensor maps are fetched while the
+  // current one streams
+  PlanCursor cur = plan_begin(S.plan, a.batch, g);
+  WorkItem it, nx;
+  bool has = plan_get(S.plan, a.batch, cur, it);
+  bool has_nx = has && plan_get(S.plan, a.batch, cur, nx);
+  if (has) {
+    prefetch_tensormap(&a.kv[it.b].tmap_k);
+    prefetch_tensormap(&a.kv[it.b].tmap_v);
+  }
+  while (has) {
+    if (has_nx) {
+      prefetch_tensormap(&a.kv[nx.b].tmap_k);
+      prefetch_tensormap(&a.kv[nx.b].tmap_v);
+    }
     const KvSeq* seq = a.kv + it.b;
     const CUtensorMap* km = &seq->tmap_k;
     const CUtensorMap* vm = &seq->tmap_v;
@@ -222,8 +243,6 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     auto load_tile = [&](const CUtensorMap* m, int t) {
       int y, a0, e0;
       tile_window(it, t, y, a0, e0);
-      constexpr int kBoxes = kFp8 ? 2 : 4;
-      constexpr uint32_t kN = kFp8 ? kRawSlots : C::kSlots;
       for (int c = 0; c < kBoxes; ++c) {
         const uint32_t slot = chunk % kN, use = chunk / kN;
         uint64_t* empty = kFp8 ? &S.raw_empty[slot] : &S.kv_empty[slot];
@@ -232,36 +251,24 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
         if (!*abort) {
           mbar_arrive_expect_tx(full, kChunkBytes);
           uint8_t* dst = kFp8 ? raw_box(S, slot) : ring_chunk<kFp8>(S, slot);
-          tma_load_2d(dst, m, (kFp8 ? 128 : 64) * c, y, full);
+          tma_load_2d(dst, m, kBoxX * c, y, full);
           issued = chunk + 1;
         }
         ++chunk;
       }
     };
-    // L2 prefetch runs kPrefetchTiles ahead of the loads, so that the shared-memory ring
-    // only has to cover L2 latency
-    auto prefetch_tile = [&](int t) {
-      if (t >= n || *abort) return;
-      int y, a0, e0;
-      tile_window(it, t, y, a0, e0);
-      constexpr int kBoxes = kFp8 ? 2 : 4;
-      for (int c = 0; c < kBoxes; ++c) {
-        tma_prefetch_2d(km, (kFp8 ? 128 : 64) * c, y);
-        tma_prefetch_2d(vm, (kFp8 ? 128 : 64) * c, y);
-      }
-    };
-    for (int t = 0; t < C::kPrefetchTiles; ++t) prefetch_tile(t);
     load_tile(km, 0);
     for (int t = 0; t < n; ++t) {
       if (t + 1 < n) load_tile(km, t + 1);
       load_tile(vm, t);
-      prefetch_tile(t + C::kPrefetchTiles);
     }
     ++item;
-  });
+    it = nx;
+    has = has_nx;
+    if (has) has_nx = plan_get(S.plan, a.batch, cur, nx);
+  }
   // Before the CTA may exit, every copy it started must have landed.
   if (*abort) {
-    constexpr uint32_t kN = kFp8 ? kRawSlots : C::kSlots;
     for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
       mbar_wait_drain(kFp8 ? &S.raw_full[c % kN] : &S.kv_full[c % kN], (c / kN) & 1);
     if (q_issued > 0) mbar_wait_drain(&S.q_full, (q_issued - 1) & 1);
@@ -352,12 +359,12 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
 }
 
 // ---------------------------------------------------------------------------------------
-// FP8 conversions, run by the 128 softmax threads
+// FP8 conversions, run by the eight softmax warps (256 threads, st = 0..255)
 // ---------------------------------------------------------------------------------------
 
 // Raw box `rbox` (e4m3, [128 positions x 128 dims], 128-byte swizzle) -> MMA ring chunks
 // `chunk` and `chunk + 1` (f16, [128 positions x 64 dims] each, same swizzle).
-__device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int tid, int lane,
+__device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int st, int lane,
                             volatile int* abort) {
   constexpr uint32_t kSlots = Cfg<true>::kSlots;
   const uint32_t rslot = rbox % kRawSlots;
@@ -369,8 +376,8 @@ __device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int tid, i
     if (fuse > 0) mbar_wait(&S.kv_empty[fslot], (fuse - 1) & 1, abort);
     uint8_t* dst = ring_chunk<true>(S, fslot);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int pc = tid + 128 * i;  // one 16-byte piece: 16 dims of one position
+    for (int i = 0; i < 2; ++i) {
+      const int pc = st + 256 * i;  // one 16-byte piece: 16 dims of one position
       const int r = pc >> 2, jj = pc & 3, j = 4 * cc + jj, sw = r & 7;
       const uint4 v = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
       const uint2 h0 = e4m3x4_to_f16x4(v.x), h1 = e4m3x4_to_f16x4(v.y);
@@ -390,14 +397,14 @@ __device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int tid, i
 
 // Q of the current item (bf16, loaded by TMA) -> f16 in place, scaled by 2^-e where e >= 0
 // is the smallest exponent that keeps every |q| below 2^15. Returns e.
-__device__ int convert_q(TcSmem& S, int item, int tid, int warp, int lane, volatile int* abort) {
+__device__ int convert_q(TcSmem& S, int item, int st, int swarp, int lane, volatile int* abort) {
   mbar_wait(&S.q_full, item & 1, abort);
   uint4* q = reinterpret_cast<uint4*>(S.q[0]);
-  constexpr int kPieces = kHeads * kHeadDim / 8 / kSoftmaxThreads;  // 16 per thread
+  constexpr int kPieces = kHeads * kHeadDim / 8 / (32 * kSoftmaxWarps);  // 8 per thread
   float mx = 0.f;
 #pragma unroll
   for (int i = 0; i < kPieces; ++i) {
-    const uint4 v = q[tid + kSoftmaxThreads * i];
+    const uint4 v = q[st + 256 * i];
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k)
@@ -405,14 +412,16 @@ __device__ int convert_q(TcSmem& S, int item, int tid, int warp, int lane, volat
                            fabsf(__uint_as_float(w[k] & 0xFFFF0000u))));
   }
   mx = warp_max_f32(mx);
-  if (lane == 0) S.red[warp - 2][0] = mx;
-  named_bar_sync(1, kSoftmaxThreads);
-  const float m = fmaxf(fmaxf(S.red[0][0], S.red[1][0]), fmaxf(S.red[2][0], S.red[3][0]));
+  if (lane == 0) S.qmax[swarp] = mx;
+  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);
+  float m = 0.f;
+#pragma unroll
+  for (int w = 0; w < kSoftmaxWarps; ++w) m = fmaxf(m, S.qmax[w]);
   const int e = (m >= 32768.f && m <= 3.0e38f) ? ilogbf(m) - 14 : 0;
   const float sc = ldexpf(1.f, -e);
 #pragma unroll
   for (int i = 0; i < kPieces; ++i) {
-    uint4& ref = q[tid + kSoftmaxThreads * i];
+    uint4& ref = q[st + 256 * i];
     const uint4 v = ref;
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
     uint32_t o[4];
@@ -422,22 +431,27 @@ __device__ int convert_q(TcSmem& S, int item, int tid, int warp, int lane, volat
     ref = make_uint4(o[0], o[1], o[2], o[3]);
   }
   fence_proxy_async_smem();
-  named_bar_sync(1, kSoftmaxThreads);  // every thread has read red before it is reused
+  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);  // qmax is read before it is reused
   __syncwarp();
   if (lane == 0) mbar_arrive(&S.q_ready);
   return e;
 }
 
 // ---------------------------------------------------------------------------------------
-// warps 2..5: softmax, rescale, epilogue (and the FP8 conversions)
+// warps 2..9: softmax, rescale, epilogue (and the FP8 conversions)
 // ---------------------------------------------------------------------------------------
 template <bool kFp8>
 __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
   volatile int* abort = &S.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tid = threadIdx.x - 64;        // 0..127
-  const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-  const int row = quad * 32 + lane;        // tile position / O^T row of this thread
+  const int swarp = warp - 2;                // 0..7
+  const int group = swarp >> 2;              // 0: heads 0..31, 1: heads 32..63
+  const int st = threadIdx.x - 64;           // 0..255 (conversions)
+  const int gt_id = st & 127;                // thread within the group
+  const uint32_t gbar = 1 + group;           // the group's named barrier
+  const int h0 = group * kGroupHeads;
+  const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
+  const int row = quad * 32 + lane;          // tile position / O^T row of this thread
   const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
   const float s_mul0 = a.scale * kLog2e * (kFp8 ? a.k_scale : 1.f);
   const float v_mul = kFp8 ? a.v_scale : 1.f;
@@ -448,17 +462,16 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
 
   plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem& it) {
     const int n = num_tiles(it);
-    // this warp's running row sums of heads 2*lane and 2*lane + 1
-    float l0 = 0.f, l1 = 0.f;
+    float lsum_w = 0.f;  // this warp's running row sum of head h0 + lane
     float s_mul = s_mul0;
     auto convert_tile = [&]() {  // one K or V tile: two raw boxes -> four ring chunks
-      convert_box(S, rbox, fchunk, tid, lane, abort);
-      convert_box(S, rbox + 1, fchunk + 2, tid, lane, abort);
+      convert_box(S, rbox, fchunk, st, lane, abort);
+      convert_box(S, rbox + 1, fchunk + 2, st, lane, abort);
       rbox += 2;
       fchunk += 4;
     };
     if constexpr (kFp8) {
-      s_mul = s_mul0 * ldexpf(1.f, convert_q(S, item, tid, warp, lane, abort));
+      s_mul = s_mul0 * ldexpf(1.f, convert_q(S, item, st, swarp, lane, abort));
       convert_tile();  // K(0)
     }
 
@@ -475,67 +488,68 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
 
       mbar_wait(&S.s_full[j], k & 1, abort);
       tc_fence_after();
-      uint32_t sr[kHeads];
-      tmem_ld_32x32b_x64(tmem + lane_addr + kTmemS + 64 * j, sr);
+      uint32_t sr[kGroupHeads];
+      tmem_ld_32x32b_x32(tmem + lane_addr + kTmemS + 64 * j + h0, sr);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.s_free[j]);
 
-      float s[kHeads];
+      float s[kGroupHeads];
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) s[h] = valid ? __uint_as_float(sr[h]) * s_mul : -INFINITY;
+      for (int h = 0; h < kGroupHeads; ++h)
+        s[h] = valid ? __uint_as_float(sr[h]) * s_mul : -INFINITY;
 
       bool need = (t == 0);
       if (!need) {
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) need |= s[h] > S.m_used[h] + kRescaleThreshold;
+        for (int h = 0; h < kGroupHeads; ++h) need |= s[h] > S.m_used[h0 + h] + kRescaleThreshold;
       }
-      if (named_bar_or(1, kSoftmaxThreads, need)) {
+      if (named_bar_or(gbar, kGroupThreads, need)) {
         // exact per-head max of this tile across the 128 positions
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
+        for (int h = 0; h < kGroupHeads; ++h) {
           const float r = warp_max_f32(s[h]);
-          if (lane == 0) S.red[warp - 2][h] = r;
+          if (lane == 0) S.red[quad][h0 + h] = r;
         }
-        named_bar_sync(1, kSoftmaxThreads);
-        if (tid < kHeads) {
-          const float mt = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]),
-                                 fmaxf(S.red[2][tid], S.red[3][tid]));
-          const float mo = t == 0 ? -INFINITY : S.m_used[tid];
+        named_bar_sync(gbar, kGroupThreads);
+        if (gt_id < kGroupHeads) {
+          const int hh = h0 + gt_id;
+          const float mt = fmaxf(fmaxf(S.red[0][hh], S.red[1][hh]), fmaxf(S.red[2][hh], S.red[3][hh]));
+          const float mo = t == 0 ? -INFINITY : S.m_used[hh];
           const float mn = fmaxf(mo, mt);
-          S.alpha[tid] = exp2f(mo - mn);
-          S.m_used[tid] = mn;
+          S.alpha[hh] = exp2f(mo - mn);
+          S.m_used[hh] = mn;
         }
-        named_bar_sync(1, kSoftmaxThreads);
+        named_bar_sync(gbar, kGroupThreads);
         if (t > 0) {
-          l0 *= S.alpha[2 * lane];
-          l1 *= S.alpha[2 * lane + 1];
+          lsum_w *= S.alpha[h0 + lane];
           // O must hold PV(t-1) before it is rescaled
           mbar_wait(&S.p_free, (tile - 1) & 1, abort);
           tc_fence_after();
 #pragma unroll 1
           for (int hf = 0; hf < 2; ++hf) {
-            uint32_t o[kHeads];
-            const uint32_t addr = tmem + lane_addr + kTmemO + 64 * hf;
-            tmem_ld_32x32b_x64(addr, o);
+            uint32_t o[kGroupHeads];
+            const uint32_t addr = tmem + lane_addr + kTmemO + 64 * hf + h0;
+            tmem_ld_32x32b_x32(addr, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < kHeads; ++h)
-              o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h]);
-            tmem_st_32x32b_x64(addr, o);
+            for (int h = 0; h < kGroupHeads; ++h)
+              o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h0 + h]);
+            tmem_st_32x32b_x32(addr, o);
           }
           tmem_wait_st();
         }
       }
 
       // probabilities (rounded to the operand type the tensor core reads: bf16, or f16
-      // for FP8 caches), the P^T row of this position, and the row sums of the rounded values
-      uint32_t pk[kHeads / 2];
+      // for FP8 caches), this group's half of the P^T row, and the row sums of the rounded
+      // values
+      uint32_t pk[kGroupHeads / 2];
 #pragma unroll
-      for (int h = 0; h < kHeads; h += 2) {
-        const float p0 = ex2(s[h] - S.m_used[h]);
-        const float p1 = ex2(s[h + 1] - S.m_used[h + 1]);
+      for (int h = 0; h < kGroupHeads; h += 2) {
+        const float p0 = ex2(s[h] - S.m_used[h0 + h]);
+        const float p1 = ex2(s[h + 1] - S.m_used[h0 + h + 1]);
         if constexpr (kFp8) {
           const uint32_t w = pack_f16x2(p0, p1);
           pk[h / 2] = w;
@@ -548,15 +562,14 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
           s[h + 1] = __uint_as_float(w & 0xFFFF0000u);
         }
       }
-      warp_transpose_sum64(s, lane);
-      l0 += s[0];
-      l1 += s[1];
+      lsum_w += warp_transpose_sum32(s, lane);
       // the P^T buffer is free once PV(t-1) has read it
       if (tile >= 1) mbar_wait(&S.p_free, (tile - 1) & 1, abort);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
+        const int cl = 4 * group + c;  // logical 16-byte chunk of the 128-byte row
         uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(p_row + ((c ^ (row & 7)) << 4)) = v;
+        *reinterpret_cast<uint4*>(p_row + ((cl ^ (row & 7)) << 4)) = v;
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -565,33 +578,35 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     }
     gt += n;
 
-    // ---- epilogue of the item ----
-    // row sums: the four warps' partial sums through shared memory
-    S.red[warp - 2][2 * lane] = l0;
-    S.red[warp - 2][2 * lane + 1] = l1;
-    named_bar_sync(1, kSoftmaxThreads);
-    if (tid < kHeads) S.lsum[tid] = S.red[0][tid] + S.red[1][tid] + S.red[2][tid] + S.red[3][tid];
+    // ---- epilogue of the item (each group for its heads) ----
+    S.red[quad][h0 + lane] = lsum_w;
+    named_bar_sync(gbar, kGroupThreads);
+    if (gt_id < kGroupHeads) {
+      const int hh = h0 + gt_id;
+      S.lsum[hh] = S.red[0][hh] + S.red[1][hh] + S.red[2][hh] + S.red[3][hh];
+    }
     // O^T holds PV of the last tile once its commit has landed
     mbar_wait(&S.p_free, (gt - 1) & 1, abort);
     tc_fence_after();
-    // one decision for all 128 threads, so they all take the same barriers below
-    const bool ok = !named_bar_or(1, kSoftmaxThreads, *abort != 0);
+    // one decision for the whole group, so that all its threads take the same barriers
+    const bool ok = !named_bar_or(gbar, kGroupThreads, *abort != 0);
     uint16_t* out = a.out + (size_t)it.b * kQWidth;
     float* pacc = it.slot >= 0 ? partial_acc(a.partials, it.slot) : nullptr;
 #pragma unroll 1
     for (int hf = 0; hf < 2; ++hf) {
-      uint32_t o[kHeads];
-      tmem_ld_32x32b_x64(tmem + lane_addr + kTmemO + 64 * hf, o);
+      uint32_t o[kGroupHeads];
+      tmem_ld_32x32b_x32(tmem + lane_addr + kTmemO + 64 * hf + h0, o);
       tmem_wait_ld();
       const int d = hf * 128 + row;
       if (ok) {
         if (it.slot < 0) {
 #pragma unroll
-          for (int h = 0; h < kHeads; ++h)
-            out[h * kHeadDim + d] = f32_to_bf16_bits(__uint_as_float(o[h]) * (v_mul / S.lsum[h]));
+          for (int h = 0; h < kGroupHeads; ++h)
+            out[(h0 + h) * kHeadDim + d] =
+                f32_to_bf16_bits(__uint_as_float(o[h]) * (v_mul / S.lsum[h0 + h]));
         } else {
 #pragma unroll
-          for (int h = 0; h < kHeads; ++h) pacc[h * kHeadDim + d] = __uint_as_float(o[h]);
+          for (int h = 0; h < kGroupHeads; ++h) pacc[(h0 + h) * kHeadDim + d] = __uint_as_float(o[h]);
         }
       }
     }
@@ -599,11 +614,12 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.o_free);
 
-    if (it.slot >= 0 && ok && tid < kHeads) {
-      partial_m(a.partials, it.slot)[tid] = S.m_used[tid];
-      partial_l(a.partials, it.slot)[tid] = S.lsum[tid];
+    if (it.slot >= 0 && ok && gt_id < kGroupHeads) {
+      partial_m(a.partials, it.slot)[h0 + gt_id] = S.m_used[h0 + gt_id];
+      partial_l(a.partials, it.slot)[h0 + gt_id] = S.lsum[h0 + gt_id];
     }
-    // m_used / lsum are rewritten by the next item only after its first barrier
+    // m_used / lsum / red of this group's heads are rewritten by the next item only after
+    // the group's next barrier
     ++item;
   });
 }
@@ -619,23 +635,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < Cfg<kFp8>::kSlots; ++i) {
-      mbar_init(&S.kv_full[i], kFp8 ? 4 : 1);  // FP8: the four converting warps arrive
+      mbar_init(&S.kv_full[i], kFp8 ? kSoftmaxWarps : 1);  // FP8: the converting warps arrive
       mbar_init(&S.kv_empty[i], 1);
     }
     for (int i = 0; i < kRawSlots; ++i) {
       mbar_init(&S.raw_full[i], 1);
-      mbar_init(&S.raw_empty[i], 4);
+      mbar_init(&S.raw_empty[i], kSoftmaxWarps);
     }
     mbar_init(&S.q_full, 1);
     mbar_init(&S.q_empty, 1);
-    mbar_init(&S.q_ready, 4);
+    mbar_init(&S.q_ready, kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_free[i], 4);
+      mbar_init(&S.s_free[i], kSoftmaxWarps);
     }
-    mbar_init(&S.p_full, 4);
+    mbar_init(&S.p_full, kSoftmaxWarps);
     mbar_init(&S.p_free, 1);
-    mbar_init(&S.o_free, 4);
+    mbar_init(&S.o_free, kSoftmaxWarps);
     mbar_init(&S.mma_done, 1);
     S.abort_flag = 0;
     fence_mbar_init();

@@ -120,33 +120,57 @@ struct WorkItem {
   int nsplit;   // CTAs sharing the sequence
 };
 
-// Call f(item) for every work item of CTA g, in order.
-template <class F>
-__device__ inline void plan_for_each_item(const PlanSmem& P, int batch, int g, F&& f) {
+// Walk over the work items of CTA g, in order: begin, then get until it returns false.
+struct PlanCursor {
+  int b;   // next sequence to look at
+  int t0;  // the CTA's tile range [t0, t1)
+  int t1;
+  int g;   // the CTA
+};
+
+__device__ inline PlanCursor plan_begin(const PlanSmem& P, int batch, int g) {
+  PlanCursor c{batch, 0, 0, g};
   const int NT = P.tile_start[batch];
   const int G = P.grid;
-  if (NT == 0 || g >= G) return;
-  const int t0 = plan_bound(g, G, NT), t1 = plan_bound(g + 1, G, NT);
-  if (t0 >= t1) return;
+  if (NT == 0 || g >= G) return c;
+  c.t0 = plan_bound(g, G, NT);
+  c.t1 = plan_bound(g + 1, G, NT);
   // largest b with tile_start[b] <= t0 (that sequence contains tile t0)
   int lo = 0, hi = batch - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (P.tile_start[mid] <= t0) lo = mid; else hi = mid - 1;
+    if (P.tile_start[mid] <= c.t0) lo = mid; else hi = mid - 1;
   }
-  for (int b = lo; b < batch && P.tile_start[b] < t1; ++b) {
+  c.b = lo;
+  return c;
+}
+
+__device__ inline bool plan_get(const PlanSmem& P, int batch, PlanCursor& c, WorkItem& it) {
+  const int NT = P.tile_start[batch];
+  const int G = P.grid;
+  for (; c.b < batch && P.tile_start[c.b] < c.t1; ++c.b) {
+    const int b = c.b;
     const int ts = P.tile_start[b], te = P.tile_start[b + 1];
-    if (te <= t0 || te == ts) continue;
-    const int a0 = max(ts, t0), a1 = min(te, t1);
-    WorkItem it;
+    if (te <= c.t0 || te == ts) continue;
+    const int a0 = max(ts, c.t0), a1 = min(te, c.t1);
     it.b = b;
     it.tok0 = (a0 - ts) * kTile;
     it.tok1 = min(P.len[b], (a1 - ts) * kTile);
     const int gf = plan_cta_of(ts, G, NT);
     it.nsplit = plan_cta_of(te - 1, G, NT) - gf + 1;
-    it.slot = it.nsplit > 1 ? P.slot_base[b] + (g - gf) : -1;
-    f(it);
+    it.slot = it.nsplit > 1 ? P.slot_base[b] + (c.g - gf) : -1;
+    ++c.b;
+    return true;
   }
+  return false;
+}
+
+// Call f(item) for every work item of CTA g, in order.
+template <class F>
+__device__ inline void plan_for_each_item(const PlanSmem& P, int batch, int g, F&& f) {
+  PlanCursor c = plan_begin(P, batch, g);
+  WorkItem it;
+  while (plan_get(P, batch, c, it)) f(it);
 }
 
 // Partial slot views.
