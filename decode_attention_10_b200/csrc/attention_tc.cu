@@ -223,6 +223,9 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     prefetch_tensormap(&a.kv[it.b].tmap_k);
     prefetch_tensormap(&a.kv[it.b].tmap_v);
   }
+  // q is written by the previous kernel of the step (the K/V rows, plan inputs and
+  // partial buffers only by kernels that have completed by the time this one launches)
+  pdl_wait();
   while (has) {
     if (has_nx) {
       prefetch_tensormap(&a.kv[nx.b].tmap_k);
@@ -706,6 +709,7 @@ constexpr int kCombineHeads = 4;
 
 __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
   pdl_wait();
+  pdl_launch_dependents();
   const int b = blockIdx.x, h0 = blockIdx.y * kCombineHeads, tid = threadIdx.x;
   const int2 info = a.seq_info[b];
   const int base = info.x, ns = info.y;
@@ -754,17 +758,8 @@ __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
 }  // namespace
 
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.batch, kHeads / kCombineHeads, 1);
-  cfg.blockDim = dim3(128, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, attention_combine_kernel, a);
+  return launch_pdl(attention_combine_kernel, dim3(a.batch, kHeads / kCombineHeads, 1), dim3(128),
+                    0, s, a);
 }
 
 size_t attention_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
@@ -775,8 +770,7 @@ static cudaError_t launch_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaSt
   cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<kFp8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attention_tc_kernel<kFp8><<<a.grid, kThreads, smem, s>>>(q_map, a);
-  return cudaGetLastError();
+  return launch_pdl(attention_tc_kernel<kFp8>, dim3(a.grid), dim3(kThreads), smem, s, q_map, a);
 }
 
 cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s) {

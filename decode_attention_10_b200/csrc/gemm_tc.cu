@@ -92,6 +92,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = C.tmem_base;
+  // X and the outputs belong to the previous kernels of the step
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -197,8 +200,7 @@ cudaError_t launch_wgemm(const CUtensorMap* w, const CUtensorMap& xmap, WGemmArg
       cudaFuncSetAttribute(wgemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(m_tiles, splits, (p.batch + 255) / 256);
-  wgemm_kernel<<<grid, kThreads, smem, s>>>(w[0], w[1], w[2], xmap, p);
-  return cudaGetLastError();
+  return launch_pdl(wgemm_kernel, grid, dim3(kThreads), smem, s, w[0], w[1], w[2], xmap, p);
 }
 
 }  // namespace mfa

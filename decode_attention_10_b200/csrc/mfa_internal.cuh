@@ -82,6 +82,27 @@ inline WsLayout ws_layout(int batch, int num_sms) {
   return L;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel on the stream is still running; it does its own set-up (barriers, TMEM, tensor-map
+// prefetch, the attention split plan) and then executes griddepcontrol.wait before it reads
+// anything the previous kernels of the step write. Every kernel of the step waits before it
+// triggers its own dependents, so "previous kernel complete" is transitive along the stream.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---------------------------------------------------------------------------------------
 // Kernel launchers (defined in the .cu files); all return cudaGetLastError().
 // ---------------------------------------------------------------------------------------

@@ -47,6 +47,8 @@ constexpr int kFinishQBlocks = kRank / 256;  // 8
 
 __global__ void __launch_bounds__(256) xproj_finish_kernel(FinishArgs a) {
   __shared__ float red[8];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
   const float* part = a.part + (size_t)b * kXProjCols;
   const size_t split_stride = (size_t)a.batch * kXProjCols;
@@ -99,8 +101,7 @@ __global__ void __launch_bounds__(256) xproj_finish_kernel(FinishArgs a) {
 }  // namespace
 
 cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s) {
-  xproj_finish_kernel<<<dim3(a.batch, kFinishQBlocks + 1), 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(xproj_finish_kernel, dim3(a.batch, kFinishQBlocks + 1), dim3(256), 0, s, a);
 }
 
 }  // namespace mfa
