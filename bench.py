@@ -59,6 +59,27 @@ def dist_env():
     return rank, world, local
 
 
+def rank_seed(wl, rank: int) -> int:
+    """Each rank draws its own sequences (weak scaling: sequences are sharded, weights are
+    replicated and drawn identically on every rank)."""
+    return 1000 + wl.index + 7919 * rank
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The slowest rank's time: every multi-GPU number is the max over ranks."""
+    if world <= 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(world: int, batch_per_rank: int, steps: int, t_ms: float) -> float:
+    """Tokens/s of the whole job: one token per sequence per step on every rank."""
+    return world * batch_per_rank * steps / (t_ms / 1e3)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -199,7 +220,7 @@ def run_ours(args, wl, rank, world, local):
     build.build()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    inp = W.generate_workload(wl, seed=1000 + wl.index + 7919 * rank)
+    inp = W.generate_workload(wl, seed=rank_seed(wl, rank))
     bsz = inp.batch
     step_bytes = WEIGHT_BYTES + kv_bytes(inp)
     copies = max(2, math.ceil(3 * L2_BYTES / step_bytes))
@@ -280,13 +301,9 @@ def run_ours(args, wl, rank, world, local):
         e1.record()
         torch.cuda.synchronize()
     barrier()
-    t_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([t_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_ms = float(t.item())
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     ms_per_step = t_ms / args.steps
-    value = world * bsz * args.steps / (t_ms / 1e3)
+    value = whole_job_throughput(world, bsz, args.steps, t_ms)
 
     # 2) the attention launch alone: K launches back to back over the rotating copies, CUDA
     #    events on the launching stream around the run (inter-launch gaps included)
@@ -320,12 +337,8 @@ def run_ours(args, wl, rank, world, local):
     e3.record()
     torch.cuda.synchronize()
     barrier()
-    t_e2e = e2.elapsed_time(e3)
-    if world > 1:
-        t = torch.tensor([t_e2e], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_e2e = float(t.item())
-    e2e_value = world * bsz * args.steps / (t_e2e / 1e3)
+    t_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
+    e2e_value = whole_job_throughput(world, bsz, args.steps, t_e2e)
 
     peak, peak_kind = measured_peaks()
     a_bytes = attention_bytes(inp)
