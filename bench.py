@@ -380,7 +380,8 @@ def run_ours(args, wl, rank, world, local):
     return result
 
 
-LAUNCHES_PER_LAYER = 4  # x-projection, split-K finish (+RMSNorm, append), q_up, attention
+LAUNCHES_PER_LAYER = 6  # split plan, x-projection, split-K finish (+RMSNorm, append), q_up,
+#                         attention, split combine
 
 
 def profiled_traffic(workload_name):

@@ -161,7 +161,9 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, i
 namespace {
 
 // The attention of one call: the tensor-core kernel, then the merge of split sequences.
+// Unless the plan was launched earlier (aa.plan_early), it is launched here first.
 mfa_status run_attention(const AttnArgs& aa, cudaStream_t s) {
+  if (!aa.plan_early && launch_attention_plan(aa, s) != cudaSuccess) return MFA_ERR_CUDA;
   CUtensorMap q_map;
   if (!encode_2d(&q_map, aa.q, (uint64_t)aa.batch * kHeads, kHeadDim, 2, 64, 64))
     return MFA_ERR_CUDA;
@@ -326,6 +328,8 @@ mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t*
   aa.batch = kv->batch;
   aa.partials = at<float>(ws, L.attn_part);
   aa.seq_info = at<int2>(ws, L.seq_info);
+  aa.plan = at<int32_t>(ws, L.plan);
+  aa.plan_early = 0;
   aa.err = at<uint32_t>(ws, L.err);
   aa.grid = L.attn_grid;
   return run_attention(aa, static_cast<cudaStream_t>(stream));
@@ -346,6 +350,25 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   if (st != MFA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int batch = kv->batch;
+  AttnArgs aa{};
+  aa.q = static_cast<const uint16_t*>(q_out);
+  aa.kv = static_cast<const KvSeq*>(kv->table);
+  aa.kv_dtype = kv->dtype;
+  aa.k_scale = kv->k_scale;
+  aa.v_scale = kv->v_scale;
+  aa.seq_lens = seq_lens;
+  aa.scale = scale;
+  aa.out = static_cast<uint16_t*>(out);
+  aa.batch = batch;
+  aa.partials = at<float>(ws, L.attn_part);
+  aa.seq_info = at<int2>(ws, L.seq_info);
+  aa.plan = at<int32_t>(ws, L.plan);
+  aa.plan_early = 1;
+  aa.err = at<uint32_t>(ws, L.err);
+  aa.grid = L.attn_grid;
+  // the split plan needs only seq_lens and the KV table: it runs first, and the attention
+  // kernel (four launches later) reads it before waiting on its predecessor
+  if (launch_attention_plan(aa, s) != cudaSuccess) return MFA_ERR_CUDA;
   // one projection of x onto [W_qdown | W_k | W_v]
   float* part = at<float>(ws, L.xproj_part);
   st = run_xproj(x, w_qdown, w_k, w_v, batch, 0, kXProjCols / 128, part,
@@ -368,20 +391,6 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
   st = run_q_up(fa.c_hat, w_qup, q_out, batch, fa.err, s);
   if (st != MFA_OK) return st;
-  AttnArgs aa{};
-  aa.q = static_cast<const uint16_t*>(q_out);
-  aa.kv = fa.kv;
-  aa.kv_dtype = kv->dtype;
-  aa.k_scale = kv->k_scale;
-  aa.v_scale = kv->v_scale;
-  aa.seq_lens = seq_lens;
-  aa.scale = scale;
-  aa.out = static_cast<uint16_t*>(out);
-  aa.batch = batch;
-  aa.partials = at<float>(ws, L.attn_part);
-  aa.seq_info = at<int2>(ws, L.seq_info);
-  aa.err = fa.err;
-  aa.grid = L.attn_grid;
   return run_attention(aa, s);
 }
 

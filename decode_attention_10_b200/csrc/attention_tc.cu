@@ -8,9 +8,10 @@
 // 64 heads: each cached byte is read from HBM once and used 64 times on chip.
 //
 // Design (one persistent CTA per SM, warp-specialized, 320 threads):
-//   warp 0      TMA producer: Q of the current work item (4 boxes of [64 heads x 64 dims]),
+//   warp 0      TMA producer: Q of each work item (4 boxes of [64 heads x 64 dims]; two Q
+//               buffers for bf16 caches, so the next item's Q loads while this one streams),
 //               then K and V tiles of 128 positions as 16 KB boxes of [128 positions x 64
-//               dims] into a 10-slot shared-memory ring (128-byte swizzle).
+//               dims] into a 6-slot shared-memory ring (128-byte swizzle).
 //   warp 1      TMEM owner and MMA issuer (one thread). Per tile t:
 //                 S^T(t)[128 pos x 64 heads] = K(t)[128 x 256] . Q^T        (M=128, N=64)
 //                 O^T[256 dims x 64 heads] += V(t)^T[256 x 128] . P^T(t)    (2 x M=128, N=64)
@@ -37,7 +38,6 @@
 // several CTAs leave (m, l, acc) partials that attention_combine_kernel merges.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 
 #include "attn_plan.cuh"
 #include "mfa_internal.cuh"
@@ -68,16 +68,21 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kBarAllSoftmax = 3;
 
 // Per cache type: the MMA operand ring (chunks of [128 positions x 64 dims], 16-bit), where
-// it sits in the ring area, and the operand type.
+// it sits in the ring area, the number of Q buffers, and the operand type. The ring area
+// holds, for bf16 caches, 6 ring chunks and the second Q buffer; for FP8 caches, the raw
+// e4m3 ring and 6 ring chunks.
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kSlots = kFp8 ? 6 : 10;  // even: a V half-tile's 2 chunks are adjacent
+  static constexpr int kSlots = 6;  // even: a V half-tile's 2 chunks are adjacent
   static constexpr int kRingOff = kFp8 ? kRawSlots * kRawBytes : 0;
+  static constexpr int kQBufs = kFp8 ? 1 : 2;
   static constexpr bool kBf16 = !kFp8;           // operands: bf16, or f16 for FP8 caches
   static constexpr uint32_t kIdescS = idesc_f16(128, 64, kBf16, false, false);  // K x Q^T
   static constexpr uint32_t kIdescPV = idesc_f16(128, 64, kBf16, true, true);   // V^T x P^T
 };
 static_assert(Cfg<true>::kRingOff + Cfg<true>::kSlots * kChunkBytes <= kRingBytes, "ring");
+constexpr int kQ1Off = Cfg<false>::kSlots * kChunkBytes;  // bf16: the second Q buffer
+static_assert(kQ1Off + 4 * kQChunkBytes <= kRingBytes, "second Q buffer");
 
 struct __align__(1024) TcSmem {
   uint8_t ring_area[kRingBytes];
@@ -93,7 +98,7 @@ struct __align__(1024) TcSmem {
   uint64_t kv_empty[kMaxSlots];
   uint64_t raw_full[kRawSlots];
   uint64_t raw_empty[kRawSlots];
-  uint64_t q_full, q_empty, q_ready;
+  uint64_t q_full[2], q_empty[2], q_ready;
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_free;
   uint64_t o_free;
@@ -108,6 +113,10 @@ __device__ __forceinline__ uint8_t* ring_chunk(TcSmem& S, uint32_t slot) {
 }
 __device__ __forceinline__ uint8_t* raw_box(TcSmem& S, uint32_t slot) {
   return S.ring_area + slot * kRawBytes;
+}
+// Q buffer qb: [4 chunks of 64 heads x 64 dims]
+__device__ __forceinline__ uint8_t* q_buf(TcSmem& S, int qb) {
+  return qb == 0 ? S.q[0] : S.ring_area + kQ1Off;
 }
 
 __device__ __forceinline__ int num_tiles(const WorkItem& it) {
@@ -145,14 +154,27 @@ __device__ __forceinline__ float f16_hi(uint32_t w) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
 }
 
-// four e4m3 codes (one 32-bit word, lowest byte first) -> two f16x2 words, exact
-__device__ __forceinline__ uint2 e4m3x4_to_f16x4(uint32_t w) {
-  const __half2_raw lo =
-      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xFFFFu), __NV_E4M3);
-  const __half2_raw hi =
-      __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
-  return make_uint2(static_cast<uint32_t>(lo.x) | (static_cast<uint32_t>(lo.y) << 16),
-                    static_cast<uint32_t>(hi.x) | (static_cast<uint32_t>(hi.y) << 16));
+// sixteen e4m3 codes (lowest byte first) -> sixteen f16 values in two 16-byte words, exact:
+// each 16-bit pair of codes becomes one f16x2 word (low byte -> low half)
+__device__ __forceinline__ void e4m3x16_to_f16x16(const uint4 v, uint4& o0, uint4& o1) {
+  asm("{\n"
+      ".reg .b16 c0, c1, c2, c3, c4, c5, c6, c7;\n"
+      "mov.b32 {c0, c1}, %8;\n"
+      "mov.b32 {c2, c3}, %9;\n"
+      "mov.b32 {c4, c5}, %10;\n"
+      "mov.b32 {c6, c7}, %11;\n"
+      "cvt.rn.f16x2.e4m3x2 %0, c0;\n"
+      "cvt.rn.f16x2.e4m3x2 %1, c1;\n"
+      "cvt.rn.f16x2.e4m3x2 %2, c2;\n"
+      "cvt.rn.f16x2.e4m3x2 %3, c3;\n"
+      "cvt.rn.f16x2.e4m3x2 %4, c4;\n"
+      "cvt.rn.f16x2.e4m3x2 %5, c5;\n"
+      "cvt.rn.f16x2.e4m3x2 %6, c6;\n"
+      "cvt.rn.f16x2.e4m3x2 %7, c7;\n"
+      "}\n"
+      : "=r"(o0.x), "=r"(o0.y), "=r"(o0.z), "=r"(o0.w), "=r"(o1.x), "=r"(o1.y), "=r"(o1.z),
+        "=r"(o1.w)
+      : "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -212,6 +234,8 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   uint32_t chunk = 0, issued = 0;
   int item = 0, q_issued = 0;
   prefetch_tensormap(q_map);
+  // every K/V byte is read once: keep it from evicting q and the split partials from L2
+  const uint64_t evict_first = policy_evict_first();
 
   // the current work item and the next one, whose tensor maps are fetched while the
   // current one streams
@@ -223,48 +247,64 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     prefetch_tensormap(&a.kv[it.b].tmap_k);
     prefetch_tensormap(&a.kv[it.b].tmap_v);
   }
-  // q is written by the previous kernel of the step (the K/V rows, plan inputs and
-  // partial buffers only by kernels that have completed by the time this one launches)
+  // Boxes of one item, in the order the MMA consumes them: K(0), then K(t+1), V(t) for each
+  // t, then V(n-1) -- 2 * n * kBoxes boxes in all.
+  auto issue_box = [&](const WorkItem& w, int j) {
+    const int n = num_tiles(w);
+    bool is_v;
+    int t, c;
+    if (j < kBoxes) {
+      is_v = false, t = 0, c = j;
+    } else {
+      const int r = j - kBoxes, tt = r / (2 * kBoxes), rr = r % (2 * kBoxes);
+      if (tt < n - 1)
+        is_v = rr >= kBoxes, t = is_v ? tt : tt + 1, c = is_v ? rr - kBoxes : rr;
+      else
+        is_v = true, t = n - 1, c = rr;
+    }
+    int y, a0, e0;
+    tile_window(w, t, y, a0, e0);
+    const KvSeq* seq = a.kv + w.b;
+    const uint32_t slot = chunk % kN, use = chunk / kN;
+    uint64_t* empty = kFp8 ? &S.raw_empty[slot] : &S.kv_empty[slot];
+    uint64_t* full = kFp8 ? &S.raw_full[slot] : &S.kv_full[slot];
+    if (use > 0) mbar_wait(empty, (use - 1) & 1, abort);
+    if (!*abort) {
+      mbar_arrive_expect_tx(full, kChunkBytes);
+      uint8_t* dst = kFp8 ? raw_box(S, slot) : ring_chunk<kFp8>(S, slot);
+      tma_load_2d_hint(dst, is_v ? &seq->tmap_v : &seq->tmap_k, kBoxX * c, y, full, evict_first);
+      issued = chunk + 1;
+    }
+    ++chunk;
+  };
+  // The K/V rows (and the split plan) were written by kernels that completed before this one
+  // launched, so the first ring-full of the first item streams in while the previous
+  // kernel (which writes q) finishes.
+  int first_done = 0;
+  if (has) {
+    const int total = 2 * num_tiles(it) * kBoxes;
+    first_done = total < static_cast<int>(kN) ? total : static_cast<int>(kN);
+    for (int j = 0; j < first_done; ++j) issue_box(it, j);
+  }
   pdl_wait();
   while (has) {
     if (has_nx) {
       prefetch_tensormap(&a.kv[nx.b].tmap_k);
       prefetch_tensormap(&a.kv[nx.b].tmap_v);
     }
-    const KvSeq* seq = a.kv + it.b;
-    const CUtensorMap* km = &seq->tmap_k;
-    const CUtensorMap* vm = &seq->tmap_v;
-    if (item > 0) mbar_wait(&S.q_empty, (item - 1) & 1, abort);
+    const int qb = item % C::kQBufs, qu = item / C::kQBufs;
+    if (qu > 0) mbar_wait(&S.q_empty[qb], (qu - 1) & 1, abort);
     if (!*abort) {
-      mbar_arrive_expect_tx(&S.q_full, 4 * kQChunkBytes);
-      for (int c = 0; c < 4; ++c) tma_load_2d(S.q[c], q_map, 64 * c, it.b * kHeads, &S.q_full);
+      mbar_arrive_expect_tx(&S.q_full[qb], 4 * kQChunkBytes);
+      uint8_t* qd = q_buf(S, qb);
+      for (int c = 0; c < 4; ++c)
+        tma_load_2d(qd + c * kQChunkBytes, q_map, 64 * c, it.b * kHeads, &S.q_full[qb]);
       q_issued = item + 1;
     }
-    const int n = num_tiles(it);
     // bf16: four [128 x 64] boxes per tile straight into the MMA ring; FP8: two raw
     // [128 x 128] e4m3 boxes per tile into the raw ring
-    auto load_tile = [&](const CUtensorMap* m, int t) {
-      int y, a0, e0;
-      tile_window(it, t, y, a0, e0);
-      for (int c = 0; c < kBoxes; ++c) {
-        const uint32_t slot = chunk % kN, use = chunk / kN;
-        uint64_t* empty = kFp8 ? &S.raw_empty[slot] : &S.kv_empty[slot];
-        uint64_t* full = kFp8 ? &S.raw_full[slot] : &S.kv_full[slot];
-        if (use > 0) mbar_wait(empty, (use - 1) & 1, abort);
-        if (!*abort) {
-          mbar_arrive_expect_tx(full, kChunkBytes);
-          uint8_t* dst = kFp8 ? raw_box(S, slot) : ring_chunk<kFp8>(S, slot);
-          tma_load_2d(dst, m, kBoxX * c, y, full);
-          issued = chunk + 1;
-        }
-        ++chunk;
-      }
-    };
-    load_tile(km, 0);
-    for (int t = 0; t < n; ++t) {
-      if (t + 1 < n) load_tile(km, t + 1);
-      load_tile(vm, t);
-    }
+    const int total = 2 * num_tiles(it) * kBoxes;
+    for (int j = (item == 0 ? first_done : 0); j < total; ++j) issue_box(it, j);
     ++item;
     it = nx;
     has = has_nx;
@@ -274,7 +314,8 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   if (*abort) {
     for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
       mbar_wait_drain(kFp8 ? &S.raw_full[c % kN] : &S.kv_full[c % kN], (c / kN) & 1);
-    if (q_issued > 0) mbar_wait_drain(&S.q_full, (q_issued - 1) & 1);
+    for (int i = (q_issued > C::kQBufs ? q_issued - C::kQBufs : 0); i < q_issued; ++i)
+      mbar_wait_drain(&S.q_full[i % C::kQBufs], (i / C::kQBufs) & 1);
   }
 }
 
@@ -289,11 +330,13 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
   uint32_t chunk = 0;
   uint32_t gt = 0;  // tiles issued so far by this CTA (all items)
   int item = 0;
-  const uint32_t q_base = smem_u32(S.q[0]);
+
   plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem& it) {
     const int n = num_tiles(it);
-    mbar_wait(kFp8 ? &S.q_ready : &S.q_full, item & 1, abort);
+    const int qb = item % C::kQBufs, qu = item / C::kQBufs;
+    mbar_wait(kFp8 ? &S.q_ready : &S.q_full[qb], qu & 1, abort);
     tc_fence_after();
+    const uint32_t q_base = smem_u32(q_buf(S, qb));
 
     auto issue_s = [&](uint32_t tile) {
       const uint32_t j = tile & 1, k = tile >> 1;
@@ -351,7 +394,7 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
       issue_s(gt + t);
       if (t >= 1) issue_pv(gt + t - 1, t - 1 == 0);
     }
-    if (!*abort) umma_commit(&S.q_empty);
+    if (!*abort) umma_commit(&S.q_empty[qb]);
     issue_pv(gt + n - 1, n == 1);
     gt += n;
     ++item;
@@ -383,12 +426,10 @@ __device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int st, in
       const int pc = st + 256 * i;  // one 16-byte piece: 16 dims of one position
       const int r = pc >> 2, jj = pc & 3, j = 4 * cc + jj, sw = r & 7;
       const uint4 v = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
-      const uint2 h0 = e4m3x4_to_f16x4(v.x), h1 = e4m3x4_to_f16x4(v.y);
-      const uint2 h2 = e4m3x4_to_f16x4(v.z), h3 = e4m3x4_to_f16x4(v.w);
-      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj) ^ sw) << 4)) =
-          make_uint4(h0.x, h0.y, h1.x, h1.y);
-      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj + 1) ^ sw) << 4)) =
-          make_uint4(h2.x, h2.y, h3.x, h3.y);
+      uint4 o0, o1;
+      e4m3x16_to_f16x16(v, o0, o1);
+      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj) ^ sw) << 4)) = o0;
+      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj + 1) ^ sw) << 4)) = o1;
     }
     fence_proxy_async_smem();
     __syncwarp();
@@ -401,7 +442,7 @@ __device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int st, in
 // Q of the current item (bf16, loaded by TMA) -> f16 in place, scaled by 2^-e where e >= 0
 // is the smallest exponent that keeps every |q| below 2^15. Returns e.
 __device__ int convert_q(TcSmem& S, int item, int st, int swarp, int lane, volatile int* abort) {
-  mbar_wait(&S.q_full, item & 1, abort);
+  mbar_wait(&S.q_full[0], item & 1, abort);
   uint4* q = reinterpret_cast<uint4*>(S.q[0]);
   constexpr int kPieces = kHeads * kHeadDim / 8 / (32 * kSoftmaxWarps);  // 8 per thread
   float mx = 0.f;
@@ -645,8 +686,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&S.raw_full[i], 1);
       mbar_init(&S.raw_empty[i], kSoftmaxWarps);
     }
-    mbar_init(&S.q_full, 1);
-    mbar_init(&S.q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.q_full[i], 1);
+      mbar_init(&S.q_empty[i], 1);
+    }
     mbar_init(&S.q_ready, kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
@@ -664,17 +707,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   pdl_launch_dependents();  // the combine kernel may start launching; it waits for us
-  plan_build(S.plan, a.seq_lens, a.kv, a.batch, a.grid, a.err, g == 0);
-  if (g == 0) {
-    // per sequence: its first partial slot and its number of splits (0 = rejected), for
-    // the combine kernel
-    const int NT = S.plan.tile_start[a.batch], G = S.plan.grid;
-    for (int b = threadIdx.x; b < a.batch; b += kThreads) {
-      const int ts = S.plan.tile_start[b], te = S.plan.tile_start[b + 1];
-      const int ns = te > ts ? plan_cta_of(te - 1, G, NT) - plan_cta_of(ts, G, NT) + 1 : 0;
-      a.seq_info[b] = make_int2(S.plan.slot_base[b], ns);
-    }
-  }
+  // the split plan, computed once per call by attention_plan_kernel
+  if (!a.plan_early) pdl_wait();
+  plan_load(S.plan, a.plan, a.batch);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -695,6 +730,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// plan: one block builds the split plan from seq_lens and the KV table, stores it for the
+// attention CTAs, and writes each sequence's (first partial slot, splits) for the combine
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) attention_plan_kernel(AttnArgs a) {
+  __shared__ PlanSmem P;
+  pdl_wait();
+  pdl_launch_dependents();
+  plan_build(P, a.seq_lens, a.kv, a.batch, a.grid, a.err, true);
+  plan_store(P, a.plan, a.batch);
+  const int NT = P.tile_start[a.batch], G = P.grid;
+  for (int b = threadIdx.x; b < a.batch; b += blockDim.x) {
+    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
+    const int ns = te > ts ? plan_cta_of(te - 1, G, NT) - plan_cta_of(ts, G, NT) + 1 : 0;
+    a.seq_info[b] = make_int2(P.slot_base[b], ns);
   }
 }
 
@@ -720,32 +773,30 @@ __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
   }
   if (ns == 1) return;
   const float v_mul = a.kv_dtype == MFA_KV_FP8_E4M3 ? a.v_scale : 1.f;
-  float M[kCombineHeads];
-#pragma unroll
-  for (int h = 0; h < kCombineHeads; ++h) M[h] = -INFINITY;
-#pragma unroll 4
-  for (int i = 0; i < ns; ++i) {
-    const float4 m = __ldcg(reinterpret_cast<const float4*>(partial_m(a.partials, base + i) + h0));
-    M[0] = fmaxf(M[0], m.x), M[1] = fmaxf(M[1], m.y), M[2] = fmaxf(M[2], m.z),
-    M[3] = fmaxf(M[3], m.w);
-  }
-  float L[kCombineHeads] = {0.f, 0.f, 0.f, 0.f};
+  // one pass with a running max per head: every split's loads are independent of the
+  // arithmetic, so several splits' worth stay in flight
+  float M[kCombineHeads], L[kCombineHeads];
   float2 o[kCombineHeads];
 #pragma unroll
-  for (int h = 0; h < kCombineHeads; ++h) o[h] = make_float2(0.f, 0.f);
+  for (int h = 0; h < kCombineHeads; ++h) M[h] = -INFINITY, L[h] = 0.f, o[h] = make_float2(0.f, 0.f);
 #pragma unroll 4
   for (int i = 0; i < ns; ++i) {
     const float4 m = __ldcg(reinterpret_cast<const float4*>(partial_m(a.partials, base + i) + h0));
     const float4 l = __ldcg(reinterpret_cast<const float4*>(partial_l(a.partials, base + i) + h0));
     const float* acc = partial_acc(a.partials, base + i) + h0 * kHeadDim + 2 * tid;
+    float2 x[kCombineHeads];
+#pragma unroll
+    for (int h = 0; h < kCombineHeads; ++h)
+      x[h] = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
     const float mm[4] = {m.x, m.y, m.z, m.w}, ll[4] = {l.x, l.y, l.z, l.w};
 #pragma unroll
     for (int h = 0; h < kCombineHeads; ++h) {
-      const float w = exp2f(mm[h] - M[h]);
-      const float2 x = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
-      L[h] = fmaf(ll[h], w, L[h]);
-      o[h].x = fmaf(w, x.x, o[h].x);
-      o[h].y = fmaf(w, x.y, o[h].y);
+      const float mn = fmaxf(M[h], mm[h]);
+      const float so = exp2f(M[h] - mn), si = exp2f(mm[h] - mn);
+      L[h] = fmaf(L[h], so, ll[h] * si);
+      o[h].x = fmaf(o[h].x, so, x[h].x * si);
+      o[h].y = fmaf(o[h].y, so, x[h].y * si);
+      M[h] = mn;
     }
   }
 #pragma unroll
@@ -756,6 +807,10 @@ __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
 }
 
 }  // namespace
+
+cudaError_t launch_attention_plan(const AttnArgs& a, cudaStream_t s) {
+  return launch_pdl(attention_plan_kernel, dim3(1), dim3(256), 0, s, a);
+}
 
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s) {
   return launch_pdl(attention_combine_kernel, dim3(a.batch, kHeads / kCombineHeads, 1), dim3(128),

@@ -112,6 +112,26 @@ __device__ inline void plan_build(PlanSmem& P, const int32_t* __restrict__ seq_l
   block_exclusive_scan(P.slot_base, batch, P.scan_tmp);
 }
 
+// The plan in global memory: tile_start[batch + 1], slot_base[batch], len[batch], grid, at
+// fixed offsets of a kPlanBytes buffer.
+__device__ inline void plan_store(const PlanSmem& P, int32_t* g, int batch) {
+  for (int i = threadIdx.x; i <= batch; i += blockDim.x) g[i] = P.tile_start[i];
+  for (int i = threadIdx.x; i < batch; i += blockDim.x) {
+    g[kMaxBatch + 1 + i] = P.slot_base[i];
+    g[2 * kMaxBatch + 1 + i] = P.len[i];
+  }
+  if (threadIdx.x == 0) g[3 * kMaxBatch + 1] = P.grid;
+}
+
+__device__ inline void plan_load(PlanSmem& P, const int32_t* __restrict__ g, int batch) {
+  for (int i = threadIdx.x; i <= batch; i += blockDim.x) P.tile_start[i] = g[i];
+  for (int i = threadIdx.x; i < batch; i += blockDim.x) {
+    P.slot_base[i] = g[kMaxBatch + 1 + i];
+    P.len[i] = g[2 * kMaxBatch + 1 + i];
+  }
+  if (threadIdx.x == 0) P.grid = g[3 * kMaxBatch + 1];
+}
+
 struct WorkItem {
   int b;        // sequence
   int tok0;     // first cached position of the item

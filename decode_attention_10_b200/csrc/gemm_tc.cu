@@ -92,33 +92,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = C.tmem_base;
-  // X and the outputs belong to the previous kernels of the step
-  pdl_wait();
-  pdl_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tensormap(wm);
       prefetch_tensormap(&xmap);
       const uint64_t evict_first = policy_evict_first();
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % stages, use = i / stages;
-        if (use > 0) mbar_wait(&C.empty[s], (use - 1) & 1, abort);
-        if (*abort) break;
-        mbar_arrive_expect_tx(&C.full[s], kATileBytes + b_bytes);
-        const int k = (kb0 + i) * kBK;
+      auto load_w = [&](int i) {
+        const int s = i % stages, k = (kb0 + i) * kBK;
         uint8_t* a = a_ring + (size_t)s * kATileBytes;
         tma_load_2d_hint(a, wm, n0, k, &C.full[s], evict_first);
         tma_load_2d_hint(a + kABoxBytes, wm, n0 + 64, k, &C.full[s], evict_first);
-        tma_load_2d(b_ring + (size_t)s * b_bytes, &xmap, k, b0, &C.full[s]);
+      };
+      // The weights depend on no earlier kernel: the first `stages` blocks of them stream in
+      // while the previous kernel of the step finishes. X (and the outputs) must wait.
+      const int early = stages < nkb ? stages : nkb;
+      for (int i = 0; i < early; ++i) {
+        mbar_arrive_expect_tx(&C.full[i], kATileBytes + b_bytes);
+        load_w(i);
+      }
+      pdl_wait();
+      pdl_launch_dependents();
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % stages, use = i / stages;
+        if (i >= early) {
+          if (use > 0) mbar_wait(&C.empty[s], (use - 1) & 1, abort);
+          if (*abort) break;
+          mbar_arrive_expect_tx(&C.full[s], kATileBytes + b_bytes);
+          load_w(i);
+        } else if (*abort) {
+          break;
+        }
+        tma_load_2d(b_ring + (size_t)s * b_bytes, &xmap, (kb0 + i) * kBK, b0, &C.full[s]);
         issued = i + 1;
       }
-      if (*abort)
-        for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i)
+      if (*abort) {
+        // stages armed early whose X box was never issued: release the missing bytes, so the
+        // phase completes once their weight boxes have landed
+        for (int i = issued; i < early; ++i) mbar_complete_tx(&C.full[i], b_bytes);
+        const int last = issued > early ? issued : early;
+        for (int i = (last > stages ? last - stages : 0); i < last; ++i)
           mbar_wait_drain(&C.full[i % stages], (i / stages) & 1);
+      }
+    } else {
+      pdl_wait();
+      pdl_launch_dependents();
     }
   } else if (warp == 1) {
+    pdl_wait();
+    pdl_launch_dependents();
     if (lane == 0) {
       const uint32_t idesc = idesc_f16(128, p.n_box, true, true, false);
       for (int i = 0; i < nkb; ++i) {
@@ -140,6 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait_drain(&C.acc_full, 0);
     }
   } else {
+    pdl_wait();
+    pdl_launch_dependents();
     // epilogue: thread = TMEM lane = output feature n0 + row
     const int quad = warp & 3;
     const int row = quad * 32 + lane;

@@ -47,9 +47,14 @@ static_assert(sizeof(KvSeq) == 384, "KvSeq layout");
 constexpr int kPartialFloats = kHeads + kHeads + kHeads * kHeadDim;  // 16512
 constexpr size_t kPartialBytes = kPartialFloats * sizeof(float);     // 66048 = 258 * 256
 
+// Bytes of the attention split plan kept in the workspace (tile_start[kMaxBatch + 1],
+// slot_base[kMaxBatch], len[kMaxBatch], grid).
+constexpr size_t kPlanBytes = sizeof(int32_t) * (3 * kMaxBatch + 2);
+
 struct WsLayout {
   size_t err;          // uint32 error bits
   size_t seq_info;     // int2 [kMaxBatch]: (first partial slot, splits) per sequence
+  size_t plan;         // the attention split plan (written by the plan kernel)
   size_t attn_part;    // partial slots
   size_t xproj_part;   // fp32 [kXProjSplits][batch][kXProjCols]
   size_t c_hat;        // bf16 [batch][kRank]
@@ -70,6 +75,8 @@ inline WsLayout ws_layout(int batch, int num_sms) {
   off += 256;
   L.seq_info = off;
   off = align_up(off + 2 * sizeof(int32_t) * kMaxBatch, 256);
+  L.plan = off;
+  off = align_up(off + kPlanBytes, 256);
   L.attn_grid = attn_grid_for(num_sms);
   L.attn_slots = L.attn_grid + batch;  // sum over sequences of their splits <= grid + batch
   L.attn_part = off;
@@ -157,9 +164,15 @@ struct AttnArgs {
   int batch;
   float* partials;          // slots
   int2* seq_info;           // [batch]: (first slot, splits), written for the combine kernel
+  int32_t* plan;            // the split plan, written by launch_attention_plan
+  int plan_early;           // 1: the plan was written two or more kernels earlier on the
+                            // stream, so it may be read before griddepcontrol.wait
   uint32_t* err;
   int grid;
 };
+// One block: the split plan of the attention (and the combine's per-sequence info) from
+// seq_lens and the KV table, written to a.plan / a.seq_info; reports rejected lengths.
+cudaError_t launch_attention_plan(const AttnArgs& a, cudaStream_t s);
 // Tensor-core attention (bf16 or FP8 KV); q_map covers q as [batch * 64 rows, 256] bf16,
 // boxes of [64 x 64] with 128-byte swizzle.
 cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s);
