@@ -70,9 +70,9 @@ mfa_status run_xproj(const void* x, const void* w_qdown, const void* w_k, const 
                      cudaStream_t s) {
   CUtensorMap wm[3];
   std::memset(wm, 0, sizeof(wm));
-  if (w_qdown && !encode_2d(&wm[0], w_qdown, kHidden, kRank, 2, 64, 64)) return MFA_ERR_CUDA;
-  if (w_k && !encode_2d(&wm[1], w_k, kHidden, kHeadDim, 2, 64, 64)) return MFA_ERR_CUDA;
-  if (w_v && !encode_2d(&wm[2], w_v, kHidden, kHeadDim, 2, 64, 64)) return MFA_ERR_CUDA;
+  if (w_qdown && !encode_2d(&wm[0], w_qdown, kHidden, kRank, 2, 64, 128)) return MFA_ERR_CUDA;
+  if (w_k && !encode_2d(&wm[1], w_k, kHidden, kHeadDim, 2, 64, 128)) return MFA_ERR_CUDA;
+  if (w_v && !encode_2d(&wm[2], w_v, kHidden, kHeadDim, 2, 64, 128)) return MFA_ERR_CUDA;
   CUtensorMap xm;
   if (!encode_2d(&xm, x, (uint64_t)batch, kHidden, 2, 64, wgemm_n_box(batch))) return MFA_ERR_CUDA;
   WGemmArgs p{};
@@ -81,7 +81,7 @@ mfa_status run_xproj(const void* x, const void* w_qdown, const void* w_k, const 
   p.three_weights = 1;
   p.w0_tiles = kRank / 128;
   p.w1_tiles = kHeadDim / 128;
-  p.kblocks_per_cta = kXProjKPerSplit / 64;
+  p.kblocks_per_cta = kXProjKPerSplit / 128;
   p.out_f32 = part;
   p.out_ld = kXProjCols;
   p.err = err;
@@ -93,7 +93,7 @@ mfa_status run_q_up(const uint16_t* c_hat, const void* w_qup, void* q, int batch
                     cudaStream_t s) {
   CUtensorMap wm[3];
   std::memset(wm, 0, sizeof(wm));
-  if (!encode_2d(&wm[0], w_qup, kRank, kQWidth, 2, 64, 64)) return MFA_ERR_CUDA;
+  if (!encode_2d(&wm[0], w_qup, kRank, kQWidth, 2, 64, 128)) return MFA_ERR_CUDA;
   CUtensorMap xm;
   if (!encode_2d(&xm, c_hat, (uint64_t)batch, kRank, 2, 64, wgemm_n_box(batch)))
     return MFA_ERR_CUDA;
@@ -101,7 +101,7 @@ mfa_status run_q_up(const uint16_t* c_hat, const void* w_qup, void* q, int batch
   p.batch = batch;
   p.tile_begin = 0;
   p.three_weights = 0;
-  p.kblocks_per_cta = kRank / 64;
+  p.kblocks_per_cta = kRank / 128;
   p.out_bf16 = static_cast<uint16_t*>(q);
   p.out_ld = kQWidth;
   p.err = err;

@@ -27,9 +27,12 @@
 //   Tiles are windows of 128 positions; the last window of a work item ends at the item's
 //   end (it may start before the item or at a negative position, which TMA zero-fills), so
 //   rows past a sequence's length are never read. Positions outside the item are masked.
-// FP8 caches: TMA brings raw e4m3 boxes of [128 positions x 128 dims] into a 4-slot ring;
-// the eight softmax warps convert them (e4m3 -> f16 is exact) into the same swizzled 16 KB
-// chunks the bf16 path uses (a 6-slot ring), and both products run with f16 operands: Q is
+// FP8 caches: TMA brings raw e4m3 boxes of [128 positions x 128 dims] into a 6-slot ring,
+// and the eight softmax warps convert them (e4m3 -> f16 is exact). A K tile goes straight
+// into tensor memory (two 128-column buffers), where the S^T product reads it as its A
+// operand; a V tile goes into the same swizzled 16 KB shared-memory chunks the bf16 path
+// uses (a 4-slot ring). Keeping K out of shared memory is what leaves room for a raw ring
+// deep enough to keep 96 KB of loads in flight. Both products run with f16 operands: Q is
 // converted to f16 in place once per item (scaled by a power of two if its magnitude could
 // overflow f16), P is written as f16. The K and V scales fold into the softmax scale and
 // the output scale.
@@ -54,27 +57,29 @@ constexpr int kGroupThreads = 128;      // one softmax group = four warps = the 
 constexpr int kGroupHeads = 32;         // heads per group
 constexpr int kChunkBytes = 16384;      // [128 positions x 64 dims] 16-bit, 128-byte swizzle
 constexpr int kRingBytes = 10 * kChunkBytes;
-constexpr int kRawSlots = 4;            // FP8: raw e4m3 boxes [128 positions x 128 dims]
+constexpr int kRawSlots = 6;            // FP8: raw e4m3 boxes [128 positions x 128 dims]
 constexpr int kRawBytes = 16384;
 constexpr int kMaxSlots = 10;
 constexpr int kQChunkBytes = 8192;      // [64 heads x 64 dims] 16-bit
 constexpr int kPBytes = 16384;          // P^T: [128 positions x 64 heads] 16-bit
-constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kTmemS = 0;          // S^T buffers: columns [0, 64) and [64, 128)
 constexpr uint32_t kTmemO = 128;        // O^T halves: columns [128, 192) and [192, 256)
+constexpr uint32_t kTmemK = 256;        // FP8: f16 K tiles (A operand), [256, 384), [384, 512)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // named barriers: 1 + group among one softmax group, 3 among all eight softmax warps
 constexpr uint32_t kBarAllSoftmax = 3;
 
-// Per cache type: the MMA operand ring (chunks of [128 positions x 64 dims], 16-bit), where
-// it sits in the ring area, the number of Q buffers, and the operand type. The ring area
-// holds, for bf16 caches, 6 ring chunks and the second Q buffer; for FP8 caches, the raw
-// e4m3 ring and 6 ring chunks.
+// Per cache type: the shared-memory operand ring (chunks of [128 positions x 64 dims],
+// 16-bit), where it sits in the ring area, the number of Q buffers, the tensor memory used,
+// and the operand type. The ring area holds, for bf16 caches, 6 ring chunks (K and V) and
+// the second Q buffer; for FP8 caches, the 6-box raw e4m3 ring and 4 ring chunks (V only:
+// converted K tiles go to tensor memory).
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kSlots = 6;  // even: a V half-tile's 2 chunks are adjacent
+  static constexpr int kSlots = kFp8 ? 4 : 6;  // even: a V half-tile's 2 chunks are adjacent
   static constexpr int kRingOff = kFp8 ? kRawSlots * kRawBytes : 0;
+  static constexpr uint32_t kTmemCols = kFp8 ? 512 : 256;
   static constexpr int kQBufs = kFp8 ? 1 : 2;
   static constexpr bool kBf16 = !kFp8;           // operands: bf16, or f16 for FP8 caches
   static constexpr uint32_t kIdescS = idesc_f16(128, 64, kBf16, false, false);  // K x Q^T
@@ -99,6 +104,7 @@ struct __align__(1024) TcSmem {
   uint64_t raw_full[kRawSlots];
   uint64_t raw_empty[kRawSlots];
   uint64_t q_full[2], q_empty[2], q_ready;
+  uint64_t k_full[2];  // FP8: K tile converted into tensor memory buffer 0 / 1
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_free;
   uint64_t o_free;
@@ -225,7 +231,8 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) 
 // warp 0: TMA producer
 // ---------------------------------------------------------------------------------------
 template <bool kFp8>
-__device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs& a, int g) {
+__device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs& a, int g,
+                             bool leader) {
   using C = Cfg<kFp8>;
   constexpr int kBoxes = kFp8 ? 2 : 4;      // boxes per K or V tile
   constexpr int kBoxX = kFp8 ? 128 : 64;    // elements per box row
@@ -233,7 +240,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   volatile int* abort = &S.abort_flag;
   uint32_t chunk = 0, issued = 0;
   int item = 0, q_issued = 0;
-  prefetch_tensormap(q_map);
+  if (leader) prefetch_tensormap(q_map);
   // every K/V byte is read once: keep it from evicting q and the split partials from L2
   const uint64_t evict_first = policy_evict_first();
 
@@ -243,7 +250,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   WorkItem it, nx;
   bool has = plan_get(S.plan, a.batch, cur, it);
   bool has_nx = has && plan_get(S.plan, a.batch, cur, nx);
-  if (has) {
+  if (has && leader) {
     prefetch_tensormap(&a.kv[it.b].tmap_k);
     prefetch_tensormap(&a.kv[it.b].tmap_v);
   }
@@ -270,9 +277,12 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     uint64_t* full = kFp8 ? &S.raw_full[slot] : &S.kv_full[slot];
     if (use > 0) mbar_wait(empty, (use - 1) & 1, abort);
     if (!*abort) {
-      mbar_arrive_expect_tx(full, kChunkBytes);
-      uint8_t* dst = kFp8 ? raw_box(S, slot) : ring_chunk<kFp8>(S, slot);
-      tma_load_2d_hint(dst, is_v ? &seq->tmap_v : &seq->tmap_k, kBoxX * c, y, full, evict_first);
+      if (leader) {
+        mbar_arrive_expect_tx(full, kChunkBytes);
+        uint8_t* dst = kFp8 ? raw_box(S, slot) : ring_chunk<kFp8>(S, slot);
+        tma_load_2d_hint(dst, is_v ? &seq->tmap_v : &seq->tmap_k, kBoxX * c, y, full,
+                         evict_first);
+      }
       issued = chunk + 1;
     }
     ++chunk;
@@ -288,17 +298,19 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   }
   pdl_wait();
   while (has) {
-    if (has_nx) {
+    if (has_nx && leader) {
       prefetch_tensormap(&a.kv[nx.b].tmap_k);
       prefetch_tensormap(&a.kv[nx.b].tmap_v);
     }
     const int qb = item % C::kQBufs, qu = item / C::kQBufs;
     if (qu > 0) mbar_wait(&S.q_empty[qb], (qu - 1) & 1, abort);
     if (!*abort) {
-      mbar_arrive_expect_tx(&S.q_full[qb], 4 * kQChunkBytes);
-      uint8_t* qd = q_buf(S, qb);
-      for (int c = 0; c < 4; ++c)
-        tma_load_2d(qd + c * kQChunkBytes, q_map, 64 * c, it.b * kHeads, &S.q_full[qb]);
+      if (leader) {
+        mbar_arrive_expect_tx(&S.q_full[qb], 4 * kQChunkBytes);
+        uint8_t* qd = q_buf(S, qb);
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(qd + c * kQChunkBytes, q_map, 64 * c, it.b * kHeads, &S.q_full[qb]);
+      }
       q_issued = item + 1;
     }
     // bf16: four [128 x 64] boxes per tile straight into the MMA ring; FP8: two raw
@@ -323,7 +335,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
 // warp 1 (one thread): MMA issue
 // ---------------------------------------------------------------------------------------
 template <bool kFp8>
-__device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
+__device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool leader) {
   using C = Cfg<kFp8>;
   constexpr uint32_t kSlots = C::kSlots;
   volatile int* abort = &S.abort_flag;
@@ -343,23 +355,40 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
       if (k > 0) mbar_wait(&S.s_free[j], (k - 1) & 1, abort);
       tc_fence_after();
       const uint32_t d = tmem + kTmemS + 64 * j;
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
-        mbar_wait(&S.kv_full[slot], use & 1, abort);
+      if constexpr (kFp8) {
+        // K(tile) in tensor memory buffer j (converted by the softmax warps)
+        mbar_wait(&S.k_full[j], k & 1, abort);
         tc_fence_after();
         if (!*abort) {
-          const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, slot));
+          const uint32_t a_tm = tmem + kTmemK + 128 * j;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
-            const uint64_t bd = sdesc_sw128(q_base + c * kQChunkBytes + 32 * kk, 16, 1024);
-            umma_f16_ss(d, ad, bd, C::kIdescS, (c | kk) != 0);
+          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
+            const uint64_t bd =
+                sdesc_sw128(q_base + (kk >> 2) * kQChunkBytes + 32 * (kk & 3), 16, 1024);
+            if (leader) umma_f16_ts(d, a_tm + 8 * kk, bd, C::kIdescS, kk != 0);
           }
-          umma_commit(&S.kv_empty[slot]);
+          if (leader) umma_commit(&S.s_full[j]);
         }
-        ++chunk;
+      } else {
+        // K(tile): four ring chunks of 64 dims
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
+          mbar_wait(&S.kv_full[slot], use & 1, abort);
+          tc_fence_after();
+          if (!*abort) {
+            const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, slot));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
+              const uint64_t bd = sdesc_sw128(q_base + c * kQChunkBytes + 32 * kk, 16, 1024);
+              if (leader) umma_f16_ss(d, ad, bd, C::kIdescS, (c | kk) != 0);
+            }
+            if (leader) umma_commit(&S.kv_empty[slot]);
+          }
+          ++chunk;
+        }
+        if (!*abort && leader) umma_commit(&S.s_full[j]);
       }
-      if (!*abort) umma_commit(&S.s_full[j]);
     };
 
     auto issue_pv = [&](uint32_t tile, bool first) {
@@ -380,27 +409,27 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
           for (int kt = 0; kt < kTile / 16; ++kt) {
             const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
             const uint64_t bd = sdesc_sw128(p_base + 2048 * kt, kPBytes, 1024);
-            umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+            if (leader) umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
           }
-          umma_commit(&S.kv_empty[s0]);
-          umma_commit(&S.kv_empty[s1]);
+          if (leader) umma_commit(&S.kv_empty[s0]);
+          if (leader) umma_commit(&S.kv_empty[s1]);
         }
       }
       chunk += 4;
-      if (!*abort) umma_commit(&S.p_free);
+      if (!*abort && leader) umma_commit(&S.p_free);
     };
 
     for (int t = 0; t < n; ++t) {
       issue_s(gt + t);
       if (t >= 1) issue_pv(gt + t - 1, t - 1 == 0);
     }
-    if (!*abort) umma_commit(&S.q_empty[qb]);
+    if (!*abort && leader) umma_commit(&S.q_empty[qb]);
     issue_pv(gt + n - 1, n == 1);
     gt += n;
     ++item;
   });
   // Every MMA issued must be complete before the tensor memory is released.
-  umma_commit(&S.mma_done);
+  if (leader) umma_commit(&S.mma_done);
   mbar_wait_drain(&S.mma_done, 0);
 }
 
@@ -408,35 +437,91 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
 // FP8 conversions, run by the eight softmax warps (256 threads, st = 0..255)
 // ---------------------------------------------------------------------------------------
 
-// Raw box `rbox` (e4m3, [128 positions x 128 dims], 128-byte swizzle) -> MMA ring chunks
-// `chunk` and `chunk + 1` (f16, [128 positions x 64 dims] each, same swizzle).
-__device__ void convert_box(TcSmem& S, uint32_t rbox, uint32_t chunk, int st, int lane,
-                            volatile int* abort) {
-  constexpr uint32_t kSlots = Cfg<true>::kSlots;
-  const uint32_t rslot = rbox % kRawSlots;
-  mbar_wait(&S.raw_full[rslot], (rbox / kRawSlots) & 1, abort);
-  const uint8_t* raw = raw_box(S, rslot);
-#pragma unroll 1
-  for (int cc = 0; cc < 2; ++cc) {
-    const uint32_t ch = chunk + cc, fslot = ch % kSlots, fuse = ch / kSlots;
-    if (fuse > 0) mbar_wait(&S.kv_empty[fslot], (fuse - 1) & 1, abort);
-    uint8_t* dst = ring_chunk<true>(S, fslot);
+// K(t) of an FP8 cache -> tensor memory buffer `buf` as the A operand of S^T = K . Q^T:
+// lane = position, 64 columns of f16 pairs per half of the 256 dims. Softmax group g
+// converts raw box `rbox + g` (dims 128 g .. 128 g + 127); thread = its TMEM lane = row of
+// the box. Each row is read as eight 16-byte pieces (128-byte swizzle: piece j of row r sits
+// at 16 (j ^ (r mod 8)), so the eight rows of a quarter warp hit distinct banks).
+__device__ void convert_k_tmem(TcSmem& S, uint32_t rbox, uint32_t tmem, uint32_t buf, int group,
+                               int row, uint32_t lane_addr, int lane, volatile int* abort) {
+  const uint32_t b = rbox + group, rslot = b % kRawSlots;
+  mbar_wait(&S.raw_full[rslot], (b / kRawSlots) & 1, abort);
+  const uint8_t* raw = raw_box(S, rslot) + row * 128;
+  const uint32_t dst = tmem + lane_addr + kTmemK + 128 * buf + 64 * group;
+  const int sw = row & 7;
+  uint4 v[8];  // all loads first: each tensor-memory store is a compiler barrier
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int pc = st + 256 * i;  // one 16-byte piece: 16 dims of one position
-      const int r = pc >> 2, jj = pc & 3, j = 4 * cc + jj, sw = r & 7;
-      const uint4 v = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
-      uint4 o0, o1;
-      e4m3x16_to_f16x16(v, o0, o1);
-      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj) ^ sw) << 4)) = o0;
-      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj + 1) ^ sw) << 4)) = o1;
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.kv_full[fslot]);
+  for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(raw + ((j ^ sw) << 4));
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint4 o0, o1;
+    e4m3x16_to_f16x16(v[j], o0, o1);
+    tmem_st_32x32b_x8(dst + 8 * j, o0, o1);
   }
+  tmem_wait_st();
+  tc_fence_before();
   __syncwarp();
-  if (lane == 0) mbar_arrive(&S.raw_empty[rslot]);
+  if (lane == 0) {
+    mbar_arrive_cnt(&S.raw_empty[rslot], 2);  // four warps per box, eight arrivals expected
+    mbar_arrive(&S.k_full[buf]);
+  }
+}
+
+// V(t) of an FP8 cache: raw boxes `rbox` and `rbox + 1` (e4m3, [128 positions x 128 dims]
+// each, 128-byte swizzle) -> MMA ring chunks `chunk` .. `chunk + 3` (f16, [128 positions x
+// 64 dims] each, same swizzle). The whole tile is one step -- both boxes and all four ring
+// slots are waited for up front, every thread issues its eight 16-byte loads before
+// converting, and one proxy fence covers all four chunks -- because each wait and fence
+// costs about as much as the conversion itself.
+__device__ void convert_v_tile(TcSmem& S, uint32_t rbox, uint32_t chunk, int st, int lane,
+                               volatile int* abort) {
+  constexpr uint32_t kSlots = Cfg<true>::kSlots;
+  uint32_t rslot[2], fslot[4];
+#pragma unroll
+  for (int bx = 0; bx < 2; ++bx) {
+    rslot[bx] = (rbox + bx) % kRawSlots;
+    mbar_wait(&S.raw_full[rslot[bx]], ((rbox + bx) / kRawSlots) & 1, abort);
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint32_t ch = chunk + c, use = ch / kSlots;
+    fslot[c] = ch % kSlots;
+    if (use > 0) mbar_wait(&S.kv_empty[fslot[c]], (use - 1) & 1, abort);
+  }
+  // piece i of this thread: 16 dims (jj) of one position (r) of one 64-dim chunk
+  uint4 v[2][2][2];
+#pragma unroll
+  for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int pc = st + 256 * i, r = pc >> 2, j = 4 * cc + (pc & 3);
+        v[bx][cc][i] =
+            *reinterpret_cast<const uint4*>(raw_box(S, rslot[bx]) + r * 128 + ((j ^ (r & 7)) << 4));
+      }
+#pragma unroll
+  for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      uint8_t* dst = ring_chunk<true>(S, fslot[2 * bx + cc]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int pc = st + 256 * i, r = pc >> 2, jj = pc & 3, sw = r & 7;
+        uint4 o0, o1;
+        e4m3x16_to_f16x16(v[bx][cc][i], o0, o1);
+        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj) ^ sw) << 4)) = o0;
+        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj + 1) ^ sw) << 4)) = o1;
+      }
+    }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) mbar_arrive(&S.kv_full[fslot[c]]);
+    mbar_arrive(&S.raw_empty[rslot[0]]);
+    mbar_arrive(&S.raw_empty[rslot[1]]);
+  }
 }
 
 // Q of the current item (bf16, loaded by TMA) -> f16 in place, scaled by 2^-e where e >= 0
@@ -508,21 +593,27 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     const int n = num_tiles(it);
     float lsum_w = 0.f;  // this warp's running row sum of head h0 + lane
     float s_mul = s_mul0;
-    auto convert_tile = [&]() {  // one K or V tile: two raw boxes -> four ring chunks
-      convert_box(S, rbox, fchunk, st, lane, abort);
-      convert_box(S, rbox + 1, fchunk + 2, st, lane, abort);
+    // FP8: a V tile is two raw boxes -> four ring chunks; a K tile is two raw boxes ->
+    // tensor memory buffer (tile mod 2). Tensor memory buffer j was last read by S(tile - 2),
+    // whose completion this warp has already waited for.
+    auto convert_v = [&]() {
+      convert_v_tile(S, rbox, fchunk, st, lane, abort);
       rbox += 2;
       fchunk += 4;
     };
+    auto convert_k = [&](uint32_t tile) {
+      convert_k_tmem(S, rbox, tmem, tile & 1, group, row, lane_addr, lane, abort);
+      rbox += 2;
+    };
     if constexpr (kFp8) {
       s_mul = s_mul0 * ldexpf(1.f, convert_q(S, item, st, swarp, lane, abort));
-      convert_tile();  // K(0)
+      convert_k(gt);  // K(0)
     }
 
     for (int t = 0; t < n; ++t) {
       if constexpr (kFp8) {
-        if (t + 1 < n) convert_tile();  // K(t + 1), consumed by S(t + 1)
-        convert_tile();                 // V(t), consumed by PV(t)
+        if (t + 1 < n) convert_k(gt + t + 1);  // consumed by S(t + 1)
+        convert_v();                           // V(t), consumed by PV(t)
       }
       const uint32_t tile = gt + t, j = tile & 1, k = tile >> 1;
       int y, a0, e0;
@@ -691,6 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&S.q_empty[i], 1);
     }
     mbar_init(&S.q_ready, kSoftmaxWarps);
+    for (int i = 0; i < 2; ++i) mbar_init(&S.k_full[i], kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_free[i], kSoftmaxWarps);
@@ -703,7 +795,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_alloc(&S.tmem_base, Cfg<kFp8>::kTmemCols);
     tmem_relinquish();
   }
   pdl_launch_dependents();  // the combine kernel may start launching; it waits for us
@@ -716,9 +808,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = S.tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) run_producer<kFp8>(S, &q_map, a, g);
+    run_producer<kFp8>(S, &q_map, a, g, lane == 0);
   } else if (warp == 1) {
-    if (lane == 0) run_mma<kFp8>(S, a, g, tmem);
+    run_mma<kFp8>(S, a, g, tmem, lane == 0);
   } else {
     run_softmax<kFp8>(S, a, g, tmem);
   }
@@ -729,7 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0 && S.abort_flag) atomicOr(a.err, kErrTimeout);
   if (warp == 1) {
     __syncwarp();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, Cfg<kFp8>::kTmemCols);
   }
 }
 

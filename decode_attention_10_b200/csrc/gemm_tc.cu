@@ -6,13 +6,17 @@
 // token rows against large weight matrices. Each weight byte is used by every row, so the
 // weights are what streams from HBM. They are put on the M side of the MMA ("swap AB"):
 //     out^T[n, b] = sum_k W[k, n] * X[b, k]
-//   A = W^T tile [128 output features x 64 k] -- read straight from the row-major [in, out]
-//       weight by TMA as two [64 features x 64 k] boxes (MN-major, 128-byte swizzle);
-//   B = X tile   [N rows x 64 k] (K-major, 128-byte swizzle), N = batch rounded up to 16;
+//   A = W^T tile [128 output features x 128 k] -- read straight from the row-major [in, out]
+//       weight by TMA as two [64 features x 128 k] boxes (MN-major, 128-byte swizzle);
+//   B = X tile   [N rows x 128 k] as two [N x 64 k] boxes (K-major, 128-byte swizzle), N =
+//       batch rounded up to 16;
 //   D = TMEM accumulator [128 lanes x N columns] fp32.
 // One CTA computes one 128-feature tile over a range of k (split-K for the 7168-long
 // reduction of the x-projection), with warp 0 issuing TMA into a multi-stage ring, one
 // thread of warp 1 issuing the MMAs, and warps 2..5 draining the accumulator.
+// A stage holds 128 k (32 KB of weights, 8 MMAs): each stage costs the MMA thread a barrier
+// wait and a commit of several hundred cycles, and at 64 k per stage that overhead, not
+// DRAM, set the weight stream's pace.
 #include <cuda_bf16.h>
 
 #include "mfa_internal.cuh"
@@ -24,8 +28,8 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 192;
-constexpr int kBK = 64;                 // k per stage (one 128-byte swizzle row of X)
-constexpr int kATileBytes = 128 * kBK * 2;  // 16 KB: [64 k rows x 128 B] x 2 boxes
+constexpr int kBK = 128;                // k per stage (two 128-byte swizzle rows of X)
+constexpr int kATileBytes = 128 * kBK * 2;  // 32 KB: [128 k rows x 128 B] x 2 boxes
 constexpr int kABoxBytes = kATileBytes / 2;
 constexpr int kMaxStages = 12;
 constexpr int kSmemBudget = 220 * 1024;
@@ -51,7 +55,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int stages = p.stages;
-  const int b_bytes = p.n_box * 128;
+  const int b_box = p.n_box * 128;  // one [N x 64 k] box of X
+  const int b_bytes = 2 * b_box;
   uint8_t* a_ring = base;                                  // stages x 16 KB
   uint8_t* b_ring = base + (size_t)stages * kATileBytes;   // stages x n_box * 128 B
   GemmCtl& C = *reinterpret_cast<GemmCtl*>(b_ring + (size_t)stages * b_bytes);
@@ -124,7 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else if (*abort) {
           break;
         }
-        tma_load_2d(b_ring + (size_t)s * b_bytes, &xmap, (kb0 + i) * kBK, b0, &C.full[s]);
+        uint8_t* bs = b_ring + (size_t)s * b_bytes;
+        tma_load_2d(bs, &xmap, (kb0 + i) * kBK, b0, &C.full[s]);
+        tma_load_2d(bs + b_box, &xmap, (kb0 + i) * kBK + 64, b0, &C.full[s]);
         issued = i + 1;
       }
       if (*abort) {
@@ -154,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(a + 2048 * kk, kABoxBytes, 1024);  // MN-major W^T
-          const uint64_t bd = sdesc_sw128(b + 32 * kk, 16, 1024);            // K-major X
+          const uint64_t bd = sdesc_sw128(b + (kk >> 2) * b_box + 32 * (kk & 3), 16, 1024);
           umma_f16_ss(tmem, ad, bd, idesc, (i | kk) != 0);
         }
         umma_commit(&C.empty[s]);
@@ -211,7 +218,7 @@ int wgemm_n_box(int batch) {
 cudaError_t launch_wgemm(const CUtensorMap* w, const CUtensorMap& xmap, WGemmArgs p,
                          int m_tiles, int splits, cudaStream_t s) {
   p.n_box = wgemm_n_box(p.batch);
-  const int stage_bytes = kATileBytes + p.n_box * 128;
+  const int stage_bytes = kATileBytes + 2 * p.n_box * 128;
   int stages = kSmemBudget / stage_bytes;
   if (stages > kMaxStages) stages = kMaxStages;
   if (stages > p.kblocks_per_cta) stages = p.kblocks_per_cta;

@@ -122,15 +122,16 @@ struct WGemmArgs {
   int tile_begin;       // first 128-feature tile (of the concatenated outputs)
   int three_weights;    // 1: tiles [0, w0_tiles) read w[0], then w1_tiles of w[1], then w[2]
   int w0_tiles, w1_tiles;
-  int kblocks_per_cta;  // 64-wide k blocks per CTA
+  int kblocks_per_cta;  // 128-wide k blocks per CTA
   float* out_f32;       // fp32 split partials [grid.y][batch][out_ld], or null
   uint16_t* out_bf16;   // bf16 [batch][out_ld] (when out_f32 is null)
   int out_ld;
   uint32_t* err;
   int n_box, stages, tmem_cols;  // filled in by launch_wgemm
 };
-// w: 3 tensor maps over row-major [K, N_out] bf16 weights, boxes [64 x 64]; xmap over X
-// [batch, K] bf16, boxes [64 x wgemm_n_box(batch)]; all with 128-byte swizzle.
+// w: 3 tensor maps over row-major [K, N_out] bf16 weights, boxes [128 k x 64 features];
+// xmap over X [batch, K] bf16, boxes [wgemm_n_box(batch) x 64 k]; all with 128-byte swizzle.
+// kblocks_per_cta counts blocks of 128 k.
 cudaError_t launch_wgemm(const CUtensorMap* w, const CUtensorMap& xmap, WGemmArgs p,
                          int m_tiles, int splits, cudaStream_t s);
 int wgemm_n_box(int batch);

@@ -48,8 +48,10 @@ __device__ __forceinline__ float block_sum_1024(float v, float* red) {
 // at once.
 __global__ void __launch_bounds__(kFinishThreads) xproj_finish_kernel(FinishArgs a) {
   __shared__ float red[32];
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // The next kernel (q_up) may launch now: it starts streaming its weights on the SMs the
+  // x-projection leaves, and it waits for this grid to complete before it reads c_hat.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x, tid = threadIdx.x;
   const float* part = a.part + (size_t)b * kXProjCols;
   const size_t split_stride = (size_t)a.batch * kXProjCols;
