@@ -42,6 +42,7 @@ _SIGNATURES = {
                                         ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
     "mfa_query_proj_noalloc": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_float, _P,
                                               ctypes.c_int32, _P]),
+    "mfa_wait_selftest": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_uint32, _P]),
 }
 NOALLOC_MAX_BATCH = 32
 
@@ -235,6 +236,13 @@ def query_proj_noalloc(x, w_qdown, gamma, w_qup, eps: float = 1e-6, q_out=None, 
                                       float(eps), _ptr(q_out), bsz, _stream(stream)),
            "mfa_query_proj_noalloc")
     return q_out
+
+
+def wait_selftest(ws: Workspace, limit_us: int = 1000, stream=None) -> None:
+    """mfa_wait_selftest: enqueue a kernel whose bounded wait on a barrier that nothing
+    completes gives up after limit_us; get_error(ws) then reports MFA_ERR_TIMEOUT."""
+    _check(load().mfa_wait_selftest(ws.ptr, ws.nbytes, int(limit_us), _stream(stream)),
+           "mfa_wait_selftest")
 
 
 class DecodeStep:

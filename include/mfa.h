@@ -205,6 +205,24 @@ MFA_API mfa_status mfa_query_proj_noalloc(const void* x, const void* w_qdown, co
                                           const void* w_qup, float eps, void* q_out,
                                           int32_t batch, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Diagnostics
+ * ------------------------------------------------------------------------------------- */
+
+/* Check of the failure detection the compute calls rely on (the Step-3 pages have no
+ * counterpart: it tests the library, not the method). Every wait inside the library's
+ * kernels is bounded: when one expires, the kernel stops, drains what it started and sets
+ * MFA_ERR_TIMEOUT in the workspace. This call enqueues one small kernel that makes exactly
+ * such a wait on a barrier nothing ever completes, with a limit of `limit_us` microseconds
+ * (1 .. 1,000,000) instead of the compute calls' 2 s.
+ *   ws: a workspace (mfa_workspace_bytes(b) for any b, initialized); only its error word is
+ *   touched. After the stream reaches the kernel's end, mfa_get_error(ws) returns
+ *   MFA_ERR_TIMEOUT, and the device and `ws` remain usable by every other call.
+ *   Returns MFA_ERR_INVALID_ARG for a null or misaligned ws, ws_bytes < 256 or a limit out
+ *   of range (nothing enqueued), MFA_ERR_CUDA if the launch fails. */
+MFA_API mfa_status mfa_wait_selftest(void* ws, size_t ws_bytes, uint32_t limit_us,
+                                     void* stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -209,6 +209,34 @@ def test_device_errors_zero_fill_and_report():
     assert np.array_equal(after[1], before[1])
 
 
+def test_bounded_wait_expires_reports_timeout_and_context_survives():
+    """Failure detection without a fault: a kernel waits, through the library's bounded
+    mbarrier wait, on a barrier that nothing completes. The wait must give up after its
+    limit, the call must report MFA_ERR_TIMEOUT, and the same context and workspace must
+    still compute correct attention afterwards."""
+    import time
+    from decode_attention_10_b200 import mfa
+    ws = mfa.Workspace(4)
+    assert mfa.get_error(ws) == 0
+    t0 = time.perf_counter()
+    mfa.wait_selftest(ws, limit_us=2000)
+    assert mfa.get_error(ws) == 7  # MFA_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0  # ended by its own bound, far below any watchdog
+    assert mfa.get_error(ws) == 0  # cleared
+    with pytest.raises(mfa.MfaError):
+        mfa.wait_selftest(ws, limit_us=0)  # out of range: rejected on the host
+    # the context is intact: a normal attention call on the same workspace is exact
+    inp = W.generate([1, 130, 300, 40], W.KV_BF16, seed=31, contiguous=False)
+    cache = mfa.KVCache([t.cuda() for t in inp.k_cache], [t.cuda() for t in inp.v_cache])
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(4, 64, 256, generator=g).to(torch.bfloat16)
+    out = mfa.decode_attn(q.cuda(), cache, inp.seq_lens.cuda(), ws=ws)
+    assert mfa.get_error(ws) == 0
+    ref = omfa.decode_attn(bf16_np(q), [codes_np(t) for t in inp.k_cache],
+                           [codes_np(t) for t in inp.v_cache], inp.seq_lens.tolist())
+    assert_close(bf16_np(out), ref, what="attention after an expired wait")
+
+
 @pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
 def test_kv_append_bit_exact(kv_dtype):
     """One-hot W makes k and v exact copies of chosen elements of x; with values on the
