@@ -610,10 +610,13 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       convert_k(gt);  // K(0)
     }
 
+    // FP8 order within a tile: K(t + 1), then the softmax of t, then V(t). The V ring frees
+    // only when PV(t - 1) completes, so converting V(t) last lets the softmax math of t run
+    // while PV(t - 1) executes; after PV(t - 1) only the P store and V(t)'s conversion stand
+    // before PV(t) can issue.
     for (int t = 0; t < n; ++t) {
       if constexpr (kFp8) {
         if (t + 1 < n) convert_k(gt + t + 1);  // consumed by S(t + 1)
-        convert_v();                           // V(t), consumed by PV(t)
       }
       const uint32_t tile = gt + t, j = tile & 1, k = tile >> 1;
       int y, a0, e0;
@@ -710,6 +713,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.p_full);
+      if constexpr (kFp8) convert_v();  // V(t), consumed by PV(t)
     }
     gt += n;
 
