@@ -161,9 +161,8 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, i
 namespace {
 
 // The attention of one call: the tensor-core kernel, then the merge of split sequences.
-// Unless the plan was launched earlier (aa.plan_early), it is launched here first.
+// Unless the plan was launched earlier (aa.plan_early), the attention CTAs build it on chip.
 mfa_status run_attention(const AttnArgs& aa, cudaStream_t s) {
-  if (!aa.plan_early && launch_attention_plan(aa, s) != cudaSuccess) return MFA_ERR_CUDA;
   CUtensorMap q_map;
   if (!encode_2d(&q_map, aa.q, (uint64_t)aa.batch * kHeads, kHeadDim, 2, 64, 64))
     return MFA_ERR_CUDA;

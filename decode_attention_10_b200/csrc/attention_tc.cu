@@ -763,6 +763,17 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
   });
 }
 
+// Per sequence: its first partial slot and the number of CTAs it is split over (0 for a
+// rejected sequence), for the combine kernel.
+__device__ void write_seq_info(const PlanSmem& P, int2* seq_info, int batch) {
+  const int NT = P.tile_start[batch], G = P.grid;
+  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
+    const int ns = te > ts ? plan_cta_of(te - 1, G, NT) - plan_cta_of(ts, G, NT) + 1 : 0;
+    seq_info[b] = make_int2(P.slot_base[b], ns);
+  }
+}
+
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap q_map, AttnArgs a) {
@@ -803,9 +814,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   pdl_launch_dependents();  // the combine kernel may start launching; it waits for us
-  // the split plan, computed once per call by attention_plan_kernel
-  if (!a.plan_early) pdl_wait();
-  plan_load(S.plan, a.plan, a.batch);
+  if (a.plan_early) {
+    // the split plan, computed at the start of the layer step by attention_plan_kernel
+    plan_load(S.plan, a.plan, a.batch);
+  } else {
+    // a standalone call: every CTA builds the (small) plan on chip once seq_lens are final;
+    // CTA 0 reports rejected lengths and writes the combine's per-sequence split info
+    pdl_wait();
+    plan_build(S.plan, a.seq_lens, a.kv, a.batch, a.grid, a.err, g == 0);
+    if (g == 0) write_seq_info(S.plan, a.seq_info, a.batch);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -839,12 +857,7 @@ __global__ void __launch_bounds__(256) attention_plan_kernel(AttnArgs a) {
   pdl_launch_dependents();
   plan_build(P, a.seq_lens, a.kv, a.batch, a.grid, a.err, true);
   plan_store(P, a.plan, a.batch);
-  const int NT = P.tile_start[a.batch], G = P.grid;
-  for (int b = threadIdx.x; b < a.batch; b += blockDim.x) {
-    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
-    const int ns = te > ts ? plan_cta_of(te - 1, G, NT) - plan_cta_of(ts, G, NT) + 1 : 0;
-    a.seq_info[b] = make_int2(P.slot_base[b], ns);
-  }
+  write_seq_info(P, a.seq_info, a.batch);
 }
 
 // ---------------------------------------------------------------------------------------
