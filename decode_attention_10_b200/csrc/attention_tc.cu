@@ -370,20 +370,20 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
           if (leader) umma_commit(&S.s_full[j]);
         }
       } else {
-        // K(tile): four ring chunks of 64 dims
+        // K(tile): four ring chunks of 64 dims, each used as soon as TMA has landed it
         for (int c = 0; c < 4; ++c) {
           const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
           mbar_wait(&S.kv_full[slot], use & 1, abort);
           tc_fence_after();
-          if (!*abort) {
+          if (!*abort && leader) {
             const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, slot));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
               const uint64_t bd = sdesc_sw128(q_base + c * kQChunkBytes + 32 * kk, 16, 1024);
-              if (leader) umma_f16_ss(d, ad, bd, C::kIdescS, (c | kk) != 0);
+              umma_f16_ss(d, ad, bd, C::kIdescS, (c | kk) != 0);
             }
-            if (leader) umma_commit(&S.kv_empty[slot]);
+            umma_commit(&S.kv_empty[slot]);
           }
           ++chunk;
         }
@@ -396,27 +396,57 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       if (first && item > 0) mbar_wait(&S.o_free, (item - 1) & 1, abort);
       tc_fence_after();
       const uint32_t p_base = smem_u32(S.p);
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t c0 = chunk + 2 * h;
-        const uint32_t s0 = c0 % kSlots, s1 = (c0 + 1) % kSlots;
-        mbar_wait(&S.kv_full[s0], (c0 / kSlots) & 1, abort);
-        mbar_wait(&S.kv_full[s1], ((c0 + 1) / kSlots) & 1, abort);
-        tc_fence_after();
-        if (!*abort) {
-          const uint32_t d = tmem + kTmemO + 64 * h;
-          const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, s0));
+      if constexpr (!kFp8) {
+        // bf16: each half of V^T (two chunks) is used as soon as TMA has landed it
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t c0 = chunk + 2 * h;
+          const uint32_t s0 = c0 % kSlots, s1 = (c0 + 1) % kSlots;
+          mbar_wait(&S.kv_full[s0], (c0 / kSlots) & 1, abort);
+          mbar_wait(&S.kv_full[s1], ((c0 + 1) / kSlots) & 1, abort);
+          tc_fence_after();
+          if (!*abort && leader) {
+            const uint32_t d = tmem + kTmemO + 64 * h;
+            const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, s0));
 #pragma unroll
-          for (int kt = 0; kt < kTile / 16; ++kt) {
-            const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
-            const uint64_t bd = sdesc_sw128(p_base + 2048 * kt, kPBytes, 1024);
-            if (leader) umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+            for (int kt = 0; kt < kTile / 16; ++kt) {
+              const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
+              const uint64_t bd = sdesc_sw128(p_base + 2048 * kt, kPBytes, 1024);
+              umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+            }
+            umma_commit(&S.kv_empty[s0]);
+            umma_commit(&S.kv_empty[s1]);
           }
-          if (leader) umma_commit(&S.kv_empty[s0]);
-          if (leader) umma_commit(&S.kv_empty[s1]);
         }
+        chunk += 4;
+        if (!*abort && leader) umma_commit(&S.p_free);
+      } else {
+        // FP8: V(t) is converted in one step, so all four chunks are waited for first and the
+        // 16 MMAs issue back to back (a wait or commit between MMAs stalls the issue stream)
+        uint32_t slot[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          slot[c] = (chunk + c) % kSlots;
+          mbar_wait(&S.kv_full[slot[c]], ((chunk + c) / kSlots) & 1, abort);
+        }
+        tc_fence_after();
+        if (!*abort && leader) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t d = tmem + kTmemO + 64 * h;
+            const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, slot[2 * h]));
+#pragma unroll
+            for (int kt = 0; kt < kTile / 16; ++kt) {
+              const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
+              const uint64_t bd = sdesc_sw128(p_base + 2048 * kt, kPBytes, 1024);
+              umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 4; ++c) umma_commit(&S.kv_empty[slot[c]]);
+          umma_commit(&S.p_free);
+        }
+        chunk += 4;
       }
-      chunk += 4;
-      if (!*abort && leader) umma_commit(&S.p_free);
     };
 
     for (int t = 0; t < n; ++t) {
