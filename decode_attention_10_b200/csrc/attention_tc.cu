@@ -57,8 +57,11 @@ constexpr int kGroupThreads = 128;      // one softmax group = four warps = the 
 constexpr int kGroupHeads = 32;         // heads per group
 constexpr int kChunkBytes = 16384;      // [128 positions x 64 dims] 16-bit, 128-byte swizzle
 constexpr int kRingBytes = 10 * kChunkBytes;
-constexpr int kRawSlots = 6;            // FP8: raw e4m3 boxes [128 positions x 128 dims]
-constexpr int kRawBytes = 16384;
+constexpr int kRawBytes = 16384;         // FP8: a raw e4m3 box [128 positions x 128 dims]
+constexpr int kKRawSlots = 2;           // FP8: raw K boxes (one K tile)
+constexpr int kVSlots = 4;              // FP8: V slots of 32 KB (two V tiles)
+constexpr int kVSlotBytes = 2 * kChunkBytes;
+constexpr int kKRawOff = kVSlots * kVSlotBytes;
 constexpr int kMaxSlots = 10;
 constexpr int kQChunkBytes = 8192;      // [64 heads x 64 dims] 16-bit
 constexpr int kPBytes = 16384;          // P^T: [128 positions x 64 heads] 16-bit
@@ -70,22 +73,21 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // named barriers: 1 + group among one softmax group, 3 among all eight softmax warps
 constexpr uint32_t kBarAllSoftmax = 3;
 
-// Per cache type: the shared-memory operand ring (chunks of [128 positions x 64 dims],
-// 16-bit), where it sits in the ring area, the number of Q buffers, the tensor memory used,
-// and the operand type. The ring area holds, for bf16 caches, 6 ring chunks (K and V) and
-// the second Q buffer; for FP8 caches, the 6-box raw e4m3 ring and 4 ring chunks (V only:
-// converted K tiles go to tensor memory).
+// Per cache type: the ring area's use, the number of Q buffers, the tensor memory used, and
+// the operand type. bf16 caches: a 6-slot ring of 16-bit chunks ([128 positions x 64 dims],
+// K and V) and the second Q buffer. FP8 caches: 4 V slots of 32 KB (a raw V box lands in a
+// slot's upper half and is converted in place into the slot's two f16 chunks; two V tiles
+// in flight) and 2 raw K boxes (converted K tiles go to tensor memory).
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kSlots = kFp8 ? 4 : 6;  // even: a V half-tile's 2 chunks are adjacent
-  static constexpr int kRingOff = kFp8 ? kRawSlots * kRawBytes : 0;
+  static constexpr int kSlots = 6;  // bf16 ring: even, so a V half-tile's 2 chunks are adjacent
   static constexpr uint32_t kTmemCols = kFp8 ? 512 : 256;
   static constexpr int kQBufs = kFp8 ? 1 : 2;
   static constexpr bool kBf16 = !kFp8;           // operands: bf16, or f16 for FP8 caches
   static constexpr uint32_t kIdescS = idesc_f16(128, 64, kBf16, false, false);  // K x Q^T
   static constexpr uint32_t kIdescPV = idesc_f16(128, 64, kBf16, true, true);   // V^T x P^T
 };
-static_assert(Cfg<true>::kRingOff + Cfg<true>::kSlots * kChunkBytes <= kRingBytes, "ring");
+static_assert(kKRawOff + kKRawSlots * kRawBytes <= kRingBytes, "FP8 ring");
 constexpr int kQ1Off = Cfg<false>::kSlots * kChunkBytes;  // bf16: the second Q buffer
 static_assert(kQ1Off + 4 * kQChunkBytes <= kRingBytes, "second Q buffer");
 
@@ -101,8 +103,9 @@ struct __align__(1024) TcSmem {
   float qmax[kSoftmaxWarps];
   uint64_t kv_full[kMaxSlots];
   uint64_t kv_empty[kMaxSlots];
-  uint64_t raw_full[kRawSlots];
-  uint64_t raw_empty[kRawSlots];
+  uint64_t raw_full[kKRawSlots];   // FP8: raw K box landed
+  uint64_t raw_empty[kKRawSlots];  // FP8: raw K box converted
+  uint64_t vraw_full[kVSlots];     // FP8: raw V box landed in a V slot
   uint64_t q_full[2], q_empty[2], q_ready;
   uint64_t k_full[2];  // FP8: K tile converted into tensor memory buffer 0 / 1
   uint64_t s_full[2], s_free[2];
@@ -113,12 +116,17 @@ struct __align__(1024) TcSmem {
   int32_t abort_flag;
 };
 
-template <bool kFp8>
+// bf16: ring chunk `slot`
 __device__ __forceinline__ uint8_t* ring_chunk(TcSmem& S, uint32_t slot) {
-  return S.ring_area + Cfg<kFp8>::kRingOff + slot * kChunkBytes;
+  return S.ring_area + slot * kChunkBytes;
 }
-__device__ __forceinline__ uint8_t* raw_box(TcSmem& S, uint32_t slot) {
-  return S.ring_area + slot * kRawBytes;
+// FP8: V slot `slot` (its f16 chunks at +0 and +16 KB; the raw box lands at +16 KB)
+__device__ __forceinline__ uint8_t* v_slot(TcSmem& S, uint32_t slot) {
+  return S.ring_area + slot * kVSlotBytes;
+}
+// FP8: raw K box slot
+__device__ __forceinline__ uint8_t* k_raw(TcSmem& S, uint32_t slot) {
+  return S.ring_area + kKRawOff + slot * kRawBytes;
 }
 // Q buffer qb: [4 chunks of 64 heads x 64 dims]
 __device__ __forceinline__ uint8_t* q_buf(TcSmem& S, int qb) {
@@ -234,11 +242,10 @@ template <bool kFp8>
 __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs& a, int g,
                              bool leader) {
   using C = Cfg<kFp8>;
-  constexpr int kBoxes = kFp8 ? 2 : 4;      // boxes per K or V tile
-  constexpr int kBoxX = kFp8 ? 128 : 64;    // elements per box row
-  constexpr uint32_t kN = kFp8 ? kRawSlots : C::kSlots;
+  constexpr uint32_t kN = C::kSlots;
   volatile int* abort = &S.abort_flag;
-  uint32_t chunk = 0, issued = 0;
+  uint32_t chunk = 0, issued = 0;                 // bf16: ring chunks
+  uint32_t kb = 0, kb_issued = 0, vb = 0, vb_issued = 0;  // FP8: raw K and V boxes
   int item = 0, q_issued = 0;
   if (leader) prefetch_tensormap(q_map);
   // every K/V byte is read once: keep it from evicting q and the split partials from L2
@@ -254,46 +261,78 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     prefetch_tensormap(&a.kv[it.b].tmap_k);
     prefetch_tensormap(&a.kv[it.b].tmap_v);
   }
-  // Boxes of one item, in the order the MMA consumes them: K(0), then K(t+1), V(t) for each
-  // t, then V(n-1) -- 2 * n * kBoxes boxes in all.
+  // bf16: the boxes of one item in the order the MMA consumes them -- K(0), then K(t+1),
+  // V(t) for each t, then V(n-1) -- as four [128 positions x 64 dims] boxes per K or V tile,
+  // straight into the ring. FP8: per tile K(t) (two raw [128 x 128] e4m3 boxes into the K
+  // raw slots), then V(t) (two raw boxes into the upper halves of two V slots).
+  constexpr int kBoxesPerTile = kFp8 ? 4 : 8;
   auto issue_box = [&](const WorkItem& w, int j) {
-    const int n = num_tiles(w);
-    bool is_v;
-    int t, c;
-    if (j < kBoxes) {
-      is_v = false, t = 0, c = j;
-    } else {
-      const int r = j - kBoxes, tt = r / (2 * kBoxes), rr = r % (2 * kBoxes);
-      if (tt < n - 1)
-        is_v = rr >= kBoxes, t = is_v ? tt : tt + 1, c = is_v ? rr - kBoxes : rr;
-      else
-        is_v = true, t = n - 1, c = rr;
-    }
-    int y, a0, e0;
-    tile_window(w, t, y, a0, e0);
     const KvSeq* seq = a.kv + w.b;
-    const uint32_t slot = chunk % kN, use = chunk / kN;
-    uint64_t* empty = kFp8 ? &S.raw_empty[slot] : &S.kv_empty[slot];
-    uint64_t* full = kFp8 ? &S.raw_full[slot] : &S.kv_full[slot];
-    if (use > 0) mbar_wait(empty, (use - 1) & 1, abort);
-    if (!*abort) {
-      if (leader) {
-        mbar_arrive_expect_tx(full, kChunkBytes);
-        uint8_t* dst = kFp8 ? raw_box(S, slot) : ring_chunk<kFp8>(S, slot);
-        tma_load_2d_hint(dst, is_v ? &seq->tmap_v : &seq->tmap_k, kBoxX * c, y, full,
-                         evict_first);
+    int y, a0, e0;
+    if constexpr (kFp8) {
+      const int t = j >> 2, r = j & 3;
+      tile_window(w, t, y, a0, e0);
+      if (r < 2) {
+        const uint32_t slot = kb % kKRawSlots, use = kb / kKRawSlots;
+        if (use > 0) mbar_wait(&S.raw_empty[slot], (use - 1) & 1, abort);
+        if (!*abort) {
+          if (leader) {
+            mbar_arrive_expect_tx(&S.raw_full[slot], kRawBytes);
+            tma_load_2d_hint(k_raw(S, slot), &seq->tmap_k, 128 * r, y, &S.raw_full[slot],
+                             evict_first);
+          }
+          kb_issued = kb + 1;
+        }
+        ++kb;
+      } else {
+        const uint32_t slot = vb % kVSlots, use = vb / kVSlots;
+        if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);  // PV(t - 2) done
+        if (!*abort) {
+          if (leader) {
+            mbar_arrive_expect_tx(&S.vraw_full[slot], kRawBytes);
+            tma_load_2d_hint(v_slot(S, slot) + kChunkBytes, &seq->tmap_v, 128 * (r - 2), y,
+                             &S.vraw_full[slot], evict_first);
+          }
+          vb_issued = vb + 1;
+        }
+        ++vb;
       }
-      issued = chunk + 1;
+    } else {
+      const int n = num_tiles(w);
+      bool is_v;
+      int t, c;
+      if (j < 4) {
+        is_v = false, t = 0, c = j;
+      } else {
+        const int rr0 = j - 4, tt = rr0 / 8, rr = rr0 % 8;
+        if (tt < n - 1)
+          is_v = rr >= 4, t = is_v ? tt : tt + 1, c = is_v ? rr - 4 : rr;
+        else
+          is_v = true, t = n - 1, c = rr;
+      }
+      tile_window(w, t, y, a0, e0);
+      const uint32_t slot = chunk % kN, use = chunk / kN;
+      if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);
+      if (!*abort) {
+        if (leader) {
+          mbar_arrive_expect_tx(&S.kv_full[slot], kChunkBytes);
+          tma_load_2d_hint(ring_chunk(S, slot), is_v ? &seq->tmap_v : &seq->tmap_k, 64 * c, y,
+                           &S.kv_full[slot], evict_first);
+        }
+        issued = chunk + 1;
+      }
+      ++chunk;
     }
-    ++chunk;
   };
   // The K/V rows (and the split plan) were written by kernels that completed before this one
-  // launched, so the first ring-full of the first item streams in while the previous
-  // kernel (which writes q) finishes.
+  // launched, so the first boxes of the first item -- those that need no free slot: a
+  // ring-full for bf16, K(0) and V(0) for FP8 -- stream in while the previous kernel (which
+  // writes q) finishes.
   int first_done = 0;
   if (has) {
-    const int total = 2 * num_tiles(it) * kBoxes;
-    first_done = total < static_cast<int>(kN) ? total : static_cast<int>(kN);
+    const int total = kBoxesPerTile * num_tiles(it);
+    const int pre = kFp8 ? 4 : static_cast<int>(kN);
+    first_done = total < pre ? total : pre;
     for (int j = 0; j < first_done; ++j) issue_box(it, j);
   }
   pdl_wait();
@@ -313,9 +352,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
       }
       q_issued = item + 1;
     }
-    // bf16: four [128 x 64] boxes per tile straight into the MMA ring; FP8: two raw
-    // [128 x 128] e4m3 boxes per tile into the raw ring
-    const int total = 2 * num_tiles(it) * kBoxes;
+    const int total = kBoxesPerTile * num_tiles(it);
     for (int j = (item == 0 ? first_done : 0); j < total; ++j) issue_box(it, j);
     ++item;
     it = nx;
@@ -324,8 +361,15 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   }
   // Before the CTA may exit, every copy it started must have landed.
   if (*abort) {
-    for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
-      mbar_wait_drain(kFp8 ? &S.raw_full[c % kN] : &S.kv_full[c % kN], (c / kN) & 1);
+    if constexpr (kFp8) {
+      for (uint32_t c = (kb_issued > kKRawSlots ? kb_issued - kKRawSlots : 0); c < kb_issued; ++c)
+        mbar_wait_drain(&S.raw_full[c % kKRawSlots], (c / kKRawSlots) & 1);
+      for (uint32_t c = (vb_issued > kVSlots ? vb_issued - kVSlots : 0); c < vb_issued; ++c)
+        mbar_wait_drain(&S.vraw_full[c % kVSlots], (c / kVSlots) & 1);
+    } else {
+      for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
+        mbar_wait_drain(&S.kv_full[c % kN], (c / kN) & 1);
+    }
     for (int i = (q_issued > C::kQBufs ? q_issued - C::kQBufs : 0); i < q_issued; ++i)
       mbar_wait_drain(&S.q_full[i % C::kQBufs], (i / C::kQBufs) & 1);
   }
@@ -376,7 +420,7 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
           mbar_wait(&S.kv_full[slot], use & 1, abort);
           tc_fence_after();
           if (!*abort && leader) {
-            const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, slot));
+            const uint32_t a_base = smem_u32(ring_chunk(S, slot));
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
@@ -406,7 +450,7 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
           tc_fence_after();
           if (!*abort && leader) {
             const uint32_t d = tmem + kTmemO + 64 * h;
-            const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, s0));
+            const uint32_t a_base = smem_u32(ring_chunk(S, s0));
 #pragma unroll
             for (int kt = 0; kt < kTile / 16; ++kt) {
               const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
@@ -420,20 +464,21 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
         chunk += 4;
         if (!*abort && leader) umma_commit(&S.p_free);
       } else {
-        // FP8: V(t) is converted in one step, so all four chunks are waited for first and the
-        // 16 MMAs issue back to back (a wait or commit between MMAs stalls the issue stream)
-        uint32_t slot[4];
+        // FP8: V(t) sits in two V slots (one per half of the head dimension, two chunks
+        // each), converted in one step, so both are waited for first and the 16 MMAs issue
+        // back to back (a wait or commit between MMAs stalls the issue stream)
+        uint32_t slot[2];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          slot[c] = (chunk + c) % kSlots;
-          mbar_wait(&S.kv_full[slot[c]], ((chunk + c) / kSlots) & 1, abort);
+        for (int h = 0; h < 2; ++h) {
+          slot[h] = (chunk + h) % kVSlots;
+          mbar_wait(&S.kv_full[slot[h]], ((chunk + h) / kVSlots) & 1, abort);
         }
         tc_fence_after();
         if (!*abort && leader) {
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint32_t d = tmem + kTmemO + 64 * h;
-            const uint32_t a_base = smem_u32(ring_chunk<kFp8>(S, slot[2 * h]));
+            const uint32_t a_base = smem_u32(v_slot(S, slot[h]));
 #pragma unroll
             for (int kt = 0; kt < kTile / 16; ++kt) {
               const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
@@ -441,11 +486,11 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
               umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
             }
           }
-#pragma unroll
-          for (int c = 0; c < 4; ++c) umma_commit(&S.kv_empty[slot[c]]);
+          umma_commit(&S.kv_empty[slot[0]]);
+          umma_commit(&S.kv_empty[slot[1]]);
           umma_commit(&S.p_free);
         }
-        chunk += 4;
+        chunk += 2;
       }
     };
 
@@ -474,9 +519,9 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
 // at 16 (j ^ (r mod 8)), so the eight rows of a quarter warp hit distinct banks).
 __device__ void convert_k_tmem(TcSmem& S, uint32_t rbox, uint32_t tmem, uint32_t buf, int group,
                                int row, uint32_t lane_addr, int lane, volatile int* abort) {
-  const uint32_t b = rbox + group, rslot = b % kRawSlots;
-  mbar_wait(&S.raw_full[rslot], (b / kRawSlots) & 1, abort);
-  const uint8_t* raw = raw_box(S, rslot) + row * 128;
+  const uint32_t b = rbox + group, rslot = b % kKRawSlots;
+  mbar_wait(&S.raw_full[rslot], (b / kKRawSlots) & 1, abort);
+  const uint8_t* raw = k_raw(S, rslot) + row * 128;
   const uint32_t dst = tmem + lane_addr + kTmemK + 128 * buf + 64 * group;
   const int sw = row & 7;
   uint4 v[8];  // all loads first: each tensor-memory store is a compiler barrier
@@ -497,28 +542,20 @@ __device__ void convert_k_tmem(TcSmem& S, uint32_t rbox, uint32_t tmem, uint32_t
   }
 }
 
-// V(t) of an FP8 cache: raw boxes `rbox` and `rbox + 1` (e4m3, [128 positions x 128 dims]
-// each, 128-byte swizzle) -> MMA ring chunks `chunk` .. `chunk + 3` (f16, [128 positions x
-// 64 dims] each, same swizzle). The whole tile is one step -- both boxes and all four ring
-// slots are waited for up front, every thread issues its eight 16-byte loads before
-// converting, and one proxy fence covers all four chunks -- because each wait and fence
-// costs about as much as the conversion itself.
-__device__ void convert_v_tile(TcSmem& S, uint32_t rbox, uint32_t chunk, int st, int lane,
-                               volatile int* abort) {
-  constexpr uint32_t kSlots = Cfg<true>::kSlots;
-  uint32_t rslot[2], fslot[4];
+// V(t) of an FP8 cache, in place: its two raw boxes (e4m3, [128 positions x 128 dims],
+// 128-byte swizzle) sit in the upper halves of V slots vbox and vbox + 1 (mod 4); box b
+// becomes the two f16 chunks ([128 positions x 64 dims], same swizzle) of its slot. Every
+// thread first loads all eight of its 16-byte pieces (16 codes of one position each), then
+// the eight warps synchronize, and only then is any slot overwritten: a thread's output
+// covers other threads' input. One proxy fence covers the whole tile.
+__device__ void convert_v_inplace(TcSmem& S, uint32_t vbox, int st, int lane,
+                                  volatile int* abort) {
+  uint32_t slot[2];
 #pragma unroll
   for (int bx = 0; bx < 2; ++bx) {
-    rslot[bx] = (rbox + bx) % kRawSlots;
-    mbar_wait(&S.raw_full[rslot[bx]], ((rbox + bx) / kRawSlots) & 1, abort);
+    slot[bx] = (vbox + bx) % kVSlots;
+    mbar_wait(&S.vraw_full[slot[bx]], ((vbox + bx) / kVSlots) & 1, abort);
   }
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint32_t ch = chunk + c, use = ch / kSlots;
-    fslot[c] = ch % kSlots;
-    if (use > 0) mbar_wait(&S.kv_empty[fslot[c]], (use - 1) & 1, abort);
-  }
-  // piece i of this thread: 16 dims (jj) of one position (r) of one 64-dim chunk
   uint4 v[2][2][2];
 #pragma unroll
   for (int bx = 0; bx < 2; ++bx)
@@ -527,14 +564,15 @@ __device__ void convert_v_tile(TcSmem& S, uint32_t rbox, uint32_t chunk, int st,
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int pc = st + 256 * i, r = pc >> 2, j = 4 * cc + (pc & 3);
-        v[bx][cc][i] =
-            *reinterpret_cast<const uint4*>(raw_box(S, rslot[bx]) + r * 128 + ((j ^ (r & 7)) << 4));
+        v[bx][cc][i] = *reinterpret_cast<const uint4*>(v_slot(S, slot[bx]) + kChunkBytes +
+                                                       r * 128 + ((j ^ (r & 7)) << 4));
       }
+  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);
 #pragma unroll
   for (int bx = 0; bx < 2; ++bx)
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
-      uint8_t* dst = ring_chunk<true>(S, fslot[2 * bx + cc]);
+      uint8_t* dst = v_slot(S, slot[bx]) + cc * kChunkBytes;
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int pc = st + 256 * i, r = pc >> 2, jj = pc & 3, sw = r & 7;
@@ -547,10 +585,8 @@ __device__ void convert_v_tile(TcSmem& S, uint32_t rbox, uint32_t chunk, int st,
   fence_proxy_async_smem();
   __syncwarp();
   if (lane == 0) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) mbar_arrive(&S.kv_full[fslot[c]]);
-    mbar_arrive(&S.raw_empty[rslot[0]]);
-    mbar_arrive(&S.raw_empty[rslot[1]]);
+    mbar_arrive(&S.kv_full[slot[0]]);
+    mbar_arrive(&S.kv_full[slot[1]]);
   }
 }
 
@@ -615,7 +651,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
   const float s_mul0 = a.scale * kLog2e * (kFp8 ? a.k_scale : 1.f);
   const float v_mul = kFp8 ? a.v_scale : 1.f;
   uint32_t gt = 0;
-  uint32_t rbox = 0, fchunk = 0;  // FP8: raw boxes and MMA-ring chunks converted so far
+  uint32_t kbox = 0, vbox = 0;  // FP8: raw K and V boxes converted so far
   int item = 0;
   uint8_t* const p_row = S.p + row * 128;
 
@@ -623,30 +659,29 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     const int n = num_tiles(it);
     float lsum_w = 0.f;  // this warp's running row sum of head h0 + lane
     float s_mul = s_mul0;
-    // FP8: a V tile is two raw boxes -> four ring chunks; a K tile is two raw boxes ->
-    // tensor memory buffer (tile mod 2). Tensor memory buffer j was last read by S(tile - 2),
-    // whose completion this warp has already waited for.
+    // FP8: a V tile is two raw boxes -> converted in place in two V slots; a K tile is two
+    // raw boxes -> tensor memory buffer (tile mod 2). Tensor memory buffer j was last read by
+    // S(tile - 2), whose completion this warp has already waited for.
     auto convert_v = [&]() {
-      convert_v_tile(S, rbox, fchunk, st, lane, abort);
-      rbox += 2;
-      fchunk += 4;
+      convert_v_inplace(S, vbox, st, lane, abort);
+      vbox += 2;
     };
     auto convert_k = [&](uint32_t tile) {
-      convert_k_tmem(S, rbox, tmem, tile & 1, group, row, lane_addr, lane, abort);
-      rbox += 2;
+      convert_k_tmem(S, kbox, tmem, tile & 1, group, row, lane_addr, lane, abort);
+      kbox += 2;
     };
     if constexpr (kFp8) {
       s_mul = s_mul0 * ldexpf(1.f, convert_q(S, item, st, swarp, lane, abort));
       convert_k(gt);  // K(0)
     }
 
-    // FP8 order within a tile: K(t + 1), then the softmax of t, then V(t). The V ring frees
-    // only when PV(t - 1) completes, so converting V(t) last lets the softmax math of t run
-    // while PV(t - 1) executes; after PV(t - 1) only the P store and V(t)'s conversion stand
-    // before PV(t) can issue.
+    // FP8 order within a tile: K(t + 1), V(t), then the softmax of t. V(t)'s slots were last
+    // read by PV(t - 2), so neither conversion waits for the tensor core's current work, and
+    // PV(t) can issue as soon as P(t) is stored.
     for (int t = 0; t < n; ++t) {
       if constexpr (kFp8) {
         if (t + 1 < n) convert_k(gt + t + 1);  // consumed by S(t + 1)
+        convert_v();                           // V(t), consumed by PV(t)
       }
       const uint32_t tile = gt + t, j = tile & 1, k = tile >> 1;
       int y, a0, e0;
@@ -743,7 +778,6 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.p_full);
-      if constexpr (kFp8) convert_v();  // V(t), consumed by PV(t)
     }
     gt += n;
 
@@ -818,10 +852,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&S.kv_full[i], kFp8 ? kSoftmaxWarps : 1);  // FP8: the converting warps arrive
       mbar_init(&S.kv_empty[i], 1);
     }
-    for (int i = 0; i < kRawSlots; ++i) {
+    for (int i = 0; i < kKRawSlots; ++i) {
       mbar_init(&S.raw_full[i], 1);
       mbar_init(&S.raw_empty[i], kSoftmaxWarps);
     }
+    for (int i = 0; i < kVSlots; ++i) mbar_init(&S.vraw_full[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
