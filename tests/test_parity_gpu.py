@@ -95,6 +95,36 @@ def test_layer_small_ragged(kv_dtype):
     _check_layer(inp)
 
 
+def test_layer_batch_over_256_rows():
+    # the weight GEMMs take token rows in slices of 256 (a second grid slice from row 256):
+    # rows on both sides of the seam
+    g = np.random.default_rng(41)
+    lens = [int(x) for x in g.integers(1, 300, size=300)]
+    inp = W.generate(lens, W.KV_BF16, seed=41, contiguous=False)
+    _check_layer(inp, sample=[0, 1, 128, 255, 256, 257, 299], e2e=True)
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_layer_max_batch(kv_dtype):
+    # MFA_MAX_BATCH sequences through the whole step: the plan's arrays full, several work
+    # items per attention CTA, short sequences split across CTA boundaries
+    from decode_attention_10_b200 import mfa
+    g = np.random.default_rng(42)
+    lens = [int(x) for x in g.integers(1, 400, size=mfa.MAX_BATCH)]
+    inp = W.generate(lens, kv_dtype, seed=42, contiguous=False)
+    _check_layer(inp, sample=[0, 1, 147, 148, 511, 512, 1022, 1023], e2e=True)
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_attention_max_batch_every_sequence(kv_dtype):
+    # every one of MFA_MAX_BATCH outputs against the oracle (attention alone)
+    from decode_attention_10_b200 import mfa
+    g = np.random.default_rng(43)
+    lens = [int(x) for x in g.integers(1, 400, size=mfa.MAX_BATCH)]
+    out, ref, _ = _attn_case(lens, kv_dtype, seed=43)
+    assert_close(out, ref, kv_dtype, "max batch")
+
+
 def test_layer_per_sequence_buffers_with_spare_capacity():
     lens = [77, 513, 1]
     caps = [100, 600, 9]
