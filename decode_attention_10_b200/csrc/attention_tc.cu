@@ -933,6 +933,8 @@ __global__ void __launch_bounds__(256) attention_plan_kernel(AttnArgs a) {
 // sequences (no split) get a zero output here.
 // ---------------------------------------------------------------------------------------
 constexpr int kCombineHeads = 4;
+constexpr int kCombineOnePass = 8;      // up to this many splits: the one-pass merge
+constexpr int kCombineMaxSplits = 256;  // above it: the one-pass merge (never with <= 256 SMs)
 
 __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
   pdl_wait();
@@ -947,8 +949,53 @@ __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
   }
   if (ns == 1) return;
   const float v_mul = a.kv_dtype == MFA_KV_FP8_E4M3 ? a.v_scale : 1.f;
-  // one pass with a running max per head: every split's loads are independent of the
-  // arithmetic, so several splits' worth stay in flight
+  if (ns > kCombineOnePass && ns <= kCombineMaxSplits) {
+    // Many splits (long sequences): a pass with a running max would chain the splits' L2
+    // round trips. Instead: (1) every (split, head) pair's m and l in one round trip; (2)
+    // the weights v_mul 2^(m_i - M) / L per head, one warp per head; (3) the accumulators,
+    // whose loads no longer depend on any arithmetic, so many splits stay in flight.
+    __shared__ float sm[kCombineHeads][kCombineMaxSplits];
+    __shared__ float sl[kCombineHeads][kCombineMaxSplits];
+    for (int t = tid; t < kCombineHeads * ns; t += 128) {
+      const int i = t >> 2, h = t & 3;
+      sm[h][i] = __ldcg(partial_m(a.partials, base + i) + h0 + h);
+      sl[h][i] = __ldcg(partial_l(a.partials, base + i) + h0 + h);
+    }
+    __syncthreads();
+    {
+      const int h = tid >> 5, lane = tid & 31;  // warp h: head h0 + h
+      float mx = -INFINITY;
+      for (int i = lane; i < ns; i += 32) mx = fmaxf(mx, sm[h][i]);
+      mx = warp_max_f32(mx);
+      float ls = 0.f;
+      for (int i = lane; i < ns; i += 32) ls = fmaf(sl[h][i], exp2f(sm[h][i] - mx), ls);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+      __syncwarp();
+      const float sc = v_mul / ls;
+      for (int i = lane; i < ns; i += 32) sl[h][i] = sc * exp2f(sm[h][i] - mx);  // weights
+    }
+    __syncthreads();
+    float2 o[kCombineHeads];
+#pragma unroll
+    for (int h = 0; h < kCombineHeads; ++h) o[h] = make_float2(0.f, 0.f);
+#pragma unroll 8
+    for (int i = 0; i < ns; ++i) {
+      const float* acc = partial_acc(a.partials, base + i) + h0 * kHeadDim + 2 * tid;
+#pragma unroll
+      for (int h = 0; h < kCombineHeads; ++h) {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
+        const float w = sl[h][i];
+        o[h].x = fmaf(w, x.x, o[h].x);
+        o[h].y = fmaf(w, x.y, o[h].y);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kCombineHeads; ++h) out[h * kHeadDim / 2 + tid] = pack_bf16x2(o[h].x, o[h].y);
+    return;
+  }
+  // few splits: one pass with a running max per head; every split's loads are independent
+  // of the arithmetic, so all splits' worth stay in flight
   float M[kCombineHeads], L[kCombineHeads];
   float2 o[kCombineHeads];
 #pragma unroll
