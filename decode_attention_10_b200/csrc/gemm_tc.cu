@@ -13,10 +13,16 @@
 //   D = TMEM accumulator [128 lanes x N columns] fp32.
 // One CTA computes one 128-feature tile over a range of k (split-K for the 7168-long
 // reduction of the x-projection), with warp 0 issuing TMA into a multi-stage ring, one
-// thread of warp 1 issuing the MMAs, and warps 2..5 draining the accumulator.
-// A stage holds 128 k (32 KB of weights, 8 MMAs): each stage costs the MMA thread a barrier
+// thread each of warps 1 and 6 issuing the MMAs (even and odd stages, into accumulators of
+// their own), and warps 2..5 draining and adding the two accumulators.
+// A stage holds 128 k (32 KB of weights, 8 MMAs): each stage costs its MMA thread a barrier
 // wait and a commit of several hundred cycles, and at 64 k per stage that overhead, not
-// DRAM, set the weight stream's pace.
+// DRAM, set the weight stream's pace. Two issuing threads: one thread keeps about one
+// M=128 x N<=32 MMA with fresh shared-memory operands in flight every ~70 cycles, two reach
+// the shared-memory operand bandwidth (~40 cycles per MMA); more add nothing. Each ring slot
+// belongs to one MMA thread (even slots to the first, odd slots to the second), so every
+// slot's barrier phases are waited for by one thread, in order: a parity wait is only
+// unambiguous when the waiter is never two phases ahead.
 #include <cuda_bf16.h>
 
 #include "mfa_internal.cuh"
@@ -27,7 +33,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // warp 0 TMA, warps 1 and 6 MMA, warps 2..5 epilogue
 constexpr int kBK = 128;                // k per stage (two 128-byte swizzle rows of X)
 constexpr int kATileBytes = 128 * kBK * 2;  // 32 KB: [128 k rows x 128 B] x 2 boxes
 constexpr int kABoxBytes = kATileBytes / 2;
@@ -85,7 +91,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&C.full[i], 1);
       mbar_init(&C.empty[i], 1);
     }
-    mbar_init(&C.acc_full, 1);
+    mbar_init(&C.acc_full, 2);  // one commit per MMA thread
     C.abort_flag = 0;
     fence_mbar_init();
   }
@@ -146,13 +152,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       pdl_wait();
       pdl_launch_dependents();
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 6) {
     pdl_wait();
     pdl_launch_dependents();
     if (lane == 0) {
+      // issuer j takes the stages in ring slots of parity j, into accumulator columns
+      // [j N, j N + N)
+      const int j = warp == 1 ? 0 : 1;
+      const uint32_t d = tmem + j * p.n_box;
       const uint32_t idesc = idesc_f16(128, p.n_box, true, true, false);
+      bool first = true;
       for (int i = 0; i < nkb; ++i) {
         const int s = i % stages;
+        if ((s & 1) != j) continue;
         mbar_wait(&C.full[s], (i / stages) & 1, abort);
         tc_fence_after();
         if (*abort) break;
@@ -162,8 +174,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(a + 2048 * kk, kABoxBytes, 1024);  // MN-major W^T
           const uint64_t bd = sdesc_sw128(b + (kk >> 2) * b_box + 32 * (kk & 3), 16, 1024);
-          umma_f16_ss(tmem, ad, bd, idesc, (i | kk) != 0);
+          umma_f16_ss(d, ad, bd, idesc, !first || kk != 0);
         }
+        first = false;
         umma_commit(&C.empty[s]);
       }
       umma_commit(&C.acc_full);
@@ -180,16 +193,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const bool ok = !*abort;
     const int n_abs = m_abs * 128 + row;  // column in the concatenated output
+    const bool two = nkb >= 2;  // the second MMA thread's first stage is stage 1
     for (int c0 = 0; c0 < p.n_box; c0 += 16) {
-      uint32_t r[16];
+      uint32_t r[16], r1[16];
       tmem_ld_32x32b_x16(tmem + lane_addr + c0, r);
+      if (two) tmem_ld_32x32b_x16(tmem + lane_addr + p.n_box + c0, r1);
       tmem_wait_ld();
       if (!ok) continue;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const int b = b0 + c0 + i;
         if (b >= p.batch) break;
-        const float v = __uint_as_float(r[i]);
+        const float v = __uint_as_float(r[i]) + (two ? __uint_as_float(r1[i]) : 0.f);
         if (p.out_f32 != nullptr)
           p.out_f32[((size_t)blockIdx.y * p.batch + b) * p.out_ld + n_abs] = v;
         else
@@ -225,7 +240,7 @@ cudaError_t launch_wgemm(const CUtensorMap* w, const CUtensorMap& xmap, WGemmArg
   if (stages < 2) stages = 2;
   p.stages = stages;
   int cols = 32;
-  while (cols < p.n_box) cols <<= 1;
+  while (cols < 2 * p.n_box) cols <<= 1;  // two accumulators of N columns
   p.tmem_cols = cols;
   const size_t smem = 1024 + (size_t)stages * stage_bytes + sizeof(GemmCtl);
   cudaError_t e =
