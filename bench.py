@@ -368,6 +368,10 @@ def run_ours(args, wl, rank, world, local):
         e3.record(copy_s)
     torch.cuda.synchronize()
     barrier()
+    # each set computes the same inputs every step: what was read back must be its output
+    for k in range(min(copies, args.steps)):
+        if not torch.equal(out_host[k], sets[k].out.cpu()):
+            raise RuntimeError("e2e: an output read back differs from the step's result")
     t_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
     e2e_value = whole_job_throughput(world, bsz, args.steps, t_e2e)
 
