@@ -12,7 +12,8 @@
 //               buffers for bf16 caches, so the next item's Q loads while this one streams),
 //               then K and V tiles of 128 positions as 16 KB boxes of [128 positions x 64
 //               dims] into a 6-slot shared-memory ring (128-byte swizzle).
-//   warp 1      TMEM owner and MMA issuer (one thread). Per tile t:
+//   warp 1      TMEM owner and MMA issuer (one elected lane; the warp runs converged). Per
+//               tile t:
 //                 S^T(t)[128 pos x 64 heads] = K(t)[128 x 256] . Q^T        (M=128, N=64)
 //                 O^T[256 dims x 64 heads] += V(t)^T[256 x 128] . P^T(t)    (2 x M=128, N=64)
 //               S^T is double-buffered in TMEM, so S(t+1) runs while the softmax of t does.
@@ -27,15 +28,16 @@
 //   Tiles are windows of 128 positions; the last window of a work item ends at the item's
 //   end (it may start before the item or at a negative position, which TMA zero-fills), so
 //   rows past a sequence's length are never read. Positions outside the item are masked.
-// FP8 caches: TMA brings raw e4m3 boxes of [128 positions x 128 dims] into a 6-slot ring,
-// and the eight softmax warps convert them (e4m3 -> f16 is exact). A K tile goes straight
-// into tensor memory (two 128-column buffers), where the S^T product reads it as its A
-// operand; a V tile goes into the same swizzled 16 KB shared-memory chunks the bf16 path
-// uses (a 4-slot ring). Keeping K out of shared memory is what leaves room for a raw ring
-// deep enough to keep 96 KB of loads in flight. Both products run with f16 operands: Q is
-// converted to f16 in place once per item (scaled by a power of two if its magnitude could
-// overflow f16), P is written as f16. The K and V scales fold into the softmax scale and
-// the output scale.
+// FP8 caches: TMA brings raw e4m3 boxes of [128 positions x 128 dims], and the eight
+// softmax warps convert them (e4m3 -> f16 is exact). A K tile (two boxes through a 2-slot raw
+// ring) goes straight into tensor memory (two 128-column buffers), where the S^T product
+// reads it as its A operand. A V box lands in the upper half of a 32 KB V slot and is
+// converted in place into the slot's two swizzled 16 KB chunks, the layout the bf16 path
+// streams; four slots hold two V tiles, so converting V(t) never waits for PV(t - 1). Per
+// tile the softmax warps do K(t + 1), V(t), then the softmax of t. Both products run with f16
+// operands: Q is converted to f16 in place once per item (scaled by a power of two if its
+// magnitude could overflow f16), P is written as f16. The K and V scales fold into the
+// softmax scale and the output scale.
 // The split plan (which CTA streams which tiles) is computed on chip: see attn_plan.cuh.
 // A sequence covered by one CTA is finished in place; the items of a sequence split over
 // several CTAs leave (m, l, acc) partials that attention_combine_kernel merges.
@@ -376,7 +378,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
 }
 
 // ---------------------------------------------------------------------------------------
-// warp 1 (one thread): MMA issue
+// warp 1 (one elected lane issues): MMA
 // ---------------------------------------------------------------------------------------
 template <bool kFp8>
 __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool leader) {
