@@ -89,6 +89,15 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s for a kernel timed alone (burst), measured, else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
+
+
 # ---------------------------------------------------------------------------------------
 # clocks during the timed region (NVML in a thread; read-only queries)
 # ---------------------------------------------------------------------------------------
@@ -216,6 +225,7 @@ def run_ours(args, wl, rank, world, local):
     import torch
     from decode_attention_10_b200 import build, mfa
     from decode_attention_10_b200 import workloads as W
+    from decode_attention_10_b200.cost_model import layer_roofline, step_counts
 
     build.build()
     torch.cuda.set_device(local)
@@ -397,6 +407,10 @@ def run_ours(args, wl, rank, world, local):
                      "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_source": peak_kind,
                      "bytes_per_launch": a_bytes, "traffic": traffic},
+        # the whole step against its roofline: max(flops/TC, bytes/HBM) for the attention plus
+        # the same for the linear projections (the pages' cost framing), at the measured peaks
+        "layer_roofline": layer_roofline(step_counts(inp.seq_lens.tolist(), inp.kv_dtype),
+                                         ms_per_step / 1e3, peak, measured_tensor_peak()),
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT,
                 "h2d_bytes_per_step": bsz * 7168 * 2 + bsz * 4,

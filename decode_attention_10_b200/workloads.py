@@ -172,6 +172,12 @@ def ragged_lengths(batch: int, seed: int) -> list:
     return [int(n) for n in torch.randint(1, MAX_CONTEXT + 1, (batch,), generator=g)]
 
 
+def workload_lens(w: Workload, seed: Optional[int] = None) -> list:
+    """The per-sequence lengths of a named workload, without drawing its tensors."""
+    seed = 1000 + w.index if seed is None else int(seed)
+    return ragged_lengths(w.batch, seed) if w.context is None else [w.context] * w.batch
+
+
 def generate_workload(w: Workload, seed: Optional[int] = None) -> Inputs:
     """Inputs of one of the named workloads (seed defaults to 1000 + index)."""
     seed = 1000 + w.index if seed is None else int(seed)
