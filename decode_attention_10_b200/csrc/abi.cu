@@ -365,9 +365,6 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   aa.plan_early = 1;
   aa.err = at<uint32_t>(ws, L.err);
   aa.grid = L.attn_grid;
-  // the split plan needs only seq_lens and the KV table: it runs first, and the attention
-  // kernel (four launches later) reads it before waiting on its predecessor
-  if (launch_attention_plan(aa, s) != cudaSuccess) return MFA_ERR_CUDA;
   // one projection of x onto [W_qdown | W_k | W_v]
   float* part = at<float>(ws, L.xproj_part);
   st = run_xproj(x, w_qdown, w_k, w_v, batch, 0, kXProjCols / 128, part,
@@ -387,6 +384,11 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   fa.pos = seq_lens;
   fa.pos_from_len = 1;
   fa.err = at<uint32_t>(ws, L.err);
+  // plus the attention's split plan (it needs only seq_lens and the KV table), which the
+  // attention kernel two launches later reads before waiting on its predecessor
+  fa.plan = aa.plan;
+  fa.seq_info = aa.seq_info;
+  fa.attn_grid = aa.grid;
   if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
   st = run_q_up(fa.c_hat, w_qup, q_out, batch, fa.err, s);
   if (st != MFA_OK) return st;

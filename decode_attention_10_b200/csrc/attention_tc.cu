@@ -829,17 +829,6 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
   });
 }
 
-// Per sequence: its first partial slot and the number of CTAs it is split over (0 for a
-// rejected sequence), for the combine kernel.
-__device__ void write_seq_info(const PlanSmem& P, int2* seq_info, int batch) {
-  const int NT = P.tile_start[batch], G = P.grid;
-  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
-    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
-    const int ns = te > ts ? plan_cta_of(te - 1, G, NT) - plan_cta_of(ts, G, NT) + 1 : 0;
-    seq_info[b] = make_int2(P.slot_base[b], ns);
-  }
-}
-
 template <bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap q_map, AttnArgs a) {
@@ -882,7 +871,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   pdl_launch_dependents();  // the combine kernel may start launching; it waits for us
   if (a.plan_early) {
-    // the split plan, computed at the start of the layer step by attention_plan_kernel
+    // the split plan, computed during the layer step's x-projection by an extra block of
+    // the x-projection's finish kernel
     plan_load(S.plan, a.plan, a.batch);
   } else {
     // a standalone call: every CTA builds the (small) plan on chip once seq_lens are final;
@@ -912,19 +902,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tmem_dealloc(tmem, Cfg<kFp8>::kTmemCols);
   }
-}
-
-// ---------------------------------------------------------------------------------------
-// plan: one block builds the split plan from seq_lens and the KV table, stores it for the
-// attention CTAs, and writes each sequence's (first partial slot, splits) for the combine
-// ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) attention_plan_kernel(AttnArgs a) {
-  __shared__ PlanSmem P;
-  pdl_wait();
-  pdl_launch_dependents();
-  plan_build(P, a.seq_lens, a.kv, a.batch, a.grid, a.err, true);
-  plan_store(P, a.plan, a.batch);
-  write_seq_info(P, a.seq_info, a.batch);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -1030,10 +1007,6 @@ __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
 }
 
 }  // namespace
-
-cudaError_t launch_attention_plan(const AttnArgs& a, cudaStream_t s) {
-  return launch_pdl(attention_plan_kernel, dim3(1), dim3(256), 0, s, a);
-}
 
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s) {
   return launch_pdl(attention_combine_kernel, dim3(a.batch, kHeads / kCombineHeads, 1), dim3(128),

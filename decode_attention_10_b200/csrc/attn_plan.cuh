@@ -1,4 +1,7 @@
-// Length-aware split plan of the decode attention, computed on chip by every CTA.
+// Length-aware split plan of the decode attention. In a layer step one extra block of the
+// x-projection's finish kernel builds it (it needs only seq_lens and the KV table) and
+// stores it for the attention CTAs; a standalone attention call builds it on chip in every
+// attention CTA.
 //
 // The cached positions of all sequences are cut into tiles of kTile positions and laid end
 // to end (sequence 0's tiles, then sequence 1's, ...). CTA g of a persistent grid of G CTAs
@@ -7,7 +10,7 @@
 // so every CTA streams the same number of KV bytes (to within one tile) whatever the mix
 // of lengths. The part of one sequence that falls in one CTA's range is a work item. A
 // sequence covered by a single CTA is finished in place; a sequence split over n > 1 CTAs
-// gets n partial slots (m, l, acc), and the last CTA to finish one of them merges all n.
+// gets n partial slots (m, l, acc), which the combine kernel merges.
 #pragma once
 
 #include "mfa_internal.cuh"
@@ -130,6 +133,17 @@ __device__ inline void plan_load(PlanSmem& P, const int32_t* __restrict__ g, int
     P.len[i] = g[2 * kMaxBatch + 1 + i];
   }
   if (threadIdx.x == 0) P.grid = g[3 * kMaxBatch + 1];
+}
+
+// Per sequence: its first partial slot and the number of CTAs it is split over (0 for a
+// rejected sequence), for the combine kernel.
+__device__ inline void write_seq_info(const PlanSmem& P, int2* seq_info, int batch) {
+  const int NT = P.tile_start[batch], G = P.grid;
+  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
+    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
+    const int ns = te > ts ? plan_cta_of(te - 1, G, NT) - plan_cta_of(ts, G, NT) + 1 : 0;
+    seq_info[b] = make_int2(P.slot_base[b], ns);
+  }
 }
 
 struct WorkItem {

@@ -54,7 +54,7 @@ constexpr size_t kPlanBytes = sizeof(int32_t) * (3 * kMaxBatch + 2);
 struct WsLayout {
   size_t err;          // uint32 error bits
   size_t seq_info;     // int2 [kMaxBatch]: (first partial slot, splits) per sequence
-  size_t plan;         // the attention split plan (written by the plan kernel)
+  size_t plan;         // the attention split plan (written by the finish kernel's plan block)
   size_t attn_part;    // partial slots
   size_t xproj_part;   // fp32 [kXProjSplits][batch][kXProjCols]
   size_t c_hat;        // bf16 [batch][kRank]
@@ -150,6 +150,12 @@ struct FinishArgs {
   const int32_t* pos;      // device [batch]: row to write
   int pos_from_len;        // 1: row = pos[b] - 1 (pos holds seq_lens)
   uint32_t* err;
+  // the attention's split plan (layer step): one extra block builds it from pos (= seq_lens)
+  // and the KV table while the x-projection runs, and stores it with the combine's
+  // per-sequence info; null = no plan block
+  int32_t* plan;
+  int2* seq_info;
+  int attn_grid;
 };
 cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s);
 
@@ -165,15 +171,12 @@ struct AttnArgs {
   int batch;
   float* partials;          // slots
   int2* seq_info;           // [batch]: (first slot, splits), written for the combine kernel
-  int32_t* plan;            // the split plan, written by launch_attention_plan
+  int32_t* plan;            // the split plan, written by the finish kernel's plan block
   int plan_early;           // 1: the plan was written two or more kernels earlier on the
                             // stream, so it may be read before griddepcontrol.wait
   uint32_t* err;
   int grid;
 };
-// One block: the split plan of the attention (and the combine's per-sequence info) from
-// seq_lens and the KV table, written to a.plan / a.seq_info; reports rejected lengths.
-cudaError_t launch_attention_plan(const AttnArgs& a, cudaStream_t s);
 // Tensor-core attention (bf16 or FP8 KV); q_map covers q as [batch * 64 rows, 256] bf16,
 // boxes of [64 x 64] with 128-byte swizzle.
 cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s);

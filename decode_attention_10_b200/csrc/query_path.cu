@@ -7,9 +7,11 @@
 //   c = sum_s partial[s][b][0:2048];  c_hat = bf16(c * rsqrt(mean(c^2) + eps) * gamma)
 //   k, v = sum_s partial[s][b][2048:2560] -> bf16, or e4m3(k / k_scale), e4m3(v / v_scale),
 //   written at cache row pos[b] (or seq_lens[b] - 1) of sequence b.
+// In a layer step one more block builds the attention's split plan (attn_plan.cuh).
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include "attn_plan.cuh"
 #include "mfa_internal.cuh"
 
 namespace mfa {
@@ -48,9 +50,19 @@ __device__ __forceinline__ float block_sum_1024(float v, float* red) {
 // at once.
 __global__ void __launch_bounds__(kFinishThreads) xproj_finish_kernel(FinishArgs a) {
   __shared__ float red[32];
+  __shared__ PlanSmem plan;
   // The next kernel (q_up) may launch now: it starts streaming its weights on the SMs the
   // x-projection leaves, and it waits for this grid to complete before it reads c_hat.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (blockIdx.x == a.batch) {
+    // The plan block. seq_lens and the KV table were final before the step began, so it
+    // does not wait for the x-projection; the attention reads the plan after this grid
+    // (and q_up after it) completed.
+    plan_build(plan, a.pos, a.kv, a.batch, a.attn_grid, a.err, true);
+    plan_store(plan, a.plan, a.batch);
+    write_seq_info(plan, a.seq_info, a.batch);
+    return;
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int b = blockIdx.x, tid = threadIdx.x;
   const float* part = a.part + (size_t)b * kXProjCols;
@@ -97,7 +109,8 @@ __global__ void __launch_bounds__(kFinishThreads) xproj_finish_kernel(FinishArgs
 }  // namespace
 
 cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s) {
-  return launch_pdl(xproj_finish_kernel, dim3(a.batch), dim3(kFinishThreads), 0, s, a);
+  const int blocks = a.batch + (a.plan != nullptr ? 1 : 0);
+  return launch_pdl(xproj_finish_kernel, dim3(blocks), dim3(kFinishThreads), 0, s, a);
 }
 
 }  // namespace mfa
