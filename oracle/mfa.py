@@ -221,3 +221,53 @@ def decode_layer(x, w_qdown, gamma, w_qup, w_k, w_v, k_cache, v_cache, seq_lens,
                       seqs)
     return dict(c_hat=c_hat, q=q, k_codes=k_codes, v_codes=v_codes, k_cache=k_cache2,
                 v_cache=v_cache2, out=out)
+
+
+# ----------------------------------------------------------------------------------------
+# the attention side of a decode step: output projection and a stack of layers
+# ----------------------------------------------------------------------------------------
+
+O_WIDTH = N_HEADS * HEAD_DIM  # 16384: the 64 heads' outputs of one token, concatenated
+
+
+def o_proj(out, w_o):
+    """y = out W_o: the attention output of all heads, [B, H, d] or [B, H * d], projected
+    back to the hidden width (bud-325 "Method": the per-token cost counts the linear
+    projections around attention, and the layer hands a hidden-width vector on to the FFN;
+    the [16384, 7168] shape of W_o is the reading that the 64 x 256 head outputs return to
+    hidden size 7168). Float64.
+
+    Pinned by: small-integer inputs against a brute-force triple loop, and a one-hot W_o
+    that copies chosen columns of out."""
+    o = np.asarray(out, np.float64)
+    o = o.reshape(o.shape[0], -1)
+    return o @ np.asarray(w_o, np.float64)
+
+
+def attention_side_step(x, layers, seq_lens, kv_dtype=KV_BF16, eps=RMS_EPS,
+                        scale=SOFTMAX_SCALE, n_heads=N_HEADS, emulate=True):
+    """The attention side of one decode step through a stack of layers. Each entry of
+    ``layers`` is a dict with w_qdown, gamma, w_qup, w_k, w_v, w_o, k_cache, v_cache,
+    k_scale, v_scale. Layer l runs decode_layer on its hidden input, projects the attention
+    output with its W_o, and the result is layer l + 1's hidden input: under Attention-FFN
+    Disaggregation (bud-325 "Key claims") the FFN runs on other GPUs and its result comes
+    back as the next layer's input, so with the FFN out of scope the projection is handed
+    on directly. With ``emulate`` the bf16 tensors the GPU path stores between calls (the
+    attention output and y) are rounded to bf16 as it does.
+
+    Returns (per-layer list of decode_layer results, each with y added; the last y)."""
+    results = []
+    h = np.asarray(x, np.float64)
+    for lay in layers:
+        r = decode_layer(h, lay["w_qdown"], lay["gamma"], lay["w_qup"], lay["w_k"],
+                         lay["w_v"], lay["k_cache"], lay["v_cache"], seq_lens, kv_dtype,
+                         lay.get("k_scale", 1.0), lay.get("v_scale", 1.0), eps, scale,
+                         n_heads, emulate=emulate)
+        out = codecs.bf16_round(r["out"]) if emulate else r["out"]
+        y = o_proj(out, lay["w_o"])
+        if emulate:
+            y = codecs.bf16_round(y)
+        r["y"] = y
+        results.append(r)
+        h = y
+    return results, h

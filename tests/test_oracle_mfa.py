@@ -329,3 +329,94 @@ def test_planted_off_by_one_append_row_is_caught():
     assert np.array_equal(k2[0][2], new[0]) and np.array_equal(k2[0][3], kc[0][3])
     k_bad, _ = mfa.kv_append(kc, kc, [3], new, new)
     assert not np.array_equal(k_bad[0][2], new[0])
+
+
+# ----------------------------------------------------------------------------------------
+# output projection and the stack of layers (the attention side of a decode step)
+# ----------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("bsz,heads,hd,dout", [(1, 2, 3, 5), (3, 4, 4, 7)])
+def test_o_proj_exact_on_small_integers(bsz, heads, hd, dout):
+    rng = np.random.default_rng(heads * hd + dout)
+    out = rng.integers(-3, 4, (bsz, heads, hd))
+    w = rng.integers(-2, 3, (heads * hd, dout))
+    flat = out.reshape(bsz, heads * hd).tolist()
+    want = np.array(_int_matmul(flat, w.tolist()), dtype=np.float64)
+    assert np.array_equal(mfa.o_proj(out, w), want)
+    # the flat [B, H * d] form is the same call
+    assert np.array_equal(mfa.o_proj(np.array(flat), w), want)
+
+
+def test_o_proj_one_hot_copies_the_chosen_head_slot():
+    # W_o routes (head h, dim j) = input column h * d + j to output column n
+    heads, hd, dout = 4, 5, 9
+    rng = np.random.default_rng(7)
+    for _ in range(10):
+        h, j, n = rng.integers(heads), rng.integers(hd), rng.integers(dout)
+        w = np.zeros((heads * hd, dout))
+        w[h * hd + j, n] = 1.0
+        out = rng.standard_normal((3, heads, hd))
+        y = mfa.o_proj(out, w)
+        expect = np.zeros((3, dout))
+        expect[:, n] = out[:, h, j]
+        assert np.array_equal(y, expect)
+
+
+def _tiny_layer(rng, dim, rank, heads, hd, lens):
+    lay = dict(
+        w_qdown=rng.standard_normal((dim, rank)) / math.sqrt(dim),
+        gamma=rng.uniform(0.5, 1.5, rank),
+        w_qup=rng.standard_normal((rank, heads * hd)) / math.sqrt(rank),
+        w_k=rng.standard_normal((dim, hd)) / math.sqrt(dim),
+        w_v=rng.standard_normal((dim, hd)) / math.sqrt(dim),
+        w_o=rng.standard_normal((heads * hd, dim)) / math.sqrt(heads * hd))
+    ck = [codecs.bf16_round(rng.standard_normal((n, hd))) for n in lens]
+    cv = [codecs.bf16_round(rng.standard_normal((n, hd))) for n in lens]
+    lay["k_rows"], lay["v_rows"] = ck, cv
+    lay["k_cache"] = [codecs.bf16_encode(t) for t in ck]
+    lay["v_cache"] = [codecs.bf16_encode(t) for t in cv]
+    return lay
+
+
+def test_attention_side_step_matches_brute_force_chain():
+    """Two layers: layer 1's input must be layer 0's projected output, each layer's output
+    projection a plain sum, and the whole chain equal to pure-Python loops."""
+    rng = np.random.default_rng(11)
+    dim, rank, heads, hd, lens = 10, 6, 3, 4, [3, 1, 5]
+    eps, scale = 1e-6, 1.0 / math.sqrt(hd)
+    layers = [_tiny_layer(rng, dim, rank, heads, hd, lens) for _ in range(2)]
+    x = rng.standard_normal((len(lens), dim))
+    res, y_last = mfa.attention_side_step(x, layers, lens, eps=eps, scale=scale,
+                                          n_heads=heads, emulate=False)
+    h = x.tolist()
+    for lay, r in zip(layers, res):
+        # the cache rounds the appended row to bf16; give brute force the same rows
+        k_new, v_new = mfa.kv_project(np.array(h), lay["w_k"], lay["w_v"])
+        ck2 = [np.vstack([lay["k_rows"][b][:lens[b] - 1], codecs.bf16_round(k_new[b])[None]])
+               for b in range(len(lens))]
+        cv2 = [np.vstack([lay["v_rows"][b][:lens[b] - 1], codecs.bf16_round(v_new[b])[None]])
+               for b in range(len(lens))]
+        out = _brute_layer(h, lay["w_qdown"].tolist(), lay["gamma"].tolist(),
+                           lay["w_qup"].tolist(), lay["w_k"].tolist(), lay["w_v"].tolist(),
+                           [t.tolist() for t in ck2], [t.tolist() for t in cv2], lens, heads,
+                           eps, scale)
+        flat = [[v for head in seq for v in head] for seq in out]
+        wo = lay["w_o"].tolist()
+        y = [[math.fsum(f[i] * wo[i][n] for i in range(len(f))) for n in range(dim)]
+             for f in flat]
+        assert np.allclose(r["out"], out, rtol=1e-12, atol=1e-13)
+        assert np.allclose(r["y"], y, rtol=1e-12, atol=1e-13)
+        h = y
+    assert np.allclose(y_last, h, rtol=1e-12, atol=1e-13)
+
+
+def test_planted_o_proj_skipped_in_the_chain_is_caught():
+    # handing the attention output on without W_o changes the next layer's input
+    rng = np.random.default_rng(5)
+    dim, rank, heads, hd, lens = 12, 6, 3, 4, [2, 4]
+    layers = [_tiny_layer(rng, dim, rank, heads, hd, lens) for _ in range(2)]
+    x = rng.standard_normal((len(lens), dim))
+    res, _ = mfa.attention_side_step(x, layers, lens, scale=0.5, n_heads=heads, emulate=False)
+    wrong = res[0]["out"].reshape(len(lens), -1)  # heads * hd == dim: shapes would fit
+    assert not np.allclose(wrong, res[0]["y"], rtol=1e-3, atol=1e-6)
