@@ -1,7 +1,7 @@
 """Benchmark of one MFA decode step (Step-3's Multi-Matrix Factorization Attention layer).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME|INDEX]
+                    [--workload NAME|INDEX] [--layers L]
 
 A step is one whole decode step of the layer on one batch of synthetic inputs: hidden-state
 projections (query down-projection + RMSNorm + up-projection, K/V projection + cache
@@ -16,6 +16,11 @@ the timed region. Between timed steps the inputs rotate over several device copi
 combined footprint is far above the 126 MB L2, so no step reads the previous step's bytes
 from L2. Multi-GPU runs (torchrun) shard sequences over ranks (weak scaling, no data-path
 collective: the decode step of one sequence needs nothing from another).
+
+`--layers L` times the attention side of a whole decode step instead: L layers, each the
+decode step above plus the output projection 16384 -> 7168, every layer with its own weights
+and cache, the whole stack one CUDA graph; its line compares the time of 61 such layers with
+the pages' per-stage budgets of a 50 ms TPOT pipeline.
 
 `--impl reference` times the float64 CPU oracle on this host's cores on a bounded sample
 of the same workload (the baseline of this build; there is no runnable reference code).
@@ -49,6 +54,9 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--layers", type=int, default=0,
+                   help="time the attention side of a whole decode step instead: this many "
+                        "layers, each the MFA decode step plus its output projection")
     return p.parse_args()
 
 
@@ -441,6 +449,115 @@ LAUNCHES_PER_LAYER = 5  # x-projection, split-K finish (+RMSNorm, append, split 
 #                         attention, split combine
 
 
+# The pages' per-stage budgets of a 50 ms TPOT pipeline, summed over the 61 layers (bud-325
+# "Key claims": 16.6 ms per stage with 3 stages, 12.5 ms with 4).
+STAGE_BUDGET_MS = {"3-stage": 16.6, "4-stage": 12.5}
+MODEL_LAYERS = 61
+
+
+def run_stack(args, wl, rank, world, local):
+    """The attention side of one decode step: ``args.layers`` layers on one stream, each the
+    MFA decode step of the workload's batch and its output projection 16384 -> 7168, layer
+    l + 1 taking layer l's projection as its hidden input (the FFN between them runs on
+    other GPUs under Attention-FFN Disaggregation and is not part of this path). Every layer
+    has its own weights and KV cache in HBM; the whole stack is one CUDA graph."""
+    import torch
+    from decode_attention_10_b200 import build, mfa
+    from decode_attention_10_b200 import workloads as W
+    from decode_attention_10_b200.cost_model import stack_roofline, step_counts
+
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    seed = rank_seed(wl, rank)
+    lens_list = W.workload_lens(wl, seed=seed)
+    bsz = len(lens_list)
+    nl = args.layers
+    layers = [W.generate_layer_on_device(lens_list, wl.kv_dtype, seed * 1000 + l, dev,
+                                         contiguous=wl.contiguous) for l in range(nl)]
+    g = torch.Generator(device=dev).manual_seed(seed)
+    x0 = torch.randn(bsz, 7168, generator=g, device=dev).to(torch.bfloat16)
+    lens = torch.tensor(lens_list, dtype=torch.int32, device=dev)
+    ws = mfa.Workspace(bsz, dev)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    x = x0
+    for lay in layers:
+        lay["cache"] = mfa.KVCache(lay["k_cache"], lay["v_cache"], lay["k_scale"],
+                                   lay["v_scale"])
+        lay["x"] = x
+        lay["q"] = torch.empty(bsz, 64, 256, dtype=torch.bfloat16, device=dev)
+        lay["out"] = torch.empty(bsz, 64, 256, dtype=torch.bfloat16, device=dev)
+        lay["y"] = torch.empty(bsz, 7168, dtype=torch.bfloat16, device=dev)
+        lay["step"] = mfa.DecodeStep(x, lay["w_qdown"], lay["gamma"], lay["w_qup"], lay["w_k"],
+                                     lay["w_v"], lay["cache"], lens, lay["q"], lay["out"], ws,
+                                     stream=side)
+        x = lay["y"]
+
+    def stack():
+        for lay in layers:
+            lay["step"]()
+            mfa.o_proj(lay["out"], lay["w_o"], y=lay["y"], ws=ws, stream=side)
+
+    with torch.cuda.stream(side):
+        stack()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            stack()
+    torch.cuda.current_stream().wait_stream(side)
+    for _ in range(max(args.warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize()
+    if mfa.get_error(ws) != 0:
+        raise RuntimeError("device error flag set during warm-up")
+    if not torch.isfinite(layers[-1]["y"].float()).all():
+        raise RuntimeError("non-finite output")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record()
+        for _ in range(args.steps):
+            graph.replay()
+        e1.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms_per_step = t_ms / args.steps
+    peak, _ = measured_peaks()
+    counts = step_counts(lens_list, wl.kv_dtype, o_proj=True)
+    per_layer_ms = ms_per_step / nl
+    return {
+        "metric": "MFA attention-side decode tokens/s (layers x [decode step + output "
+                  "projection])",
+        "value": whole_job_throughput(world, bsz, args.steps, t_ms), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if wl.kv_dtype == "bf16" else "bf16+fp8kv", "data": "synthetic",
+        "config": {"workload": wl.name, "layers": nl, "batch_per_gpu": bsz,
+                   "global_batch": bsz * world, "context": wl.context,
+                   "kv_dtype": wl.kv_dtype, "o_proj": "16384 -> 7168",
+                   "l2": "every layer has its own weights and KV cache "
+                         f"({(counts.linear_bytes + counts.attn_bytes) / 1e6:.0f} MB per "
+                         "layer, > 126 MB L2)",
+                   "parallelism": f"dp{world} (sequences sharded, weights replicated)"},
+        "ms_per_layer": per_layer_ms,
+        "stage_ms_61_layers": per_layer_ms * MODEL_LAYERS,
+        "stage_budget_ms": STAGE_BUDGET_MS,
+        "within_budget": {k: per_layer_ms * MODEL_LAYERS <= v
+                          for k, v in STAGE_BUDGET_MS.items()},
+        "stack_roofline": stack_roofline(counts, nl, ms_per_step / 1e3, peak,
+                                         measured_tensor_peak()),
+        "clocks": clk.summary(),
+        "gpu_launches": 7 * nl * args.steps,
+        "timing": "CUDA-graph replay of the whole stack; CUDA events on the launching "
+                  "stream",
+    }
+
+
 def profiled_traffic(workload_name):
     """DRAM bytes per attention launch from the committed ncu summary, if it was taken on
     the current attention source; otherwise None."""
@@ -512,7 +629,10 @@ def main():
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        res = run_ours(args, wl, rank, world, local)
+        if args.layers > 0:
+            res = run_stack(args, wl, rank, world, local)
+        else:
+            res = run_ours(args, wl, rank, world, local)
     finally:
         if world > 1:
             import torch

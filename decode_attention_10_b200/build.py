@@ -14,7 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmfa.so")
-SOURCES = ["abi.cu", "query_path.cu", "gemm_tc.cu", "attention_tc.cu", "noalloc.cu", "selftest.cu"]
+SOURCES = ["abi.cu", "query_path.cu", "gemm_tc.cu", "attention_tc.cu", "out_proj.cu", "noalloc.cu",
+           "selftest.cu"]
 HEADERS = ["mfa_internal.cuh", "attn_plan.cuh", "sm100.cuh"]
 
 

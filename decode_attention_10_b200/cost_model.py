@@ -29,6 +29,7 @@ Q_WIDTH = HEADS * HEAD_DIM
 WEIGHT_ELEMS = HIDDEN * Q_RANK + Q_RANK * Q_WIDTH + 2 * HIDDEN * HEAD_DIM
 WEIGHT_BYTES = 2 * WEIGHT_ELEMS  # bf16
 ATTN_FLOPS_PER_POSITION = 4 * HEADS * HEAD_DIM  # 65,536
+O_PROJ_ELEMS = Q_WIDTH * HIDDEN  # the output projection W_o [16384, 7168]
 
 
 @dataclass
@@ -57,7 +58,9 @@ def kv_row_bytes(kv_dtype: str) -> int:
     return HEAD_DIM * (2 if kv_dtype == "bf16" else 1)
 
 
-def step_counts(seq_lens: Iterable[int], kv_dtype: str) -> StepCounts:
+def step_counts(seq_lens: Iterable[int], kv_dtype: str, o_proj: bool = False) -> StepCounts:
+    """Counts of one step of the layer; with ``o_proj`` the output projection (W_o, out
+    read, y written) is added to the linear part."""
     lens = [int(n) for n in seq_lens]
     batch, positions = len(lens), sum(lens)
     row = kv_row_bytes(kv_dtype)
@@ -67,6 +70,9 @@ def step_counts(seq_lens: Iterable[int], kv_dtype: str) -> StepCounts:
     linear_flops = 2.0 * batch * WEIGHT_ELEMS
     # weights once; x read (bf16); q written (bf16); the appended K and V rows written
     linear_bytes = WEIGHT_BYTES + batch * HIDDEN * 2 + batch * Q_WIDTH * 2 + batch * 2 * row
+    if o_proj:
+        linear_flops += 2.0 * batch * O_PROJ_ELEMS
+        linear_bytes += 2 * O_PROJ_ELEMS + batch * Q_WIDTH * 2 + batch * HIDDEN * 2
     return StepCounts(batch, positions, attn_flops, float(attn_bytes), linear_flops,
                       float(linear_bytes))
 
@@ -92,6 +98,18 @@ def layer_roofline(c: StepCounts, measured_step_s: float, hbm_gbs: float,
             "linear_us": t.linear_s * 1e6, "attention_bound": t.attn_bound,
             "linear_bound": t.linear_bound,
             "gpu_seconds_per_m_tokens": t.gpu_seconds_per_m}
+
+
+def stack_roofline(c: StepCounts, layers: int, measured_step_s: float, hbm_gbs: float,
+                   tensor_tflops: float) -> dict:
+    """A stack of ``layers`` identical layer steps (each counted by ``c``) against a measured
+    time for the whole stack."""
+    t = step_times(c, hbm_gbs, tensor_tflops)
+    model = t.step_s * layers
+    return {"model_us": model * 1e6, "measured_us": measured_step_s * 1e6,
+            "frac": model / measured_step_s, "layers": layers,
+            "model_us_per_layer": t.step_s * 1e6,
+            "measured_us_per_layer": measured_step_s * 1e6 / layers}
 
 
 def main(argv: Optional[list] = None) -> None:

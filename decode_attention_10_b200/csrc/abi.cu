@@ -334,6 +334,37 @@ mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t*
   return run_attention(aa, static_cast<cudaStream_t>(stream));
 }
 
+mfa_status mfa_o_proj(const void* out, const void* w_o, void* y, int32_t batch, void* ws,
+                      size_t ws_bytes, void* stream) {
+  if (batch < 1 || batch > kMaxBatch) return MFA_ERR_INVALID_ARG;
+  const void* ptrs[] = {out, w_o, y};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  mfa_status st = check_ws(ws, ws_bytes, batch, &L);
+  if (st != MFA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // W_o^T tiles of 128 output features on the M side, out [batch, 16384] on the N side
+  CUtensorMap wm[3];
+  std::memset(wm, 0, sizeof(wm));
+  if (!encode_2d(&wm[0], w_o, kQWidth, kHidden, 2, 64, 128)) return MFA_ERR_CUDA;
+  CUtensorMap xm;
+  if (!encode_2d(&xm, out, (uint64_t)batch, kQWidth, 2, 64, wgemm_n_box(batch)))
+    return MFA_ERR_CUDA;
+  float* part = at<float>(ws, L.oproj_part);
+  WGemmArgs p{};
+  p.batch = batch;
+  p.tile_begin = 0;
+  p.three_weights = 0;
+  p.kblocks_per_cta = kOProjKPerSplit / 128;
+  p.out_f32 = part;
+  p.out_ld = kHidden;
+  p.err = at<uint32_t>(ws, L.err);
+  if (launch_wgemm(wm, xm, p, kHidden / 128, kOProjSplits, s) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  return cuda_status(launch_oproj_finish(part, static_cast<uint16_t*>(y), batch, s));
+}
+
 mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamma,
                             const void* w_qup, const void* w_k, const void* w_v, float eps,
                             const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,

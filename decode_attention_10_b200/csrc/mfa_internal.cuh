@@ -24,6 +24,11 @@ constexpr int kXProjSplits = 7;                   // split-K of the 7168-long re
 constexpr int kXProjKPerSplit = kHidden / kXProjSplits;  // 1024
 static_assert(kHidden % kXProjSplits == 0, "split-K must divide the hidden width");
 
+// Output projection out [B, 16384] -> y [B, 7168]: split-K of the 16384-long reduction
+// (56 tiles of 128 features x 2 splits = 112 CTAs).
+constexpr int kOProjSplits = 2;
+constexpr int kOProjKPerSplit = kQWidth / kOProjSplits;  // 8192
+
 // Attention work unit: the plan hands out whole tiles of this many cached positions.
 constexpr int kTile = 128;
 
@@ -58,6 +63,7 @@ struct WsLayout {
   size_t attn_part;    // partial slots
   size_t xproj_part;   // fp32 [kXProjSplits][batch][kXProjCols]
   size_t c_hat;        // bf16 [batch][kRank]
+  size_t oproj_part;   // fp32 [kOProjSplits][batch][kHidden]
   size_t total;
   int attn_slots;
   int attn_grid;
@@ -85,6 +91,8 @@ inline WsLayout ws_layout(int batch, int num_sms) {
   off = align_up(off + sizeof(float) * kXProjSplits * (size_t)batch * kXProjCols, 256);
   L.c_hat = off;
   off = align_up(off + sizeof(uint16_t) * (size_t)batch * kRank, 256);
+  L.oproj_part = off;
+  off = align_up(off + sizeof(float) * kOProjSplits * (size_t)batch * kHidden, 256);
   L.total = off;
   return L;
 }
@@ -158,6 +166,9 @@ struct FinishArgs {
   int attn_grid;
 };
 cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s);
+
+// y = bf16(partial[0] + partial[1]) over batch x 7168 fp32 partials (out_proj.cu).
+cudaError_t launch_oproj_finish(const float* part, uint16_t* y, int batch, cudaStream_t s);
 
 
 struct AttnArgs {

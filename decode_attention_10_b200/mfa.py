@@ -40,6 +40,7 @@ _SIGNATURES = {
                                        _P]),
     "mfa_decode_layer": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
                                         ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
+    "mfa_o_proj": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "mfa_query_proj_noalloc": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_float, _P,
                                               ctypes.c_int32, _P]),
     "mfa_wait_selftest": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_uint32, _P]),
@@ -224,6 +225,19 @@ def decode_layer(x, w_qdown, gamma, w_qup, w_k, w_v, cache: KVCache, seq_lens,
                                 ws.nbytes, _stream(stream)),
            "mfa_decode_layer")
     return q_out, out
+
+
+def o_proj(out, w_o, y=None, ws=None, stream=None) -> torch.Tensor:
+    """y = bf16(out W_o): the attention output [B, 64, 256] (or [B, 16384]) projected back to
+    the hidden width 7168."""
+    lib = load()
+    bsz = int(out.shape[0])
+    if y is None:
+        y = torch.empty(bsz, HIDDEN, dtype=torch.bfloat16, device=out.device)
+    ws = ws if ws is not None else Workspace(bsz, out.device)
+    _check(lib.mfa_o_proj(_ptr(out), _ptr(w_o), _ptr(y), bsz, ws.ptr, ws.nbytes,
+                          _stream(stream)), "mfa_o_proj")
+    return y
 
 
 def query_proj_noalloc(x, w_qdown, gamma, w_qup, eps: float = 1e-6, q_out=None, stream=None):

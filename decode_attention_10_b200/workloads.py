@@ -166,6 +166,54 @@ def generate(seq_lens: Sequence[int], kv_dtype: str = KV_BF16, seed: int = 0,
                   v_buffer=v_buf, meta=dict(seed=int(seed), capacity=caps))
 
 
+def generate_w_o(seed: int) -> torch.Tensor:
+    """The output projection W_o [16384, 7168] of one layer, bf16 ~ N(0, 1/16384) (the same
+    fan-in scaling as the other projections)."""
+    g = torch.Generator().manual_seed(int(seed))
+    width = N_HEADS * HEAD_DIM
+    return _randn(g, width, HIDDEN, std=width ** -0.5).to(torch.bfloat16)
+
+
+def generate_layer_on_device(seq_lens: Sequence[int], kv_dtype: str, seed: int, device,
+                             contiguous: bool = True) -> dict:
+    """One layer's weights (W_qdown, gamma, W_qup, W_k, W_v, W_o) and KV cache drawn on the
+    device with the distributions of ``generate`` and ``generate_w_o``, for stacks of many
+    layers whose tensors would take minutes to draw on the host. Returns a dict with those
+    tensors, k_cache / v_cache (per-sequence views) and k_scale / v_scale."""
+    lens = [int(n) for n in seq_lens]
+    bsz = len(lens)
+    g = torch.Generator(device=device).manual_seed(int(seed))
+
+    def randn(*shape, std=1.0):
+        t = torch.randn(*shape, generator=g, dtype=torch.float32, device=device)
+        return t.mul_(std) if std != 1.0 else t
+
+    width = N_HEADS * HEAD_DIM
+    d = dict(w_qdown=randn(HIDDEN, Q_RANK, std=HIDDEN ** -0.5).to(torch.bfloat16),
+             w_qup=randn(Q_RANK, width, std=Q_RANK ** -0.5).to(torch.bfloat16),
+             w_k=randn(HIDDEN, HEAD_DIM, std=HIDDEN ** -0.5).to(torch.bfloat16),
+             w_v=randn(HIDDEN, HEAD_DIM, std=HIDDEN ** -0.5).to(torch.bfloat16),
+             w_o=randn(width, HIDDEN, std=width ** -0.5).to(torch.bfloat16),
+             gamma=torch.ones(Q_RANK, dtype=torch.bfloat16, device=device))
+    for name in ("k", "v"):
+        if contiguous:
+            vals = [randn(bsz, max(lens), HEAD_DIM)]
+        else:
+            vals = [randn(n, HEAD_DIM) for n in lens]
+        if kv_dtype == KV_BF16:
+            scale = 1.0
+            store = [t.to(torch.bfloat16) for t in vals]
+        else:
+            amax = max(float(t.abs().max()) for t in vals)
+            scale = float(torch.tensor(amax / 448.0, dtype=torch.float32)) if amax else 1.0
+            store = [(t / scale).to(torch.float8_e4m3fn) for t in vals]
+        del vals
+        d[name + "_scale"] = scale
+        d[name + "_buffer"] = store
+        d[name + "_cache"] = [store[0][b] for b in range(bsz)] if contiguous else store
+    return d
+
+
 def ragged_lengths(batch: int, seed: int) -> list:
     """Per-sequence lengths drawn uniform in [1, 65536] -- the first draw of the seed."""
     g = torch.Generator().manual_seed(int(seed))

@@ -160,7 +160,8 @@ MFA_API mfa_status mfa_kv_append(const void* x, const void* w_k, const void* w_v
  * with K_b, V_b the cache rows (e4m3 codes times their scale for FP8 caches).
  * q: device bf16 [kv->batch, 64, 256]; seq_lens: device int32 [kv->batch]; out: device
  * bf16 [kv->batch, 64, 256]; scale > 0 (1/16 for the layer). The work is split over the
- * GPU's SMs by length (split-K over the cache, merged in the same kernel). A sequence with
+ * GPU's SMs by length (split-K over the cache; a second kernel on the same stream merges
+ * the splits). A sequence with
  * L_b == 0 or L_b > capacity[b] gets a zero output and sets MFA_ERR_EMPTY /
  * MFA_ERR_CAPACITY in the workspace. */
 MFA_API mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t* seq_lens,
@@ -174,6 +175,20 @@ MFA_API mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const vo
                             const void* w_qup, const void* w_k, const void* w_v, float eps,
                             const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
                             void* q_out, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Output projection of the attention (pages: bud-325 "Method" -- the per-token decoding
+ * cost counts the linear projections around attention, and each layer's attention hands a
+ * hidden-width vector to the FFN; the 16384 -> 7168 shape is the reading that the 64 x 256
+ * head outputs return to the hidden width 7168):
+ *   y = bf16(out W_o), fp32 accumulation.
+ * out: device bf16 [batch, 64 * 256] (the attention output, heads in order, as written by
+ * mfa_decode_attn / mfa_decode_layer); w_o: device bf16 [16384, 7168], row-major [in, out];
+ * y: device bf16 [batch, 7168]. 1 <= batch <= MFA_MAX_BATCH.
+ * ws: device workspace of mfa_workspace_bytes(batch) bytes (initialized once); it holds the
+ * split-K partials. Errors: INVALID_ARG (null/misaligned pointer, batch out of range),
+ * WORKSPACE (ws too small), CUDA (launch failure). */
+MFA_API mfa_status mfa_o_proj(const void* out, const void* w_o, void* y, int32_t batch,
+                              void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Without a caller-provided workspace

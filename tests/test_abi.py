@@ -96,6 +96,11 @@ def test_invalid_arguments_are_rejected_before_any_device_work(lib):
     kv = mfa.KvCacheDesc(4, 0, 1.0, 1.0, 4096)
     assert lib.mfa_decode_layer(fake, fake, fake, fake, fake, fake, 1e-6, ctypes.byref(kv),
                                 fake, -1.0, fake, fake, fake, 1 << 30, None) == 1
+    # output projection: batch range, null / misaligned pointers
+    assert lib.mfa_o_proj(fake, fake, fake, 0, fake, 1 << 30, None) == 1
+    assert lib.mfa_o_proj(fake, fake, fake, 1025, fake, 1 << 30, None) == 1
+    assert lib.mfa_o_proj(None, fake, fake, 4, fake, 1 << 30, None) == 1
+    assert lib.mfa_o_proj(fake, fake, P(4104), 4, fake, 1 << 30, None) == 1
     # table init: bad batch, null arrays, unknown dtype, table too small, capacity range
     arr = (ctypes.c_void_p * 2)(4096, 8192)
     caps = (ctypes.c_int32 * 2)(16, 16)

@@ -57,3 +57,18 @@ def test_workload_lens_match_the_generator():
     assert cm.step_counts(W.workload_lens(w), w.kv_dtype).batch == 16
     assert W.workload_lens(w) == W.ragged_lengths(16, 1004)
     assert W.workload_lens(W.workload(1)) == [4096] * 32
+
+
+def test_o_proj_counts_and_stack_model():
+    base = cm.step_counts([4096] * 32, "bf16")
+    full = cm.step_counts([4096] * 32, "bf16", o_proj=True)
+    assert cm.O_PROJ_ELEMS == 16384 * 7168
+    assert full.linear_flops - base.linear_flops == 2 * 32 * 16384 * 7168
+    # W_o once (234,881,024 B) + out read + y written
+    assert full.linear_bytes - base.linear_bytes == 234_881_024 + 32 * 16384 * 2 + 32 * 7168 * 2
+    assert full.attn_bytes == base.attn_bytes
+    t = cm.step_times(full, 1000.0, 1000.0)
+    r = cm.stack_roofline(full, 61, 61 * 2 * t.step_s, 1000.0, 1000.0)
+    assert r["frac"] == pytest.approx(0.5)
+    assert r["model_us_per_layer"] == pytest.approx(t.step_s * 1e6)
+    assert r["measured_us_per_layer"] == pytest.approx(2 * t.step_s * 1e6)

@@ -340,3 +340,90 @@ def test_named_workload_sampled(index):
     b = inp.batch
     sample = sorted(set([0, b // 3, b // 2, b - 1]))
     _check_layer(inp, sample=sample, e2e=True)
+
+
+# ----------------------------------------------------------------------------------------
+# output projection, and the attention side of a step through a stack of layers
+# ----------------------------------------------------------------------------------------
+
+
+def _y_close(y_gpu, y_ref):
+    # y is stored as bf16, so the float64 reference is rounded to bf16 as the oracle's
+    # emulation does for stored tensors; then two bf16 ulps plus a small absolute slack
+    y_ref = codecs.bf16_round(y_ref)
+    ulp = np.ldexp(1.0, np.frexp(np.abs(y_ref))[1] - 8)
+    bad = np.abs(y_gpu - y_ref) > 2 * ulp + 1e-4
+    assert not bad.any(), f"{bad.sum()} y elements off, max {max_abs(y_gpu, y_ref):.3e}"
+    assert rel_l2(y_gpu, y_ref) <= 1e-3
+
+
+@pytest.mark.parametrize("bsz", [1, 32, 300])
+def test_o_proj_matches_oracle(bsz):
+    from decode_attention_10_b200 import mfa
+    g = torch.Generator().manual_seed(40 + bsz)
+    out = (torch.randn(bsz, 64, 256, generator=g) * 0.05).to(torch.bfloat16)
+    w_o = W.generate_w_o(41)
+    y = mfa.o_proj(out.cuda(), w_o.cuda())
+    torch.cuda.synchronize()
+    # every 7th output column: all 56 tiles of 128 features, both split-K halves
+    cols = np.arange(0, 7168, 7)
+    ref = omfa.o_proj(bf16_np(out), bf16_np(w_o[:, cols]))
+    _y_close(bf16_np(y)[:, cols], ref)
+
+
+def test_o_proj_bit_exact_on_small_integers():
+    # integer inputs: every fp32 partial sum is exact (|y| <= 16384 * 6 < 2**24), so the
+    # split-K order cannot matter and y must equal bf16(exact) bit for bit
+    from decode_attention_10_b200 import mfa
+    g = torch.Generator().manual_seed(43)
+    out = torch.randint(-3, 4, (40, 64, 256), generator=g).to(torch.bfloat16)
+    w_o = torch.randint(-2, 3, (16384, 7168), generator=g).to(torch.bfloat16)
+    y = mfa.o_proj(out.cuda(), w_o.cuda())
+    torch.cuda.synchronize()
+    cols = np.arange(3, 7168, 11)
+    exact = omfa.o_proj(bf16_np(out), bf16_np(w_o[:, cols]))
+    got = codes_np(y)[:, cols]
+    assert np.array_equal(got, codecs.bf16_encode(exact))
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_attention_side_two_layers(kv_dtype):
+    """Two layers chained on one stream as a serving loop runs them: layer 1's hidden input
+    is layer 0's projected output. Per layer the oracle reads the GPU's own inputs of that
+    layer; end to end it runs its own chain from x and the original caches."""
+    from decode_attention_10_b200 import mfa
+    lens = [1, 130, 300]
+    inps = [W.generate(lens, kv_dtype, seed=60 + l) for l in range(2)]
+    w_os = [W.generate_w_o(70 + l) for l in range(2)]
+    steps = [GpuStep(inp) for inp in inps]
+    k_before = [[codes_np(t) for t in st.k] for st in steps]
+    v_before = [[codes_np(t) for t in st.v] for st in steps]
+    x = steps[0].x
+    xs, outs, ys = [], [], []
+    for st, w_o in zip(steps, w_os):
+        _, out = mfa.decode_layer(x, st.w_qdown, st.gamma, st.w_qup, st.w_k, st.w_v, st.cache,
+                                  st.seq_lens, ws=st.ws)
+        y = mfa.o_proj(out, w_o.cuda(), ws=st.ws)
+        xs.append(x)
+        outs.append(out)
+        ys.append(y)
+        x = y
+    torch.cuda.synchronize()
+    assert all(mfa.get_error(st.ws) == 0 for st in steps)
+    od = oracle_dtype(kv_dtype)
+    layers = []
+    for l, (inp, st) in enumerate(zip(inps, steps)):
+        ow = oracle_weights(inp)
+        lay = dict(w_qdown=ow["w_qdown"], gamma=ow["gamma"], w_qup=ow["w_qup"], w_k=ow["w_k"],
+                   w_v=ow["w_v"], w_o=bf16_np(w_os[l]), k_cache=k_before[l],
+                   v_cache=v_before[l], k_scale=inp.k_scale, v_scale=inp.v_scale)
+        layers.append(lay)
+        # per layer: the GPU's own hidden input of this layer
+        r = omfa.decode_layer(bf16_np(xs[l]), lay["w_qdown"], lay["gamma"], lay["w_qup"],
+                              lay["w_k"], lay["w_v"], lay["k_cache"], lay["v_cache"], lens, od,
+                              inp.k_scale, inp.v_scale)
+        assert_close(bf16_np(outs[l]), r["out"], kv_dtype, f"layer {l} attention")
+        _y_close(bf16_np(ys[l]), omfa.o_proj(bf16_np(outs[l]), lay["w_o"]))
+    # end to end through both layers: two layers' worth of the per-layer tolerance
+    _, y_ref = omfa.attention_side_step(oracle_weights(inps[0])["x"], layers, lens, od)
+    assert rel_l2(bf16_np(ys[-1]), y_ref) <= 2 * 5e-3
