@@ -54,6 +54,11 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--page-size", type=int, default=0,
+                   help="keep the KV cache in shuffled pages of this many rows (a multiple of "
+                        "64) behind a page table, instead of one buffer per sequence")
+    p.add_argument("--page-order", choices=["shuffled", "sequential"], default="shuffled",
+                   help="with --page-size: pages handed out in random or in sequence order")
     p.add_argument("--layers", type=int, default=0,
                    help="time the attention side of a whole decode step instead: this many "
                         "layers, each the MFA decode step plus its output projection")
@@ -258,7 +263,14 @@ def run_ours(args, wl, rank, world, local):
         else:
             c.k = [t.to(dev) for t in inp.k_cache]
             c.v = [t.to(dev) for t in inp.v_cache]
-        c.cache = mfa.KVCache(c.k, c.v, inp.k_scale, inp.v_scale)
+        if args.page_size:
+            kp, vp, pt, npages = W.to_paged(c.k, c.v, args.page_size, seed=len(sets),
+                                            shuffle=args.page_order == "shuffled")
+            c.keep = (kp, vp, pt)
+            c.k = c.v = None
+            c.cache = mfa.PagedKVCache(kp, vp, pt, npages, inp.k_scale, inp.v_scale)
+        else:
+            c.cache = mfa.KVCache(c.k, c.v, inp.k_scale, inp.v_scale)
         c.q = torch.empty(bsz, 64, 256, dtype=torch.bfloat16, device=dev)
         c.out = torch.empty(bsz, 64, 256, dtype=torch.bfloat16, device=dev)
         sets.append(c)
@@ -396,7 +408,7 @@ def run_ours(args, wl, rank, world, local):
     peak, peak_kind = measured_peaks()
     a_bytes = attention_bytes(inp)
     achieved = a_bytes / (attn_ms / 1e3) / 1e9
-    traffic = profiled_traffic(wl.name)
+    traffic = None if args.page_size else profiled_traffic(wl.name)
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -404,6 +416,8 @@ def run_ours(args, wl, rank, world, local):
         "dtype": "bf16" if inp.kv_dtype == "bf16" else "bf16+fp8kv", "data": "synthetic",
         "config": {"workload": wl.name, "batch_per_gpu": bsz, "global_batch": bsz * world,
                    "context": wl.context, "kv_dtype": inp.kv_dtype,
+                   "kv_layout": (f"paged, {args.page_size} rows per page, {args.page_order}"
+                                 if args.page_size else "one buffer per sequence"),
                    "heads": 64, "head_dim": 256, "hidden": 7168, "q_rank": 2048,
                    "l2": f"inputs rotate over {copies} device copies "
                          f"({step_bytes / 1e6:.0f} MB each, > 126 MB L2)",

@@ -46,6 +46,8 @@ mfa_status check_kv(const mfa_kv_cache* kv) {
   if (kv->dtype != MFA_KV_BF16 && kv->dtype != MFA_KV_FP8_E4M3) return MFA_ERR_UNSUPPORTED;
   if (kv->dtype == MFA_KV_FP8_E4M3 && !(kv->k_scale > 0.f && kv->v_scale > 0.f))
     return MFA_ERR_INVALID_ARG;
+  const int ps = kv->page_size;
+  if (ps != 0 && (ps < 64 || (ps & (ps - 1)) != 0)) return MFA_ERR_INVALID_ARG;
   return MFA_OK;
 }
 
@@ -158,6 +160,23 @@ bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, i
   return r == CUDA_SUCCESS;
 }
 
+bool encode_pool(CUtensorMap* m, const void* base, uint64_t pages, uint64_t page_rows,
+                 int elem_bytes, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (enc == nullptr) return false;
+  const uint64_t row_bytes = (uint64_t)kHeadDim * elem_bytes;
+  cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)page_rows, (cuuint64_t)pages};
+  cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)(row_bytes * page_rows)};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / elem_bytes), box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(
+      m, elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+      const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 // The attention of one call: the tensor-core kernel, then the merge of split sequences.
@@ -230,6 +249,54 @@ mfa_status mfa_kv_table_init(void* table, size_t table_bytes, int32_t batch, int
   return cuda_status(e);
 }
 
+mfa_status mfa_kv_table_init_paged(void* table, size_t table_bytes, int32_t batch,
+                                   int32_t dtype, void* k_pool, void* v_pool, int32_t num_pages,
+                                   int32_t page_size, const int32_t* page_table,
+                                   int32_t max_pages, const int32_t* pages_per_seq,
+                                   void* stream) {
+  if (batch < 1 || batch > kMaxBatch) return MFA_ERR_INVALID_ARG;
+  if (table == nullptr || k_pool == nullptr || v_pool == nullptr || page_table == nullptr ||
+      pages_per_seq == nullptr)
+    return MFA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(table) & 127u) != 0) return MFA_ERR_INVALID_ARG;
+  if (!aligned16(k_pool) || !aligned16(v_pool) ||
+      (reinterpret_cast<uintptr_t>(page_table) & 3u) != 0)
+    return MFA_ERR_INVALID_ARG;
+  if (dtype != MFA_KV_BF16 && dtype != MFA_KV_FP8_E4M3) return MFA_ERR_UNSUPPORTED;
+  if (page_size < 64 || (page_size & (page_size - 1)) != 0 || page_size > MFA_MAX_CONTEXT)
+    return MFA_ERR_UNSUPPORTED;
+  if (num_pages < 1 || max_pages < 1) return MFA_ERR_INVALID_ARG;
+  if (table_bytes < mfa_kv_table_bytes(batch)) return MFA_ERR_WORKSPACE;
+  for (int b = 0; b < batch; ++b) {
+    const int64_t cap = (int64_t)pages_per_seq[b] * page_size;
+    if (pages_per_seq[b] < 1 || pages_per_seq[b] > max_pages || cap > MFA_MAX_CONTEXT)
+      return MFA_ERR_INVALID_ARG;
+  }
+  if (encode_tiled_fn() == nullptr) return MFA_ERR_CUDA;
+  const int elem = dtype == MFA_KV_FP8_E4M3 ? 1 : 2;
+  KvSeq proto;
+  std::memset(&proto, 0, sizeof(proto));
+  if (!encode_pool(&proto.tmap_k, k_pool, num_pages, page_size, elem,
+                   paged_box_rows(page_size)) ||
+      !encode_pool(&proto.tmap_v, v_pool, num_pages, page_size, elem,
+                   paged_box_rows(page_size)))
+    return MFA_ERR_INVALID_ARG;
+  proto.k = k_pool;
+  proto.v = v_pool;
+  proto.page_size = page_size;
+  proto.num_pages = num_pages;
+  std::vector<KvSeq> host(batch, proto);
+  for (int b = 0; b < batch; ++b) {
+    host[b].capacity = pages_per_seq[b] * page_size;
+    host[b].pages = page_table + (size_t)b * max_pages;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(table, host.data(), sizeof(KvSeq) * batch,
+                                  cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e);
+}
+
 size_t mfa_workspace_bytes(int32_t batch) {
   if (batch < 1 || batch > kMaxBatch) return 0;
   int sms = 0;
@@ -257,6 +324,7 @@ mfa_status mfa_get_error(void* ws, void* stream) {
   if (cudaStreamSynchronize(s) != cudaSuccess) return MFA_ERR_CUDA;
   if (bits & kErrCapacity) return MFA_ERR_CAPACITY;
   if (bits & kErrEmpty) return MFA_ERR_EMPTY;
+  if (bits & kErrLayout) return MFA_ERR_INVALID_ARG;
   return MFA_ERR_TIMEOUT;
 }
 
@@ -331,6 +399,7 @@ mfa_status mfa_decode_attn(const void* q, const mfa_kv_cache* kv, const int32_t*
   aa.plan_early = 0;
   aa.err = at<uint32_t>(ws, L.err);
   aa.grid = L.attn_grid;
+  aa.page_size = kv->page_size;
   return run_attention(aa, static_cast<cudaStream_t>(stream));
 }
 
@@ -396,6 +465,7 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   aa.plan_early = 1;
   aa.err = at<uint32_t>(ws, L.err);
   aa.grid = L.attn_grid;
+  aa.page_size = kv->page_size;
   // one projection of x onto [W_qdown | W_k | W_v]
   float* part = at<float>(ws, L.xproj_part);
   st = run_xproj(x, w_qdown, w_k, w_v, batch, 0, kXProjCols / 128, part,

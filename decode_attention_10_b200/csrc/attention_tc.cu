@@ -70,6 +70,7 @@ constexpr int kPBytes = 16384;          // P^T: [128 positions x 64 heads] 16-bi
 constexpr uint32_t kTmemS = 0;          // S^T buffers: columns [0, 64) and [64, 128)
 constexpr uint32_t kTmemO = 128;        // O^T halves: columns [128, 192) and [192, 256)
 constexpr uint32_t kTmemK = 256;        // FP8: f16 K tiles (A operand), [256, 384), [384, 512)
+constexpr int kPageIds = 128;          // paged caches: page ids held per work item
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // named barriers: 1 + group among one softmax group, 3 among all eight softmax warps
@@ -116,7 +117,12 @@ struct __align__(1024) TcSmem {
   uint64_t mma_done;
   uint32_t tmem_base;
   int32_t abort_flag;
+  int32_t page_ids[2][kPageIds];  // paged caches: the first page ids of this and the next item
 };
+
+// the dynamic shared memory of one CTA (TcSmem plus its 1024-byte alignment) fits the
+// 227 KB a block may have
+static_assert(sizeof(TcSmem) + 1024 <= 232448, "shared memory per CTA");
 
 // bf16: ring chunk `slot`
 __device__ __forceinline__ uint8_t* ring_chunk(TcSmem& S, uint32_t slot) {
@@ -140,10 +146,29 @@ __device__ __forceinline__ int num_tiles(const WorkItem& it) {
 }
 
 // Window of tile t of an item: rows [y, y + 128) are loaded, positions [a, e) are used.
-__device__ __forceinline__ void tile_window(const WorkItem& it, int t, int& y, int& a, int& e) {
+// Contiguous caches: an item's last window slides back to end at the item's end, so no row
+// past the sequence is read (rows before a are the sequence's own, or zero-filled below row
+// 0). Paged caches: windows stay on 128-position boundaries, so each 64-row half lies in one
+// page; rows [e, y + 128) past the sequence's end are loaded (from its last page, or zeros
+// past it) and their V values zeroed on chip.
+__device__ __forceinline__ void tile_window(const WorkItem& it, int t, bool paged, int& y,
+                                            int& a, int& e) {
   a = it.tok0 + t * kTile;
   e = min(a + kTile, it.tok1);
-  y = (a + kTile <= it.tok1) ? a : it.tok1 - kTile;
+  y = (paged || a + kTile <= it.tok1) ? a : it.tok1 - kTile;
+}
+
+// Paged caches: rows of a window whose V values are used (the rest are zeroed before PV).
+__device__ __forceinline__ int window_rows_kept(bool paged, int y, int e) {
+  return paged ? e - y : kTile;
+}
+
+// Zero rows [from, 128) of a [128 x 128 B] 16-bit chunk (row r is bytes [128 r, 128 r + 128)
+// whatever the swizzle), by the 32 lanes of a warp.
+__device__ __forceinline__ void zero_chunk_rows(uint8_t* chunk, int from, int lane) {
+  uint4* p = reinterpret_cast<uint4*>(chunk + from * 128);
+  const int n = (kTile - from) * 8;
+  for (int i = lane; i < n; i += 32) p[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
@@ -240,12 +265,17 @@ __device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) 
 // ---------------------------------------------------------------------------------------
 // warp 0: TMA producer
 // ---------------------------------------------------------------------------------------
-template <bool kFp8>
+template <bool kFp8, bool kPaged>
 __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs& a, int g,
                              bool leader) {
   using C = Cfg<kFp8>;
   constexpr uint32_t kN = C::kSlots;
   volatile int* abort = &S.abort_flag;
+  const int lane = threadIdx.x & 31;
+  constexpr bool paged = kPaged;
+  const int page_size = kPaged ? S.plan.page_size : 1;  // read only by the paged code
+  const int page_shift = 31 - __clz(page_size);         // page sizes are powers of two
+  const int box_rows = kPaged ? paged_box_rows(page_size) : kTile;
   uint32_t chunk = 0, issued = 0;                 // bf16: ring chunks
   uint32_t kb = 0, kb_issued = 0, vb = 0, vb_issued = 0;  // FP8: raw K and V boxes
   int item = 0, q_issued = 0;
@@ -268,35 +298,75 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   // straight into the ring. FP8: per tile K(t) (two raw [128 x 128] e4m3 boxes into the K
   // raw slots), then V(t) (two raw boxes into the upper halves of two V slots).
   constexpr int kBoxesPerTile = kFp8 ? 4 : 8;
+  // Paged caches: the page ids of work item k, pages [p0, p_last] of its sequence (p_last =
+  // the page of its last position), sit in S.page_ids[k & 1] (the first kPageIds of them; the
+  // leader reads any further id straight from the table). Each lane fetches its share of the
+  // next item's ids into registers while the current item streams, and stores them when
+  // that item begins, so no copy waits for the page table.
+  constexpr int kIdsPerLane = kPageIds / 32;
+  int32_t ids_next[kIdsPerLane];
+  auto first_page = [&](const WorkItem& w) { return w.tok0 >> page_shift; };
+  auto last_page = [&](const WorkItem& w) { return (w.tok1 - 1) >> page_shift; };
+  auto fetch_ids = [&](const WorkItem& w) {
+    const int32_t* pages = a.kv[w.b].pages;
+    const int p0 = first_page(w), n = last_page(w) - p0 + 1;
+#pragma unroll
+    for (int k = 0; k < kIdsPerLane; ++k) {
+      const int i = lane + 32 * k;
+      ids_next[k] = i < n ? pages[p0 + i] : 0;
+    }
+  };
+  auto store_ids = [&](int buf) {
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < kIdsPerLane; ++k) S.page_ids[buf][lane + 32 * k] = ids_next[k];
+    __syncwarp();
+  };
+  // one box of 128 rows at window row y: a 2-D load, or for a paged cache 128 / box_rows
+  // 3-D loads of box_rows rows, each from its page. Every lane makes the page lookups (the
+  // refills are warp-wide); the leader issues the copies if ok.
+  auto load_rows = [&](uint8_t* dst, const CUtensorMap* map, int x, const WorkItem& w, int y,
+                       uint64_t* bar, uint64_t policy, bool ok) {
+    if constexpr (!kPaged) {
+      if (leader && ok) tma_load_2d_hint(dst, map, x, y, bar, policy);
+    } else {
+      // rows past the item's last page (the sequence's end) are read from that page at a
+      // row >= page_size, which the tensor map fills with zeros
+      const int p0 = first_page(w), pl = last_page(w);
+      for (int r0 = 0; r0 < kTile; r0 += box_rows) {
+        const int pos = y + r0;  // >= 0: paged windows start on tile boundaries
+        const int pidx = min(pos >> page_shift, pl);
+        if (leader && ok) {
+          const int i = pidx - p0;
+          const int page = i < kPageIds ? S.page_ids[item & 1][i] : a.kv[w.b].pages[pidx];
+          tma_load_3d_hint(dst + r0 * 128, map, x, pos - (pidx << page_shift), page, bar, policy);
+        }
+      }
+    }
+  };
   auto issue_box = [&](const WorkItem& w, int j) {
     const KvSeq* seq = a.kv + w.b;
     int y, a0, e0;
     if constexpr (kFp8) {
       const int t = j >> 2, r = j & 3;
-      tile_window(w, t, y, a0, e0);
+      tile_window(w, t, paged, y, a0, e0);
       if (r < 2) {
         const uint32_t slot = kb % kKRawSlots, use = kb / kKRawSlots;
         if (use > 0) mbar_wait(&S.raw_empty[slot], (use - 1) & 1, abort);
-        if (!*abort) {
-          if (leader) {
-            mbar_arrive_expect_tx(&S.raw_full[slot], kRawBytes);
-            tma_load_2d_hint(k_raw(S, slot), &seq->tmap_k, 128 * r, y, &S.raw_full[slot],
-                             evict_first);
-          }
-          kb_issued = kb + 1;
-        }
+        const bool ok = !*abort;
+        if (leader && ok) mbar_arrive_expect_tx(&S.raw_full[slot], kRawBytes);
+        load_rows(k_raw(S, slot), &seq->tmap_k, 128 * r, w, y, &S.raw_full[slot],
+                  evict_first, ok);
+        if (ok) kb_issued = kb + 1;
         ++kb;
       } else {
         const uint32_t slot = vb % kVSlots, use = vb / kVSlots;
         if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);  // PV(t - 2) done
-        if (!*abort) {
-          if (leader) {
-            mbar_arrive_expect_tx(&S.vraw_full[slot], kRawBytes);
-            tma_load_2d_hint(v_slot(S, slot) + kChunkBytes, &seq->tmap_v, 128 * (r - 2), y,
-                             &S.vraw_full[slot], evict_first);
-          }
-          vb_issued = vb + 1;
-        }
+        const bool ok = !*abort;
+        if (leader && ok) mbar_arrive_expect_tx(&S.vraw_full[slot], kRawBytes);
+        load_rows(v_slot(S, slot) + kChunkBytes, &seq->tmap_v, 128 * (r - 2), w, y,
+                  &S.vraw_full[slot], evict_first, ok);
+        if (ok) vb_issued = vb + 1;
         ++vb;
       }
     } else {
@@ -312,17 +382,14 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
         else
           is_v = true, t = n - 1, c = rr;
       }
-      tile_window(w, t, y, a0, e0);
+      tile_window(w, t, paged, y, a0, e0);
       const uint32_t slot = chunk % kN, use = chunk / kN;
       if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);
-      if (!*abort) {
-        if (leader) {
-          mbar_arrive_expect_tx(&S.kv_full[slot], kChunkBytes);
-          tma_load_2d_hint(ring_chunk(S, slot), is_v ? &seq->tmap_v : &seq->tmap_k, 64 * c, y,
-                           &S.kv_full[slot], evict_first);
-        }
-        issued = chunk + 1;
-      }
+      const bool ok = !*abort;
+      if (leader && ok) mbar_arrive_expect_tx(&S.kv_full[slot], kChunkBytes);
+      load_rows(ring_chunk(S, slot), is_v ? &seq->tmap_v : &seq->tmap_k, 64 * c, w, y,
+                &S.kv_full[slot], evict_first, ok);
+      if (ok) issued = chunk + 1;
       ++chunk;
     }
   };
@@ -331,6 +398,13 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   // ring-full for bf16, K(0) and V(0) for FP8 -- stream in while the previous kernel (which
   // writes q) finishes.
   int first_done = 0;
+  if constexpr (kPaged) {
+    if (has) {
+      fetch_ids(it);
+      store_ids(0);
+      if (has_nx) fetch_ids(nx);
+    }
+  }
   if (has) {
     const int total = kBoxesPerTile * num_tiles(it);
     const int pre = kFp8 ? 4 : static_cast<int>(kN);
@@ -339,6 +413,12 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   }
   pdl_wait();
   while (has) {
+    if constexpr (kPaged) {
+      if (item > 0) {  // this item's ids, fetched while the previous one streamed
+        store_ids(item & 1);
+        if (has_nx) fetch_ids(nx);
+      }
+    }
     if (has_nx && leader) {
       prefetch_tensormap(&a.kv[nx.b].tmap_k);
       prefetch_tensormap(&a.kv[nx.b].tmap_v);
@@ -380,17 +460,24 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
 // ---------------------------------------------------------------------------------------
 // warp 1 (one elected lane issues): MMA
 // ---------------------------------------------------------------------------------------
-template <bool kFp8>
+template <bool kFp8, bool kPaged>
 __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool leader) {
   using C = Cfg<kFp8>;
   constexpr uint32_t kSlots = C::kSlots;
   volatile int* abort = &S.abort_flag;
+  const int lane = threadIdx.x & 31;
+  constexpr bool paged = kPaged;
   uint32_t chunk = 0;
   uint32_t gt = 0;  // tiles issued so far by this CTA (all items)
   int item = 0;
 
   plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem& it) {
     const int n = num_tiles(it);
+    auto rows_kept = [&](int t) {
+      int y, a0, e0;
+      tile_window(it, t, paged, y, a0, e0);
+      return window_rows_kept(paged, y, e0);
+    };
     const int qb = item % C::kQBufs, qu = item / C::kQBufs;
     mbar_wait(kFp8 ? &S.q_ready : &S.q_full[qb], qu & 1, abort);
     tc_fence_after();
@@ -437,7 +524,7 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       }
     };
 
-    auto issue_pv = [&](uint32_t tile, bool first) {
+    auto issue_pv = [&](uint32_t tile, bool first, int keep) {
       mbar_wait(&S.p_full, tile & 1, abort);
       if (first && item > 0) mbar_wait(&S.o_free, (item - 1) & 1, abort);
       tc_fence_after();
@@ -450,6 +537,15 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
           mbar_wait(&S.kv_full[s0], (c0 / kSlots) & 1, abort);
           mbar_wait(&S.kv_full[s1], ((c0 + 1) / kSlots) & 1, abort);
           tc_fence_after();
+          if (kPaged && keep < kTile && __shfl_sync(0xffffffffu, *abort, 0) == 0) {
+            // paged cache, the sequence's last window: V rows past its end may hold any
+            // bytes (NaN too) and meet a zero weight, so they are zeroed before PV (the
+            // whole warp runs this loop; the abort flag is read once for all its lanes)
+            zero_chunk_rows(ring_chunk(S, s0), keep, lane);
+            zero_chunk_rows(ring_chunk(S, s1), keep, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
           if (!*abort && leader) {
             const uint32_t d = tmem + kTmemO + 64 * h;
             const uint32_t a_base = smem_u32(ring_chunk(S, s0));
@@ -498,10 +594,10 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
 
     for (int t = 0; t < n; ++t) {
       issue_s(gt + t);
-      if (t >= 1) issue_pv(gt + t - 1, t - 1 == 0);
+      if (t >= 1) issue_pv(gt + t - 1, t - 1 == 0, rows_kept(t - 1));
     }
     if (!*abort && leader) umma_commit(&S.q_empty[qb]);
-    issue_pv(gt + n - 1, n == 1);
+    issue_pv(gt + n - 1, n == 1, rows_kept(n - 1));
     gt += n;
     ++item;
   });
@@ -550,7 +646,7 @@ __device__ void convert_k_tmem(TcSmem& S, uint32_t rbox, uint32_t tmem, uint32_t
 // thread first loads all eight of its 16-byte pieces (16 codes of one position each), then
 // the eight warps synchronize, and only then is any slot overwritten: a thread's output
 // covers other threads' input. One proxy fence covers the whole tile.
-__device__ void convert_v_inplace(TcSmem& S, uint32_t vbox, int st, int lane,
+__device__ void convert_v_inplace(TcSmem& S, uint32_t vbox, int st, int lane, int keep,
                                   volatile int* abort) {
   uint32_t slot[2];
 #pragma unroll
@@ -580,6 +676,7 @@ __device__ void convert_v_inplace(TcSmem& S, uint32_t vbox, int st, int lane,
         const int pc = st + 256 * i, r = pc >> 2, jj = pc & 3, sw = r & 7;
         uint4 o0, o1;
         e4m3x16_to_f16x16(v[bx][cc][i], o0, o1);
+        if (r >= keep) o0 = o1 = make_uint4(0u, 0u, 0u, 0u);  // paged: past the sequence
         *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj) ^ sw) << 4)) = o0;
         *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj + 1) ^ sw) << 4)) = o1;
       }
@@ -637,7 +734,7 @@ __device__ int convert_q(TcSmem& S, int item, int st, int swarp, int lane, volat
 // ---------------------------------------------------------------------------------------
 // warps 2..9: softmax, rescale, epilogue (and the FP8 conversions)
 // ---------------------------------------------------------------------------------------
-template <bool kFp8>
+template <bool kFp8, bool kPaged>
 __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
   volatile int* abort = &S.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -652,6 +749,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
   const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
   const float s_mul0 = a.scale * kLog2e * (kFp8 ? a.k_scale : 1.f);
   const float v_mul = kFp8 ? a.v_scale : 1.f;
+  constexpr bool paged = kPaged;
   uint32_t gt = 0;
   uint32_t kbox = 0, vbox = 0;  // FP8: raw K and V boxes converted so far
   int item = 0;
@@ -664,8 +762,8 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     // FP8: a V tile is two raw boxes -> converted in place in two V slots; a K tile is two
     // raw boxes -> tensor memory buffer (tile mod 2). Tensor memory buffer j was last read by
     // S(tile - 2), whose completion this warp has already waited for.
-    auto convert_v = [&]() {
-      convert_v_inplace(S, vbox, st, lane, abort);
+    auto convert_v = [&](int keep) {
+      convert_v_inplace(S, vbox, st, lane, keep, abort);
       vbox += 2;
     };
     auto convert_k = [&](uint32_t tile) {
@@ -681,13 +779,13 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     // read by PV(t - 2), so neither conversion waits for the tensor core's current work, and
     // PV(t) can issue as soon as P(t) is stored.
     for (int t = 0; t < n; ++t) {
+      int y, a0, e0;
+      tile_window(it, t, paged, y, a0, e0);
       if constexpr (kFp8) {
-        if (t + 1 < n) convert_k(gt + t + 1);  // consumed by S(t + 1)
-        convert_v();                           // V(t), consumed by PV(t)
+        if (t + 1 < n) convert_k(gt + t + 1);      // consumed by S(t + 1)
+        convert_v(window_rows_kept(paged, y, e0));  // V(t), consumed by PV(t)
       }
       const uint32_t tile = gt + t, j = tile & 1, k = tile >> 1;
-      int y, a0, e0;
-      tile_window(it, t, y, a0, e0);
       const int pos = y + row;
       const bool valid = pos >= a0 && pos < e0;
 
@@ -829,7 +927,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
   });
 }
 
-template <bool kFp8>
+template <bool kFp8, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap q_map, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -881,17 +979,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     plan_build(S.plan, a.seq_lens, a.kv, a.batch, a.grid, a.err, g == 0);
     if (g == 0) write_seq_info(S.plan, a.seq_info, a.batch);
   }
+  // This kernel was picked for the layout the caller stated; a table of the other layout
+  // gets no attention (an empty plan) and an error bit.
+  if (threadIdx.x == 0 && (S.plan.page_size != 0) != kPaged) {
+    S.plan.grid = 0;
+    atomicOr(a.err, kErrLayout);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
   if (warp == 0) {
-    run_producer<kFp8>(S, &q_map, a, g, lane == 0);
+    run_producer<kFp8, kPaged>(S, &q_map, a, g, lane == 0);
   } else if (warp == 1) {
-    run_mma<kFp8>(S, a, g, tmem, lane == 0);
+    run_mma<kFp8, kPaged>(S, a, g, tmem, lane == 0);
   } else {
-    run_softmax<kFp8>(S, a, g, tmem);
+    run_softmax<kFp8, kPaged>(S, a, g, tmem);
   }
 
   tc_fence_before();
@@ -1015,17 +1119,23 @@ cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s) {
 
 size_t attention_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
 
-template <bool kFp8>
+template <bool kFp8, bool kPaged>
 static cudaError_t launch_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s) {
   const size_t smem = attention_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<kFp8>,
+  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<kFp8, kPaged>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attention_tc_kernel<kFp8>, dim3(a.grid), dim3(kThreads), smem, s, q_map, a);
+  return launch_pdl(attention_tc_kernel<kFp8, kPaged>, dim3(a.grid), dim3(kThreads), smem, s,
+                    q_map, a);
 }
 
+// Contiguous and paged caches have kernels of their own (the caller's description picks
+// one): a paged window never slides, and page lookups would slow the contiguous loop.
 cudaError_t launch_attention_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s) {
-  return a.kv_dtype == MFA_KV_FP8_E4M3 ? launch_tc<true>(q_map, a, s) : launch_tc<false>(q_map, a, s);
+  const bool fp8 = a.kv_dtype == MFA_KV_FP8_E4M3;
+  if (a.page_size != 0)
+    return fp8 ? launch_tc<true, true>(q_map, a, s) : launch_tc<false, true>(q_map, a, s);
+  return fp8 ? launch_tc<true, false>(q_map, a, s) : launch_tc<false, false>(q_map, a, s);
 }
 
 }  // namespace mfa

@@ -24,6 +24,7 @@ struct PlanSmem {
   int32_t scan_tmp[33];
   int32_t grid;  // CTAs that get work: min(G, total tiles), so none of them is empty
   int32_t flag;
+  int32_t page_size;  // the KV table's layout: 0 contiguous, else rows per page
 };
 
 __device__ __forceinline__ int plan_bound(int g, int G, int NT) {
@@ -83,6 +84,7 @@ __device__ inline void plan_build(PlanSmem& P, const int32_t* __restrict__ seq_l
   for (int b = threadIdx.x; b < batch; b += blockDim.x) {
     const int L = seq_lens[b];
     const int cap = kv[b].capacity;
+    if (b == 0) P.page_size = kv[0].page_size;  // the same in every entry
     int len = L;
     if (L <= 0) {
       len = 0;
@@ -115,15 +117,18 @@ __device__ inline void plan_build(PlanSmem& P, const int32_t* __restrict__ seq_l
   block_exclusive_scan(P.slot_base, batch, P.scan_tmp);
 }
 
-// The plan in global memory: tile_start[batch + 1], slot_base[batch], len[batch], grid, at
-// fixed offsets of a kPlanBytes buffer.
+// The plan in global memory: tile_start[batch + 1], slot_base[batch], len[batch], grid,
+// page_size, at fixed offsets of a kPlanBytes buffer.
 __device__ inline void plan_store(const PlanSmem& P, int32_t* g, int batch) {
   for (int i = threadIdx.x; i <= batch; i += blockDim.x) g[i] = P.tile_start[i];
   for (int i = threadIdx.x; i < batch; i += blockDim.x) {
     g[kMaxBatch + 1 + i] = P.slot_base[i];
     g[2 * kMaxBatch + 1 + i] = P.len[i];
   }
-  if (threadIdx.x == 0) g[3 * kMaxBatch + 1] = P.grid;
+  if (threadIdx.x == 0) {
+    g[3 * kMaxBatch + 1] = P.grid;
+    g[3 * kMaxBatch + 2] = P.page_size;
+  }
 }
 
 __device__ inline void plan_load(PlanSmem& P, const int32_t* __restrict__ g, int batch) {
@@ -132,7 +137,10 @@ __device__ inline void plan_load(PlanSmem& P, const int32_t* __restrict__ g, int
     P.slot_base[i] = g[kMaxBatch + 1 + i];
     P.len[i] = g[2 * kMaxBatch + 1 + i];
   }
-  if (threadIdx.x == 0) P.grid = g[3 * kMaxBatch + 1];
+  if (threadIdx.x == 0) {
+    P.grid = g[3 * kMaxBatch + 1];
+    P.page_size = g[3 * kMaxBatch + 2];
+  }
 }
 
 // Per sequence: its first partial slot and the number of CTAs it is split over (0 for a

@@ -33,19 +33,32 @@ constexpr int kOProjKPerSplit = kQWidth / kOProjSplits;  // 8192
 constexpr int kTile = 128;
 
 // Device-side error bits kept in the workspace header.
-enum : uint32_t { kErrCapacity = 1u, kErrEmpty = 2u, kErrTimeout = 4u };
+enum : uint32_t { kErrCapacity = 1u, kErrEmpty = 2u, kErrTimeout = 4u, kErrLayout = 8u };
 
-// One entry of the device KV table: TMA tensor maps of the sequence's K and V rows
-// ([capacity, 256] elements, row-major) plus the raw pointers and capacity.
+// One entry of the device KV table. Contiguous caches: TMA tensor maps of the sequence's own
+// K and V rows ([capacity, 256] elements, row-major), their base pointers, page_size 0.
+// Paged caches: the maps cover the whole pools ([num_pages, page_size, 256]), k / v are the
+// pool bases, and row j of the sequence is row j % page_size of page pages[j / page_size];
+// capacity = (pages given to the sequence) * page_size. Every entry of one table has the
+// same layout.
 struct alignas(128) KvSeq {
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   void* k;
   void* v;
   int32_t capacity;
-  int32_t reserved[27];
+  int32_t page_size;      // 0: contiguous
+  const int32_t* pages;   // paged: this sequence's row of the page table (device)
+  int32_t num_pages;      // paged: pages in each pool
+  int32_t reserved[23];
 };
 static_assert(sizeof(KvSeq) == 384, "KvSeq layout");
+
+// Paged caches: rows per TMA box (a 128-position window is 128 / box rows boxes, each
+// inside one page).
+__host__ __device__ inline int paged_box_rows(int page_size) {
+  return page_size % 128 == 0 ? 128 : 64;
+}
 
 // Split-K partial of one attention work item: running max m (log2 domain) and sum l per
 // head, and the unnormalized accumulator acc[head][dim], all fp32.
@@ -53,8 +66,8 @@ constexpr int kPartialFloats = kHeads + kHeads + kHeads * kHeadDim;  // 16512
 constexpr size_t kPartialBytes = kPartialFloats * sizeof(float);     // 66048 = 258 * 256
 
 // Bytes of the attention split plan kept in the workspace (tile_start[kMaxBatch + 1],
-// slot_base[kMaxBatch], len[kMaxBatch], grid).
-constexpr size_t kPlanBytes = sizeof(int32_t) * (3 * kMaxBatch + 2);
+// slot_base[kMaxBatch], len[kMaxBatch], grid, page_size).
+constexpr size_t kPlanBytes = sizeof(int32_t) * (3 * kMaxBatch + 3);
 
 struct WsLayout {
   size_t err;          // uint32 error bits
@@ -187,6 +200,7 @@ struct AttnArgs {
                             // stream, so it may be read before griddepcontrol.wait
   uint32_t* err;
   int grid;
+  int page_size;            // the caller's mfa_kv_cache.page_size: picks the kernel
 };
 // Tensor-core attention (bf16 or FP8 KV); q_map covers q as [batch * 64 rows, 256] bf16,
 // boxes of [64 x 64] with 128-byte swizzle.
@@ -213,5 +227,9 @@ EncodeTiledFn encode_tiled_fn();
 // 128-byte swizzle. Returns false if the driver rejects it.
 bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int elem_bytes,
                uint32_t box_cols, uint32_t box_rows);
+// 3-D map over a page pool [pages, page_rows, 256] (elem_bytes each), box
+// [128 bytes of a row x box_rows x 1 page], 128-byte swizzle.
+bool encode_pool(CUtensorMap* m, const void* base, uint64_t pages, uint64_t page_rows,
+                 int elem_bytes, uint32_t box_rows);
 
 }  // namespace mfa

@@ -95,14 +95,25 @@ __global__ void __launch_bounds__(kFinishThreads) xproj_finish_kernel(FinishArgs
     if (tid == 0) atomicOr(a.err, kErrCapacity);
     return;
   }
+  // the row's index in the buffer: the sequence's own rows, or for a paged cache row
+  // row % page_size of page pages[row / page_size] of the pool
+  size_t at = (size_t)row;
+  if (s->page_size != 0) {
+    const int page = s->pages[row / s->page_size];
+    if (page < 0 || page >= s->num_pages) {
+      if (tid == 0) atomicOr(a.err, kErrCapacity);
+      return;
+    }
+    at = (size_t)page * s->page_size + row % s->page_size;
+  }
   const bool is_v = tid >= kHeadDim;
   const int j = is_v ? tid - kHeadDim : tid;
   void* base = is_v ? s->v : s->k;
   if (a.kv_dtype == MFA_KV_BF16) {
-    static_cast<uint16_t*>(base)[(size_t)row * kHeadDim + j] = f32_to_bf16_bits(ck);
+    static_cast<uint16_t*>(base)[at * kHeadDim + j] = f32_to_bf16_bits(ck);
   } else {
     const float scale = is_v ? a.v_scale : a.k_scale;
-    static_cast<uint8_t*>(base)[(size_t)row * kHeadDim + j] = f32_to_e4m3(__fdiv_rn(ck, scale));
+    static_cast<uint8_t*>(base)[at * kHeadDim + j] = f32_to_e4m3(__fdiv_rn(ck, scale));
   }
 }
 

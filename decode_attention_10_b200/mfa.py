@@ -30,6 +30,9 @@ _SIGNATURES = {
     "mfa_kv_table_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
     "mfa_kv_table_init": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int32,
                                          _P, _P, _P, _P]),
+    "mfa_kv_table_init_paged": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_int32,
+                                               ctypes.c_int32, _P, _P, ctypes.c_int32,
+                                               ctypes.c_int32, _P, ctypes.c_int32, _P, _P]),
     "mfa_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int32]),
     "mfa_workspace_init": (ctypes.c_int, [_P, ctypes.c_size_t, _P]),
     "mfa_get_error": (ctypes.c_int, [_P, _P]),
@@ -52,7 +55,7 @@ class KvCacheDesc(ctypes.Structure):
     """mfa_kv_cache."""
     _fields_ = [("batch", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
-                ("table", ctypes.c_void_p)]
+                ("table", ctypes.c_void_p), ("page_size", ctypes.c_int32)]
 
 
 class MfaError(RuntimeError):
@@ -147,7 +150,52 @@ class KVCache:
                                      ctypes.cast(cp, _P), _stream(stream)),
                "mfa_kv_table_init")
         self.desc = KvCacheDesc(self.batch, self.dtype, self.k_scale, self.v_scale,
-                                self.table.data_ptr())
+                                self.table.data_ptr(), 0)
+
+
+class PagedKVCache:
+    """A paged KV cache described to the library: K and V page pools ([num_pages, page_size,
+    256] CUDA tensors of bf16 or float8_e4m3fn; page_size a power of two >= 64), a CUDA int32 page
+    table [batch, max_pages] whose row b lists sequence b's pages in order, and the number of
+    pages given to each sequence. The kernels read the page table on every call, so its
+    contents may change between calls (a growing sequence's next page) without a new
+    description; the pools and the table must stay in place."""
+
+    def __init__(self, k_pool: torch.Tensor, v_pool: torch.Tensor, page_table: torch.Tensor,
+                 pages_per_seq: Sequence[int], k_scale: float = 1.0, v_scale: float = 1.0,
+                 stream: Optional[torch.cuda.Stream] = None):
+        lib = load()
+        if k_pool.dim() != 3 or k_pool.shape[2] != HEAD_DIM or k_pool.shape != v_pool.shape:
+            raise ValueError("K and V pools must both be [num_pages, page_size, 256]")
+        self.dtype = _dtype_code(k_pool)
+        if _dtype_code(v_pool) != self.dtype:
+            raise ValueError("mixed KV dtypes")
+        if (page_table.dtype != torch.int32 or page_table.dim() != 2 or not page_table.is_cuda
+                or not page_table.is_contiguous()):
+            raise ValueError("page_table must be a contiguous CUDA int32 [batch, max_pages]")
+        self.batch, max_pages = int(page_table.shape[0]), int(page_table.shape[1])
+        pps = [int(n) for n in pages_per_seq]
+        if len(pps) != self.batch:
+            raise ValueError("one page count per sequence")
+        _ptr(k_pool), _ptr(v_pool)
+        self.k_pool, self.v_pool, self.page_table = k_pool, v_pool, page_table
+        self.num_pages, self.page_size = int(k_pool.shape[0]), int(k_pool.shape[1])
+        self.pages_per_seq = pps
+        self.capacity = [n * self.page_size for n in pps]
+        self.k_scale, self.v_scale = float(k_scale), float(v_scale)
+        nbytes = lib.mfa_kv_table_bytes(self.batch)
+        if nbytes == 0:
+            raise ValueError(f"batch {self.batch} out of range")
+        self.table = torch.empty(nbytes, dtype=torch.uint8, device=k_pool.device)
+        cp = (ctypes.c_int32 * self.batch)(*pps)
+        _check(lib.mfa_kv_table_init_paged(self.table.data_ptr(), nbytes, self.batch,
+                                           self.dtype, k_pool.data_ptr(), v_pool.data_ptr(),
+                                           self.num_pages, self.page_size,
+                                           page_table.data_ptr(), max_pages,
+                                           ctypes.cast(cp, _P), _stream(stream)),
+               "mfa_kv_table_init_paged")
+        self.desc = KvCacheDesc(self.batch, self.dtype, self.k_scale, self.v_scale,
+                                self.table.data_ptr(), self.page_size)
 
 
 class Workspace:

@@ -214,6 +214,41 @@ def generate_layer_on_device(seq_lens: Sequence[int], kv_dtype: str, seed: int, 
     return d
 
 
+def to_paged(k_cache: Sequence[torch.Tensor], v_cache: Sequence[torch.Tensor], page_size: int,
+             seed: int, spare_pages: int = 0, shuffle: bool = True):
+    """The per-sequence caches ([capacity_b, 256] tensors, on any device) copied into K and V
+    page pools [num_pages, page_size, 256] at shuffled pool positions (a serving engine's
+    page allocator hands pages out in no particular order). Rows of a sequence's last page
+    past its capacity are zero; ``shuffle=False`` lays the pages out in sequence order
+    instead. Returns (k_pool, v_pool, page_table int32 [B, max_pages] on
+    the caches' device, pages per sequence)."""
+    caps = [int(t.shape[0]) for t in k_cache]
+    need = [-(-c // page_size) for c in caps]
+    total = sum(need) + int(spare_pages)
+    g = torch.Generator().manual_seed(int(seed))
+    order = torch.randperm(total, generator=g) if shuffle else torch.arange(total)
+    table = torch.zeros(len(caps), max(need), dtype=torch.int32)
+    at = 0
+    for b, n in enumerate(need):
+        table[b, :n] = order[at:at + n].to(torch.int32)
+        at += n
+    dev = k_cache[0].device
+    pools = []
+    for cache in (k_cache, v_cache):
+        pool = torch.zeros(total, page_size, HEAD_DIM, dtype=cache[0].dtype, device=dev)
+        flat = pool.view(-1) if cache[0].element_size() == 2 else pool.view(torch.uint8).view(-1)
+        for b, t in enumerate(cache):
+            rows = t.reshape(-1) if t.element_size() == 2 else t.view(torch.uint8).reshape(-1)
+            # page p of sequence b: rows [p * page_size, (p + 1) * page_size) of its cache
+            for p in range(need[b]):
+                lo = p * page_size * HEAD_DIM
+                hi = min(caps[b] * HEAD_DIM, lo + page_size * HEAD_DIM)
+                base = int(table[b, p]) * page_size * HEAD_DIM
+                flat[base:base + hi - lo].copy_(rows[lo:hi])
+        pools.append(pool)
+    return pools[0], pools[1], table.to(dev), need
+
+
 def ragged_lengths(batch: int, seed: int) -> list:
     """Per-sequence lengths drawn uniform in [1, 65536] -- the first draw of the seed."""
     g = torch.Generator().manual_seed(int(seed))

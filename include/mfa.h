@@ -84,6 +84,10 @@ typedef struct {
   float k_scale;       /* FP8 only: K rows hold e4m3(k / k_scale); must be > 0 */
   float v_scale;       /* FP8 only: V rows hold e4m3(v / v_scale); must be > 0 */
   const void* table;   /* device */
+  int32_t page_size;   /* 0 for a table of mfa_kv_table_init, the page size for one of
+                          mfa_kv_table_init_paged (it picks the kernel; a value the table
+                          contradicts computes no attention and sets MFA_ERR_INVALID_ARG in
+                          the workspace) */
 } mfa_kv_cache;
 
 /* ---------------------------------------------------------------------------------------
@@ -113,6 +117,30 @@ MFA_API mfa_status mfa_kv_table_init(void* table, size_t table_bytes, int32_t ba
                              void* const* k_ptrs, void* const* v_ptrs,
                              const int32_t* capacity, void* stream);
 
+/* Describe a paged KV cache, the block-table layout of serving engines (step3-fp8 model
+ * page, "Deployment": inference with vLLM and SGLang, which both keep the KV cache in
+ * fixed-size pages listed per sequence in a page table). k_pool and v_pool
+ * are DEVICE buffers [num_pages, page_size, 256] of `dtype`, 16-byte aligned; row j of
+ * sequence b is row j % page_size of page page_table[b * max_pages + j / page_size].
+ * page_table: DEVICE int32 [batch, max_pages] (4-byte aligned), read by the kernels (not
+ * copied): its contents may change between calls, e.g. when a sequence gets a new page.
+ * pages_per_seq: HOST int32 [batch], the pages given to each sequence (1..max_pages); the
+ * sequence's capacity is pages_per_seq[b] * page_size <= MFA_MAX_CONTEXT.
+ * page_size: a power of two, at least 64 (64-row pages take two TMA operations per
+ * 128-position window, larger pages one).
+ * Rows of a sequence's pages past its length may hold any bytes, NaN included: attention
+ * never weights them, and the values it loads for them are zeroed on chip before the
+ * tensor core multiplies by a zero weight. An append whose page id is outside
+ * [0, num_pages) writes nothing and sets MFA_ERR_CAPACITY; the attention reads such pages
+ * as zeros. `table` as in mfa_kv_table_init; the call waits for its copy. Errors:
+ * INVALID_ARG, UNSUPPORTED (dtype, or page_size not a power of two >= 64), WORKSPACE
+ * (table too small), CUDA. */
+MFA_API mfa_status mfa_kv_table_init_paged(void* table, size_t table_bytes, int32_t batch,
+                                           int32_t dtype, void* k_pool, void* v_pool,
+                                           int32_t num_pages, int32_t page_size,
+                                           const int32_t* page_table, int32_t max_pages,
+                                           const int32_t* pages_per_seq, void* stream);
+
 /* Bytes of the workspace the compute calls need for `batch` sequences on the current
  * device (0 if batch is out of range). One workspace must not be used by two calls that
  * can run at the same time. */
@@ -123,8 +151,9 @@ MFA_API size_t mfa_workspace_bytes(int32_t batch);
 MFA_API mfa_status mfa_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Wait for `stream`, then report and clear the device-side error flags of `ws`:
- * MFA_OK, MFA_ERR_CAPACITY, MFA_ERR_EMPTY or MFA_ERR_TIMEOUT (the first set, in that
- * order), or MFA_ERR_CUDA if the stream reports an error. */
+ * MFA_OK, MFA_ERR_CAPACITY, MFA_ERR_EMPTY, MFA_ERR_INVALID_ARG (an mfa_kv_cache whose
+ * page_size the table contradicts) or MFA_ERR_TIMEOUT (the first set, in that order), or
+ * MFA_ERR_CUDA if the stream reports an error. */
 MFA_API mfa_status mfa_get_error(void* ws, void* stream);
 
 /* ---------------------------------------------------------------------------------------

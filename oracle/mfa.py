@@ -134,6 +134,20 @@ def kv_load(codes, kv_dtype, scale=1.0):
     raise ValueError(f"unknown kv dtype {kv_dtype!r}")
 
 
+def kv_gather_paged(pool, page_ids, n_rows, page_size):
+    """Rows [0, n_rows) of one sequence of a paged cache: row j is row j % page_size of page
+    page_ids[j // page_size] of ``pool`` [num_pages, page_size, d] (the page-table layout of
+    the serving engines the step3-fp8 model page deploys with, vLLM and SGLang). Returns the
+    codes [n_rows, d].
+
+    Pinned by: a contiguous cache cut into pages placed at shuffled pool slots gathers back
+    to itself; rows past n_rows and pages outside the list are never read."""
+    rows = [pool[int(page_ids[j // page_size])][j % page_size] for j in range(int(n_rows))]
+    if not rows:
+        return np.zeros((0,) + tuple(np.shape(pool)[2:]), dtype=np.asarray(pool).dtype)
+    return np.stack(rows)
+
+
 def kv_append(k_cache, v_cache, pos, k_codes, v_codes):
     """Write the new token's K/V codes at row ``pos[b]`` of sequence b's cache.
 

@@ -89,6 +89,10 @@ def test_invalid_arguments_are_rejected_before_any_device_work(lib):
     kv = mfa.KvCacheDesc(4, 1, 0.0, 1.0, 4096)  # FP8 needs positive scales
     assert lib.mfa_decode_attn(fake, ctypes.byref(kv), fake, 0.0625, fake, fake, 1 << 30,
                                None) == 1
+    for ps in (32, 100, 192):  # a stated page size must be 0 or a power of two >= 64
+        kv = mfa.KvCacheDesc(4, 0, 1.0, 1.0, 4096, ps)
+        assert lib.mfa_decode_attn(fake, ctypes.byref(kv), fake, 0.0625, fake, fake, 1 << 30,
+                                   None) == 1
     kv = mfa.KvCacheDesc(4, 0, 1.0, 1.0, 4096 + 64)  # table must be 128-byte aligned
     assert lib.mfa_kv_append(fake, fake, fake, ctypes.byref(kv), fake, fake, 1 << 30,
                              None) == 1
@@ -101,6 +105,16 @@ def test_invalid_arguments_are_rejected_before_any_device_work(lib):
     assert lib.mfa_o_proj(fake, fake, fake, 1025, fake, 1 << 30, None) == 1
     assert lib.mfa_o_proj(None, fake, fake, 4, fake, 1 << 30, None) == 1
     assert lib.mfa_o_proj(fake, fake, P(4104), 4, fake, 1 << 30, None) == 1
+    # paged table init: page sizes that are not a power of two >= 64, bad page counts
+    pages = (ctypes.c_int32 * 2)(1, 1)
+    for ps in (0, 32, 96, 192):
+        assert lib.mfa_kv_table_init_paged(P(4096), 1 << 20, 2, 0, fake, fake, 8, ps, fake, 4,
+                                           pages, None) == 2
+    bad_pages = (ctypes.c_int32 * 2)(1, 5)  # more than max_pages
+    assert lib.mfa_kv_table_init_paged(P(4096), 1 << 20, 2, 0, fake, fake, 8, 128, fake, 4,
+                                       bad_pages, None) == 1
+    assert lib.mfa_kv_table_init_paged(P(4096), 1 << 20, 2, 0, None, fake, 8, 128, fake, 4,
+                                       pages, None) == 1
     # table init: bad batch, null arrays, unknown dtype, table too small, capacity range
     arr = (ctypes.c_void_p * 2)(4096, 8192)
     caps = (ctypes.c_int32 * 2)(16, 16)

@@ -33,3 +33,22 @@ def test_attention_bytes_are_the_algorithmic_count():
     assert bench.attention_bytes(inp) == 2 * 512 * 400 + 2 * 2 * 64 * 256 * 2
     inp8 = W.generate([100, 300], W.KV_FP8, seed=1)
     assert bench.kv_bytes(inp8) == 2 * 256 * 400
+
+
+def test_paged_layout_holds_every_sequence_row_in_its_listed_pages():
+    import torch
+
+    from decode_attention_10_b200 import workloads as W
+    for dtype, page in (("bf16", 128), ("fp8_e4m3", 64), ("bf16", 192)):
+        inp = W.generate([5, 130, 300], dtype, seed=1, capacity=[64, 200, 300])
+        kp, vp, pt, need = W.to_paged(inp.k_cache, inp.v_cache, page, seed=3, spare_pages=2)
+        assert kp.shape == (sum(need) + 2, page, 256) and kp.dtype == inp.k_cache[0].dtype
+        assert need == [-(-c // page) for c in (64, 200, 300)]
+        used = pt[0, :need[0]].tolist() + pt[1, :need[1]].tolist() + pt[2, :need[2]].tolist()
+        assert len(set(used)) == len(used)  # no page shared
+        for pool, cache in ((kp, inp.k_cache), (vp, inp.v_cache)):
+            for b, t in enumerate(cache):
+                raw = pool.view(torch.uint8) if t.element_size() == 1 else pool.view(torch.int16)
+                rows = torch.cat([raw[int(pt[b, p])] for p in range(need[b])])[:t.shape[0]]
+                want = t.view(torch.uint8) if t.element_size() == 1 else t.view(torch.int16)
+                assert torch.equal(rows, want)

@@ -420,3 +420,34 @@ def test_planted_o_proj_skipped_in_the_chain_is_caught():
     res, _ = mfa.attention_side_step(x, layers, lens, scale=0.5, n_heads=heads, emulate=False)
     wrong = res[0]["out"].reshape(len(lens), -1)  # heads * hd == dim: shapes would fit
     assert not np.allclose(wrong, res[0]["y"], rtol=1e-3, atol=1e-6)
+
+
+# ----------------------------------------------------------------------------------------
+# paged caches: the page-table layout
+# ----------------------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("page_size,lens", [(4, [1, 4, 9, 13]), (8, [7, 8, 17])])
+def test_kv_gather_paged_reassembles_a_shuffled_cache(page_size, lens):
+    rng = np.random.default_rng(page_size)
+    d = 3
+    seqs = [rng.integers(0, 1 << 16, (n, d)).astype(np.uint16) for n in lens]
+    need = [-(-n // page_size) for n in lens]
+    total = sum(need) + 3  # spare pages that no sequence uses
+    order = rng.permutation(total)
+    pool = np.full((total, page_size, d), 0xFFFF, dtype=np.uint16)  # poison everywhere
+    tables, at = [], 0
+    for s, n_pages in zip(seqs, need):
+        ids = order[at:at + n_pages]
+        at += n_pages
+        for p, pid in enumerate(ids):
+            chunk = s[p * page_size:(p + 1) * page_size]
+            pool[pid][:len(chunk)] = chunk
+        tables.append(ids)
+    for s, ids, n in zip(seqs, tables, lens):
+        assert np.array_equal(mfa.kv_gather_paged(pool, ids, n, page_size), s)
+    # the page list alone decides where rows come from
+    swapped = tables[2][::-1]
+    if len(swapped) > 1:
+        assert not np.array_equal(mfa.kv_gather_paged(pool, swapped, lens[2], page_size),
+                                  seqs[2])

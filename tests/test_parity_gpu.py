@@ -427,3 +427,148 @@ def test_attention_side_two_layers(kv_dtype):
     # end to end through both layers: two layers' worth of the per-layer tolerance
     _, y_ref = omfa.attention_side_step(oracle_weights(inps[0])["x"], layers, lens, od)
     assert rel_l2(bf16_np(ys[-1]), y_ref) <= 2 * 5e-3
+
+
+# ----------------------------------------------------------------------------------------
+# paged KV caches (page tables, shuffled pages, unused rows poisoned with NaN)
+# ----------------------------------------------------------------------------------------
+
+
+def _paged_from(inp: W.Inputs, page_size: int, seed: int, spare: int = 5):
+    """The caches of ``inp`` copied into shuffled pages of K and V pools. Rows past each
+    sequence's length, and unused pages, hold NaN codes. Returns (PagedKVCache, k_pool,
+    v_pool, page_table (host numpy), pages per sequence)."""
+    from decode_attention_10_b200 import mfa
+    rng = np.random.default_rng(seed)
+    lens = inp.seq_lens.tolist()
+    caps = inp.meta["capacity"]
+    need = [-(-c // page_size) for c in caps]
+    total = sum(need) + spare
+    order = rng.permutation(total)
+    fp8 = inp.kv_dtype == W.KV_FP8
+    nan_code = 0x7F if fp8 else 0x7FC0
+    np_dtype = np.uint8 if fp8 else np.uint16
+    pools = []
+    table = np.zeros((len(lens), max(need)), dtype=np.int32)
+    at = 0
+    for b, n_pages in enumerate(need):
+        table[b, :n_pages] = order[at:at + n_pages]
+        at += n_pages
+    for cache in (inp.k_cache, inp.v_cache):
+        pool = np.full((total, page_size, 256), nan_code, dtype=np_dtype)
+        for b, n in enumerate(lens):
+            rows = codes_np(cache[b])[:n]
+            for p in range(need[b]):
+                chunk = rows[p * page_size:(p + 1) * page_size]
+                pool[table[b, p], :len(chunk)] = chunk
+        t = torch.from_numpy(pool.view(np.int8 if fp8 else np.int16))
+        t = t.view(torch.float8_e4m3fn if fp8 else torch.bfloat16)
+        pools.append(t.cuda())
+    pt = torch.from_numpy(table).cuda()
+    cache = mfa.PagedKVCache(pools[0], pools[1], pt, need, inp.k_scale, inp.v_scale)
+    return cache, pools[0], pools[1], table, need
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+@pytest.mark.parametrize("page_size", [64, 128, 256, 512])
+def test_paged_attention_matches_oracle(kv_dtype, page_size):
+    from decode_attention_10_b200 import mfa
+    lens = [1, 130, 300, 129, 128, 2, 777, 64]
+    inp = W.generate(lens, kv_dtype, seed=80 + page_size)
+    cache, k_pool, v_pool, table, need = _paged_from(inp, page_size, seed=page_size)
+    g = torch.Generator().manual_seed(81)
+    q = torch.randn(len(lens), 64, 256, generator=g).to(torch.bfloat16).cuda()
+    seq_lens = inp.seq_lens.cuda()
+    ws = mfa.Workspace(len(lens))
+    out = mfa.decode_attn(q, cache, seq_lens, ws=ws)
+    torch.cuda.synchronize()
+    assert mfa.get_error(ws) == 0
+    od = oracle_dtype(kv_dtype)
+    kp, vp = codes_np(k_pool), codes_np(v_pool)
+    k_rows = [omfa.kv_gather_paged(kp, table[b], n, page_size) for b, n in enumerate(lens)]
+    v_rows = [omfa.kv_gather_paged(vp, table[b], n, page_size) for b, n in enumerate(lens)]
+    for b, n in enumerate(lens):  # the layout itself: the pages hold the original rows
+        assert np.array_equal(k_rows[b], codes_np(inp.k_cache[b])[:n])
+    ref = omfa.decode_attn(bf16_np(q), k_rows, v_rows, lens, od, inp.k_scale, inp.v_scale)
+    out_np = bf16_np(out)
+    assert np.isfinite(out_np).all()
+    assert_close(out_np, ref, kv_dtype, f"paged attention, page size {page_size}")
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_paged_layer_appends_into_the_right_page(kv_dtype):
+    from decode_attention_10_b200 import mfa
+    page_size = 128
+    # lengths whose appended row opens a fresh page (129, 257), ends one (128), or sits
+    # inside one
+    lens = [129, 128, 257, 5, 400]
+    inp = W.generate(lens, kv_dtype, seed=90, capacity=[c + 60 for c in lens])
+    cache, k_pool, v_pool, table, need = _paged_from(inp, page_size, seed=91)
+    k_before, v_before = codes_np(k_pool).copy(), codes_np(v_pool).copy()
+    step = GpuStep(inp)
+    q, out = mfa.decode_layer(step.x, step.w_qdown, step.gamma, step.w_qup, step.w_k, step.w_v,
+                              cache, step.seq_lens, ws=step.ws)
+    torch.cuda.synchronize()
+    assert mfa.get_error(step.ws) == 0
+    od = oracle_dtype(kv_dtype)
+    ow = oracle_weights(inp)
+    k_new, v_new = omfa.kv_project(ow["x"], ow["w_k"], ow["w_v"])
+    k_codes = omfa.kv_store(k_new, od, inp.k_scale)
+    v_codes = omfa.kv_store(v_new, od, inp.v_scale)
+    kp, vp = codes_np(k_pool), codes_np(v_pool)
+    for pool, before, want in ((kp, k_before, k_codes), (vp, v_before, v_codes)):
+        changed = np.zeros(pool.shape[:2], bool)
+        for b, n in enumerate(lens):
+            page, r = table[b, (n - 1) // page_size], (n - 1) % page_size
+            changed[page, r] = True
+            diff = np.abs(pool[page, r].astype(np.int64) - want[b].astype(np.int64))
+            assert diff.max() <= 1, f"seq {b}: appended row differs by {diff.max()} codes"
+        assert np.array_equal(pool[~changed], before[~changed]), "other rows changed"
+    k_rows = [omfa.kv_gather_paged(kp, table[b], n, page_size) for b, n in enumerate(lens)]
+    v_rows = [omfa.kv_gather_paged(vp, table[b], n, page_size) for b, n in enumerate(lens)]
+    ref = omfa.decode_attn(bf16_np(q), k_rows, v_rows, lens, od, inp.k_scale, inp.v_scale)
+    assert_close(bf16_np(out), ref, kv_dtype, "paged layer (per op)")
+
+
+def test_paged_append_to_a_page_outside_the_pool_is_rejected():
+    from decode_attention_10_b200 import mfa
+    lens = [129, 40]
+    inp = W.generate(lens, W.KV_BF16, seed=95)
+    cache, k_pool, v_pool, table, need = _paged_from(inp, 128, seed=96, spare=0)
+    # sequence 0 appends at row 128: its second page id now points past the pool
+    bad = torch.from_numpy(table).clone()
+    bad[0, 1] = k_pool.shape[0] + 7
+    cache.page_table.copy_(bad.cuda())
+    k_before = codes_np(k_pool).copy()
+    step = GpuStep(inp)
+    _, out = mfa.decode_layer(step.x, step.w_qdown, step.gamma, step.w_qup, step.w_k, step.w_v,
+                              cache, step.seq_lens, ws=step.ws)
+    torch.cuda.synchronize()
+    assert mfa.get_error(step.ws) == 3  # MFA_ERR_CAPACITY
+    kp = codes_np(k_pool)
+    assert np.array_equal(kp[:, :, :][np.arange(kp.shape[0]) != table[1, 0]],
+                          k_before[np.arange(kp.shape[0]) != table[1, 0]])
+    assert np.isfinite(bf16_np(out)).all()  # the missing page reads as zeros
+
+
+def test_cache_description_contradicting_its_table_is_reported():
+    # a paged table described as contiguous (and the reverse) computes no attention, loads
+    # nothing through the wrong kind of tensor map, and reports MFA_ERR_INVALID_ARG
+    from decode_attention_10_b200 import mfa
+    lens = [130, 7]
+    inp = W.generate(lens, W.KV_BF16, seed=97)
+    paged, *_ = _paged_from(inp, 128, seed=98)
+    q = torch.randn(len(lens), 64, 256).to(torch.bfloat16).cuda()
+    seq_lens = inp.seq_lens.cuda()
+    ws = mfa.Workspace(len(lens))
+    paged.desc.page_size = 0
+    mfa.decode_attn(q, paged, seq_lens, ws=ws)
+    assert mfa.get_error(ws) == 1
+    step = GpuStep(inp)
+    step.cache.desc.page_size = 128
+    mfa.decode_attn(q, step.cache, seq_lens, ws=ws)
+    assert mfa.get_error(ws) == 1
+    step.cache.desc.page_size = 0  # described right again: the same context computes
+    out = mfa.decode_attn(q, step.cache, seq_lens, ws=ws)
+    assert mfa.get_error(ws) == 0
+    assert np.isfinite(bf16_np(out)).all()
