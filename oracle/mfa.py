@@ -285,3 +285,84 @@ def attention_side_step(x, layers, seq_lens, kv_dtype=KV_BF16, eps=RMS_EPS,
         results.append(r)
         h = y
     return results, h
+
+
+# ----------------------------------------------------------------------------------------
+# FP8 projections: block-FP8 weights (the step3-fp8 model page: checkpoints in bf16 and
+# block-fp8) and FP8 activations (the Step-3 pages: the whole model runs in FP8, bud-325
+# "Key claims")
+# ----------------------------------------------------------------------------------------
+
+W8_BLOCK = 128  # reading: one float32 scale per 128 x 128 block of a weight
+A8_GROUP = 128  # reading: one float32 scale per 128 consecutive values of an activation row
+
+
+def w8_dequantize(codes, scales, block=W8_BLOCK):
+    """A block-FP8 weight as real values: ``codes`` [out, in] uint8 are e4m3 codes in the
+    checkpoints' [out, in] order, ``scales`` [ceil(out / block), ceil(in / block)] float32;
+    weight[o, i] = code[o, i] * scale[o // block, i // block], exactly. Returns float64
+    [in, out] (the [in, out] order of the other projections). The page names the format
+    without a block size; 128 x 128 is the reading taken.
+
+    Pinned by: power-of-two scales placed per block and ragged edge blocks, against
+    code * scale element by element."""
+    c = codecs.e4m3_decode(np.asarray(codes))
+    s = np.asarray(scales, np.float64)
+    s_full = np.repeat(np.repeat(s, block, axis=0), block, axis=1)[:c.shape[0], :c.shape[1]]
+    return (c * s_full).T
+
+
+def a8_quantize(a, group=A8_GROUP):
+    """An activation [rows, n] (bf16 values) in FP8: per row and group of ``group``
+    consecutive values, scale = max |a| / 448 (1 for an all-zero group) and code =
+    e4m3(a / scale), round to nearest even, saturating. The scale and the quotient are
+    float32 operations (round to nearest even), so both sides of a comparison decide each
+    code in the same precision. Returns (codes uint8 [rows, n], scales float32
+    [rows, ceil(n / group)]).
+
+    Pinned by: a group whose max is a power of two times 448 (exact scale and codes), the
+    max element always coding to +-448, zero groups, and brute force on small rows."""
+    a = np.asarray(a, np.float64)
+    rows, n = a.shape
+    ng = -(-n // group)
+    codes = np.zeros((rows, n), np.uint8)
+    scales = np.ones((rows, ng), np.float32)
+    for g in range(ng):
+        blk = a[:, g * group:(g + 1) * group].astype(np.float32)
+        amax = np.abs(blk).max(axis=1)
+        sc = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+        q = (blk / sc[:, None]).astype(np.float32)
+        codes[:, g * group:(g + 1) * group] = codecs.e4m3_encode(q.astype(np.float64))
+        scales[:, g] = sc
+    return codes, scales
+
+
+def a8_dequantize(codes, scales, group=A8_GROUP):
+    """codes [rows, n] and scales [rows, ceil(n / group)] -> float64 values, exactly."""
+    c = codecs.e4m3_decode(np.asarray(codes))
+    s = np.repeat(np.asarray(scales, np.float64), group, axis=1)[:, :c.shape[1]]
+    return c * s
+
+
+def fp8_project(a, w_codes, w_scales):
+    """A projection on the FP8 path: the activation rows quantized by ``a8_quantize``, the
+    weight block-FP8; the products of the real values, summed in float64. Returns [rows,
+    out]."""
+    ac, asc = a8_quantize(a)
+    return a8_dequantize(ac, asc) @ w8_dequantize(w_codes, w_scales)
+
+
+def query_proj_fp8(x, wq_codes, wq_scales, gamma, wu_codes, wu_scales, eps=RMS_EPS,
+                   n_heads=N_HEADS, emulate=True):
+    """The query path on the FP8 path: c = fp8_project(x, W_qdown), RMSNorm as ever, then
+    q = fp8_project(c_hat, W_qup) (c_hat rounded to bf16 first with ``emulate``, as stored).
+    Returns (c_hat, q)."""
+    c_hat = rms_norm(fp8_project(x, wq_codes, wq_scales), gamma, eps)
+    if emulate:
+        c_hat = codecs.bf16_round(c_hat)
+    q = fp8_project(c_hat, wu_codes, wu_scales)
+    b, n = q.shape
+    q = q.reshape(b, n_heads, n // n_heads)
+    if emulate:
+        q = codecs.bf16_round(q)
+    return c_hat, q

@@ -451,3 +451,78 @@ def test_kv_gather_paged_reassembles_a_shuffled_cache(page_size, lens):
     if len(swapped) > 1:
         assert not np.array_equal(mfa.kv_gather_paged(pool, swapped, lens[2], page_size),
                                   seqs[2])
+
+
+# ----------------------------------------------------------------------------------------
+# block-FP8 weights
+# ----------------------------------------------------------------------------------------
+
+
+def test_w8_dequantize_places_each_block_scale():
+    # power-of-two scales make every product exact: the result must be code * scale of the
+    # element's own block, transposed to [in, out]
+    rng = np.random.default_rng(3)
+    out_dim, in_dim, blk = 10, 7, 4  # ragged last blocks in both directions
+    codes = rng.integers(0, 256, (out_dim, in_dim)).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x11  # no NaN codes
+    scales = np.ldexp(1.0, rng.integers(-6, 6, (3, 2))).astype(np.float32)
+    w = mfa.w8_dequantize(codes, scales, block=blk)
+    assert w.shape == (in_dim, out_dim)
+    for o in range(out_dim):
+        for i in range(in_dim):
+            want = codecs.e4m3_decode(codes[o, i]) * float(scales[o // blk, i // blk])
+            assert w[i, o] == want
+
+
+def test_a8_quantize_exact_cases():
+    # max 448 * 2**-3 -> scale 2**-3 exactly; every value a multiple of the e4m3 grid
+    a = np.zeros((2, 256))
+    a[0, :128] = np.linspace(-56, 56, 128)
+    a[0, 5] = 56.0  # the max
+    a[1, 128:] = 0.0  # an all-zero group
+    a[1, :128] = 3.0
+    codes, scales = mfa.a8_quantize(a)
+    assert scales.dtype == np.float32 and scales.shape == (2, 2)
+    assert scales[0, 0] == np.float32(56.0 / 448.0) == 0.125
+    assert scales[1, 1] == 1.0 and (codes[1, 128:] == 0).all()
+    assert codecs.e4m3_decode(codes[0, 5]) == 448.0  # the max codes to 448
+    assert codecs.e4m3_decode(codes[1, 0]) == 448.0  # 3 / (3 / 448)
+    back = mfa.a8_dequantize(codes, scales)
+    assert np.allclose(back[0, :128], a[0, :128], rtol=2 ** -4, atol=0)
+    assert back[0, 5] == 56.0
+
+
+def test_a8_quantize_brute_force():
+    rng = np.random.default_rng(8)
+    a = codecs.bf16_round(rng.standard_normal((3, 300)) * rng.uniform(0.01, 10, (3, 1)))
+    codes, scales = mfa.a8_quantize(a)
+    for r in range(3):
+        for g in range(3):
+            blk = a[r, 128 * g:128 * (g + 1)]
+            amax = max(abs(float(v)) for v in blk)
+            sc = _f32_rne(_f32_rne(amax) / 448.0)
+            assert scales[r, g] == sc
+            for j, v in enumerate(blk):
+                q = _f32_rne(float(v) / sc)  # float32 quotient
+                assert codes[r, 128 * g + j] == codecs.e4m3_encode(q)
+
+
+def test_fp8_project_is_the_sum_of_real_products():
+    rng = np.random.default_rng(9)
+    x = codecs.bf16_round(rng.standard_normal((2, 256)))
+    w = codecs.bf16_round(rng.standard_normal((256, 130)) * 0.05)  # [in, out]
+    wc = codecs.e4m3_encode(w.T / 0.01)
+    ws = np.full((2, 2), 0.01, np.float32)
+    xc, xs = mfa.a8_quantize(x)
+    want = np.zeros((2, 130))
+    for b in range(2):
+        for o in range(130):
+            want[b, o] = math.fsum(float(codecs.e4m3_decode(xc[b, k])) * float(xs[b, k // 128])
+                                   * float(codecs.e4m3_decode(wc[o, k])) * float(ws[o // 128, k // 128])
+                                   for k in range(256))
+    assert np.allclose(mfa.fp8_project(x, wc, ws), want, rtol=1e-12, atol=1e-12)
+
+
+def _f32_rne(x):
+    import struct
+    return struct.unpack("<f", struct.pack("<f", x))[0]
