@@ -57,6 +57,9 @@ def parse_args():
     p.add_argument("--page-size", type=int, default=0,
                    help="keep the KV cache in shuffled pages of this many rows (a multiple of "
                         "64) behind a page table, instead of one buffer per sequence")
+    p.add_argument("--weights", choices=["bf16", "fp8"], default="bf16",
+                   help="projection weights in bf16, or block-FP8 (e4m3 codes, one float32 "
+                        "scale per 128 x 128 block; the layer uses bf16(code * scale))")
     p.add_argument("--page-order", choices=["shuffled", "sequential"], default="shuffled",
                    help="with --page-size: pages handed out in random or in sequence order")
     p.add_argument("--layers", type=int, default=0,
@@ -245,7 +248,7 @@ def run_ours(args, wl, rank, world, local):
     dev = torch.device("cuda", local)
     inp = W.generate_workload(wl, seed=rank_seed(wl, rank))
     bsz = inp.batch
-    step_bytes = WEIGHT_BYTES + kv_bytes(inp)
+    step_bytes = (WEIGHT_BYTES // (2 if args.weights == "fp8" else 1)) + kv_bytes(inp)
     copies = max(2, math.ceil(3 * L2_BYTES / step_bytes))
 
     class Copy:
@@ -256,6 +259,9 @@ def run_ours(args, wl, rank, world, local):
         c = Copy()
         c.x = inp.x.to(dev)
         c.w = [t.to(dev) for t in (inp.w_qdown, inp.gamma, inp.w_qup, inp.w_k, inp.w_v)]
+        if args.weights == "fp8":
+            c.w = [c.w[1] if i == 1 else mfa.BlockFP8Weight(*W.quantize_w8(t))
+                   for i, t in enumerate(c.w)]
         if inp.k_buffer is not None:
             kb, vb = inp.k_buffer.to(dev), inp.v_buffer.to(dev)
             c.k, c.v = [kb[b] for b in range(bsz)], [vb[b] for b in range(bsz)]
@@ -416,6 +422,8 @@ def run_ours(args, wl, rank, world, local):
         "dtype": "bf16" if inp.kv_dtype == "bf16" else "bf16+fp8kv", "data": "synthetic",
         "config": {"workload": wl.name, "batch_per_gpu": bsz, "global_batch": bsz * world,
                    "context": wl.context, "kv_dtype": inp.kv_dtype,
+                   "weights": ("block-fp8 e4m3, 128 x 128 blocks" if args.weights == "fp8"
+                               else "bf16"),
                    "kv_layout": (f"paged, {args.page_size} rows per page, {args.page_order}"
                                  if args.page_size else "one buffer per sequence"),
                    "heads": 64, "head_dim": 256, "hidden": 7168, "q_rank": 2048,
@@ -431,7 +439,9 @@ def run_ours(args, wl, rank, world, local):
                      "bytes_per_launch": a_bytes, "traffic": traffic},
         # the whole step against its roofline: max(flops/TC, bytes/HBM) for the attention plus
         # the same for the linear projections (the pages' cost framing), at the measured peaks
-        "layer_roofline": layer_roofline(step_counts(inp.seq_lens.tolist(), inp.kv_dtype),
+        "layer_roofline": layer_roofline(step_counts(inp.seq_lens.tolist(), inp.kv_dtype,
+                                                     weight_bytes=1 if args.weights == "fp8"
+                                                     else 2),
                                          ms_per_step / 1e3, peak, measured_tensor_peak()),
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT,

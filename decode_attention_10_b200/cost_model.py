@@ -58,9 +58,11 @@ def kv_row_bytes(kv_dtype: str) -> int:
     return HEAD_DIM * (2 if kv_dtype == "bf16" else 1)
 
 
-def step_counts(seq_lens: Iterable[int], kv_dtype: str, o_proj: bool = False) -> StepCounts:
+def step_counts(seq_lens: Iterable[int], kv_dtype: str, o_proj: bool = False,
+                weight_bytes: int = 2) -> StepCounts:
     """Counts of one step of the layer; with ``o_proj`` the output projection (W_o, out
-    read, y written) is added to the linear part."""
+    read, y written) is added to the linear part. ``weight_bytes`` = 1 counts block-FP8
+    projection weights (codes, plus one float32 scale per 128 x 128 block)."""
     lens = [int(n) for n in seq_lens]
     batch, positions = len(lens), sum(lens)
     row = kv_row_bytes(kv_dtype)
@@ -69,7 +71,8 @@ def step_counts(seq_lens: Iterable[int], kv_dtype: str, o_proj: bool = False) ->
     attn_flops = float(ATTN_FLOPS_PER_POSITION) * positions
     linear_flops = 2.0 * batch * WEIGHT_ELEMS
     # weights once; x read (bf16); q written (bf16); the appended K and V rows written
-    linear_bytes = WEIGHT_BYTES + batch * HIDDEN * 2 + batch * Q_WIDTH * 2 + batch * 2 * row
+    w_bytes = WEIGHT_BYTES if weight_bytes == 2 else WEIGHT_ELEMS + 4 * (WEIGHT_ELEMS // 16384)
+    linear_bytes = w_bytes + batch * HIDDEN * 2 + batch * Q_WIDTH * 2 + batch * 2 * row
     if o_proj:
         linear_flops += 2.0 * batch * O_PROJ_ELEMS
         linear_bytes += 2 * O_PROJ_ELEMS + batch * Q_WIDTH * 2 + batch * HIDDEN * 2

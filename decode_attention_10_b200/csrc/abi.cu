@@ -39,6 +39,11 @@ bool encode_rows(CUtensorMap* m, void* base, int rows, int dtype) {
 
 mfa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MFA_OK : MFA_ERR_CUDA; }
 
+bool valid_w8(const mfa_w8& w) {
+  return w.codes != nullptr && aligned16(w.codes) && w.scales != nullptr &&
+         (reinterpret_cast<uintptr_t>(w.scales) & 3u) == 0;
+}
+
 mfa_status check_kv(const mfa_kv_cache* kv) {
   if (kv == nullptr || kv->table == nullptr) return MFA_ERR_INVALID_ARG;
   if (kv->batch < 1 || kv->batch > kMaxBatch) return MFA_ERR_INVALID_ARG;
@@ -65,19 +70,52 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
+// The tensor map of a weight of in_dim x out_dim: bf16 stored [in, out] (boxes [128 k x 64
+// features]), or block-FP8 codes stored [out, in] (boxes [128 features x 128 k]).
+bool encode_weight(CUtensorMap* m, WRef w, int in_dim, int out_dim) {
+  if (w.scales != nullptr) return encode_2d(m, w.ptr, out_dim, in_dim, 1, 128, 128);
+  return encode_2d(m, w.ptr, in_dim, out_dim, 2, 64, 128);
+}
+
+void set_weight_scales(WGemmArgs& p, int i, WRef w, int in_dim) {
+  p.wscale[i] = w.scales;
+  p.wscale_ld[i] = in_dim / 128;
+}
+
+// Where the FP8 path keeps an activation's e4m3 codes and scales (codes null: bf16 path).
+struct Act8 {
+  uint8_t* codes;
+  float* scales;
+};
+
+// X of a projection: bf16 [batch, k] as it is, or (FP8 path) quantized into `a8` first by a
+// kernel of its own; the GEMM's tensor map and scale arguments for it.
+bool prepare_x(CUtensorMap* xm, WGemmArgs& p, const void* x, int batch, int k, Act8 a8,
+               bool quantize, cudaStream_t s) {
+  if (a8.codes == nullptr)
+    return encode_2d(xm, x, (uint64_t)batch, k, 2, 64, wgemm_n_box(batch));
+  if (quantize && launch_quantize_rows(static_cast<const uint16_t*>(x), batch, k, a8.codes,
+                                       a8.scales, s) != cudaSuccess)
+    return false;
+  p.xscale = a8.scales;
+  p.xscale_ld = k / 128;
+  return encode_2d(xm, a8.codes, (uint64_t)batch, k, 1, 128, wgemm_n_box_fp8(batch));
+}
+
 // x [batch, 7168] onto the 128-column tiles [tile_begin, tile_end) of [W_qdown | W_k | W_v]
-// (16 + 2 + 2 tiles), split-K partials into the workspace. Null weights are not read.
-mfa_status run_xproj(const void* x, const void* w_qdown, const void* w_k, const void* w_v,
-                     int batch, int tile_begin, int tile_end, float* part, uint32_t* err,
+// (16 + 2 + 2 tiles), split-K partials into the workspace. Null weights are not read; the
+// three are all bf16 (a8.codes null) or all block-FP8 (x then quantized into a8).
+mfa_status run_xproj(const void* x, WRef w_qdown, WRef w_k, WRef w_v, int batch,
+                     int tile_begin, int tile_end, float* part, uint32_t* err, Act8 a8,
                      cudaStream_t s) {
   CUtensorMap wm[3];
   std::memset(wm, 0, sizeof(wm));
-  if (w_qdown && !encode_2d(&wm[0], w_qdown, kHidden, kRank, 2, 64, 128)) return MFA_ERR_CUDA;
-  if (w_k && !encode_2d(&wm[1], w_k, kHidden, kHeadDim, 2, 64, 128)) return MFA_ERR_CUDA;
-  if (w_v && !encode_2d(&wm[2], w_v, kHidden, kHeadDim, 2, 64, 128)) return MFA_ERR_CUDA;
-  CUtensorMap xm;
-  if (!encode_2d(&xm, x, (uint64_t)batch, kHidden, 2, 64, wgemm_n_box(batch))) return MFA_ERR_CUDA;
+  if (w_qdown.ptr && !encode_weight(&wm[0], w_qdown, kHidden, kRank)) return MFA_ERR_CUDA;
+  if (w_k.ptr && !encode_weight(&wm[1], w_k, kHidden, kHeadDim)) return MFA_ERR_CUDA;
+  if (w_v.ptr && !encode_weight(&wm[2], w_v, kHidden, kHeadDim)) return MFA_ERR_CUDA;
   WGemmArgs p{};
+  CUtensorMap xm;
+  if (!prepare_x(&xm, p, x, batch, kHidden, a8, true, s)) return MFA_ERR_CUDA;
   p.batch = batch;
   p.tile_begin = tile_begin;
   p.three_weights = 1;
@@ -87,19 +125,24 @@ mfa_status run_xproj(const void* x, const void* w_qdown, const void* w_k, const 
   p.out_f32 = part;
   p.out_ld = kXProjCols;
   p.err = err;
+  if (w_qdown.scales != nullptr) {
+    set_weight_scales(p, 0, w_qdown, kHidden);
+    set_weight_scales(p, 1, w_k, kHidden);
+    set_weight_scales(p, 2, w_v, kHidden);
+  }
   return cuda_status(launch_wgemm(wm, xm, p, tile_end - tile_begin, kXProjSplits, s));
 }
 
 // q = bf16(c_hat W_qup): c_hat [batch, 2048], W_qup [2048, 16384], q [batch, 16384].
-mfa_status run_q_up(const uint16_t* c_hat, const void* w_qup, void* q, int batch, uint32_t* err,
-                    cudaStream_t s) {
+mfa_status run_q_up(const uint16_t* c_hat, WRef w_qup, void* q, int batch, uint32_t* err,
+                    Act8 a8, cudaStream_t s) {
   CUtensorMap wm[3];
   std::memset(wm, 0, sizeof(wm));
-  if (!encode_2d(&wm[0], w_qup, kRank, kQWidth, 2, 64, 128)) return MFA_ERR_CUDA;
-  CUtensorMap xm;
-  if (!encode_2d(&xm, c_hat, (uint64_t)batch, kRank, 2, 64, wgemm_n_box(batch)))
-    return MFA_ERR_CUDA;
+  if (!encode_weight(&wm[0], w_qup, kRank, kQWidth)) return MFA_ERR_CUDA;
   WGemmArgs p{};
+  CUtensorMap xm;
+  // (the finish kernel already wrote c_hat's codes and scales on the FP8 path)
+  if (!prepare_x(&xm, p, c_hat, batch, kRank, a8, false, s)) return MFA_ERR_CUDA;
   p.batch = batch;
   p.tile_begin = 0;
   p.three_weights = 0;
@@ -107,18 +150,22 @@ mfa_status run_q_up(const uint16_t* c_hat, const void* w_qup, void* q, int batch
   p.out_bf16 = static_cast<uint16_t*>(q);
   p.out_ld = kQWidth;
   p.err = err;
+  if (w_qup.scales != nullptr) set_weight_scales(p, 0, w_qup, kRank);
   return cuda_status(launch_wgemm(wm, xm, p, kQWidth / 128, 1, s));
 }
 
 
 }  // namespace
 
-mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
-                          const void* w_qup, float eps, void* q_out, int batch, void* ws,
-                          const WsLayout& L, cudaStream_t s) {
+mfa_status run_query_proj(const void* x, WRef w_qdown, const void* gamma, WRef w_qup, float eps,
+                          void* q_out, int batch, void* ws, const WsLayout& L, cudaStream_t s) {
   float* part = at<float>(ws, L.xproj_part);
   uint32_t* err = at<uint32_t>(ws, L.err);
-  mfa_status st = run_xproj(x, w_qdown, nullptr, nullptr, batch, 0, kRank / 128, part, err, s);
+  const bool fp8 = w_qdown.scales != nullptr;
+  const Act8 x8 = fp8 ? Act8{at<uint8_t>(ws, L.x8), at<float>(ws, L.x8_scale)} : Act8{};
+  const Act8 c8 = fp8 ? Act8{at<uint8_t>(ws, L.chat8), at<float>(ws, L.chat8_scale)} : Act8{};
+  mfa_status st =
+      run_xproj(x, w_qdown, WRef{}, WRef{}, batch, 0, kRank / 128, part, err, x8, s);
   if (st != MFA_OK) return st;
   FinishArgs fa{};
   fa.part = part;
@@ -126,9 +173,11 @@ mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
   fa.gamma = static_cast<const uint16_t*>(gamma);
   fa.eps = eps;
   fa.c_hat = at<uint16_t>(ws, L.c_hat);
+  fa.chat8 = c8.codes;
+  fa.chat8_scale = c8.scales;
   fa.err = err;
   if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
-  return run_q_up(fa.c_hat, w_qup, q_out, batch, err, s);
+  return run_q_up(fa.c_hat, w_qup, q_out, batch, err, c8, s);
 }
 
 EncodeTiledFn encode_tiled_fn() {
@@ -339,7 +388,24 @@ mfa_status mfa_query_proj(const void* x, const void* w_qdown, const void* gamma,
   WsLayout L;
   mfa_status st = check_ws(ws, ws_bytes, batch, &L);
   if (st != MFA_OK) return st;
-  return run_query_proj(x, w_qdown, gamma, w_qup, eps, q_out, batch, ws, L,
+  return run_query_proj(x, WRef{w_qdown, nullptr}, gamma, WRef{w_qup, nullptr}, eps, q_out,
+                        batch, ws, L, static_cast<cudaStream_t>(stream));
+}
+
+mfa_status mfa_query_proj_w8(const void* x, mfa_w8 w_qdown, const void* gamma, mfa_w8 w_qup,
+                             float eps, void* q_out, int32_t batch, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (batch < 1 || batch > kMaxBatch) return MFA_ERR_INVALID_ARG;
+  if (!(eps > 0.f)) return MFA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, gamma, q_out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  if (!valid_w8(w_qdown) || !valid_w8(w_qup)) return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  mfa_status st = check_ws(ws, ws_bytes, batch, &L);
+  if (st != MFA_OK) return st;
+  return run_query_proj(x, WRef{w_qdown.codes, w_qdown.scales}, gamma,
+                        WRef{w_qup.codes, w_qup.scales}, eps, q_out, batch, ws, L,
                         static_cast<cudaStream_t>(stream));
 }
 
@@ -356,8 +422,8 @@ mfa_status mfa_kv_append(const void* x, const void* w_k, const void* w_v,
   if (st != MFA_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float* part = at<float>(ws, L.xproj_part);
-  st = run_xproj(x, nullptr, w_k, w_v, kv->batch, kRank / 128, kXProjCols / 128, part,
-                 at<uint32_t>(ws, L.err), s);
+  st = run_xproj(x, WRef{}, WRef{w_k, nullptr}, WRef{w_v, nullptr}, kv->batch, kRank / 128,
+                 kXProjCols / 128, part, at<uint32_t>(ws, L.err), Act8{}, s);
   if (st != MFA_OK) return st;
   FinishArgs fa{};
   fa.part = part;
@@ -434,20 +500,18 @@ mfa_status mfa_o_proj(const void* out, const void* w_o, void* y, int32_t batch, 
   return cuda_status(launch_oproj_finish(part, static_cast<uint16_t*>(y), batch, s));
 }
 
-mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamma,
-                            const void* w_qup, const void* w_k, const void* w_v, float eps,
-                            const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
-                            void* q_out, void* out, void* ws, size_t ws_bytes, void* stream) {
-  mfa_status st = check_kv(kv);
-  if (st != MFA_OK) return st;
-  if (!(eps > 0.f) || !(scale > 0.f)) return MFA_ERR_INVALID_ARG;
-  const void* ptrs[] = {x, w_qdown, gamma, w_qup, w_k, w_v, seq_lens, q_out, out};
-  for (const void* p : ptrs)
-    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
-  WsLayout L;
-  st = check_ws(ws, ws_bytes, kv->batch, &L);
-  if (st != MFA_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+}  // extern "C"
+
+namespace mfa {
+namespace {
+
+// The whole decode step after the host-side checks: x-projection, finish (RMSNorm, append,
+// split plan), q_up, attention, combine.
+mfa_status decode_layer_impl(const void* x, WRef w_qdown, const void* gamma, WRef w_qup,
+                             WRef w_k, WRef w_v, float eps, const mfa_kv_cache* kv,
+                             const int32_t* seq_lens, float scale, void* q_out, void* out,
+                             void* ws, const WsLayout& L, cudaStream_t s) {
+  mfa_status st;
   const int batch = kv->batch;
   AttnArgs aa{};
   aa.q = static_cast<const uint16_t*>(q_out);
@@ -468,8 +532,11 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   aa.page_size = kv->page_size;
   // one projection of x onto [W_qdown | W_k | W_v]
   float* part = at<float>(ws, L.xproj_part);
+  const bool fp8 = w_qdown.scales != nullptr;
+  const Act8 x8 = fp8 ? Act8{at<uint8_t>(ws, L.x8), at<float>(ws, L.x8_scale)} : Act8{};
+  const Act8 c8 = fp8 ? Act8{at<uint8_t>(ws, L.chat8), at<float>(ws, L.chat8_scale)} : Act8{};
   st = run_xproj(x, w_qdown, w_k, w_v, batch, 0, kXProjCols / 128, part,
-                 at<uint32_t>(ws, L.err), s);
+                 at<uint32_t>(ws, L.err), x8, s);
   if (st != MFA_OK) return st;
   // split-K sums, RMSNorm of the query half, K/V append at row seq_lens[b] - 1
   FinishArgs fa{};
@@ -478,6 +545,8 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   fa.gamma = static_cast<const uint16_t*>(gamma);
   fa.eps = eps;
   fa.c_hat = at<uint16_t>(ws, L.c_hat);
+  fa.chat8 = c8.codes;
+  fa.chat8_scale = c8.scales;
   fa.kv = static_cast<const KvSeq*>(kv->table);
   fa.kv_dtype = kv->dtype;
   fa.k_scale = kv->k_scale;
@@ -491,9 +560,53 @@ mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamm
   fa.seq_info = aa.seq_info;
   fa.attn_grid = aa.grid;
   if (launch_xproj_finish(fa, s) != cudaSuccess) return MFA_ERR_CUDA;
-  st = run_q_up(fa.c_hat, w_qup, q_out, batch, fa.err, s);
+  st = run_q_up(fa.c_hat, w_qup, q_out, batch, fa.err, c8, s);
   if (st != MFA_OK) return st;
   return run_attention(aa, s);
+}
+
+}  // namespace
+}  // namespace mfa
+
+extern "C" {
+
+mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamma,
+                            const void* w_qup, const void* w_k, const void* w_v, float eps,
+                            const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
+                            void* q_out, void* out, void* ws, size_t ws_bytes, void* stream) {
+  mfa_status st = check_kv(kv);
+  if (st != MFA_OK) return st;
+  if (!(eps > 0.f) || !(scale > 0.f)) return MFA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_qdown, gamma, w_qup, w_k, w_v, seq_lens, q_out, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  st = check_ws(ws, ws_bytes, kv->batch, &L);
+  if (st != MFA_OK) return st;
+  return decode_layer_impl(x, WRef{w_qdown, nullptr}, gamma, WRef{w_qup, nullptr},
+                           WRef{w_k, nullptr}, WRef{w_v, nullptr}, eps, kv, seq_lens, scale,
+                           q_out, out, ws, L, static_cast<cudaStream_t>(stream));
+}
+
+mfa_status mfa_decode_layer_w8(const void* x, mfa_w8 w_qdown, const void* gamma, mfa_w8 w_qup,
+                               mfa_w8 w_k, mfa_w8 w_v, float eps, const mfa_kv_cache* kv,
+                               const int32_t* seq_lens, float scale, void* q_out, void* out,
+                               void* ws, size_t ws_bytes, void* stream) {
+  mfa_status st = check_kv(kv);
+  if (st != MFA_OK) return st;
+  if (!(eps > 0.f) || !(scale > 0.f)) return MFA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, gamma, seq_lens, q_out, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
+  if (!valid_w8(w_qdown) || !valid_w8(w_qup) || !valid_w8(w_k) || !valid_w8(w_v))
+    return MFA_ERR_INVALID_ARG;
+  WsLayout L;
+  st = check_ws(ws, ws_bytes, kv->batch, &L);
+  if (st != MFA_OK) return st;
+  return decode_layer_impl(x, WRef{w_qdown.codes, w_qdown.scales}, gamma,
+                           WRef{w_qup.codes, w_qup.scales}, WRef{w_k.codes, w_k.scales},
+                           WRef{w_v.codes, w_v.scales}, eps, kv, seq_lens, scale, q_out, out,
+                           ws, L, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -197,27 +197,6 @@ __device__ __forceinline__ float f16_hi(uint32_t w) {
 
 // sixteen e4m3 codes (lowest byte first) -> sixteen f16 values in two 16-byte words, exact:
 // each 16-bit pair of codes becomes one f16x2 word (low byte -> low half)
-__device__ __forceinline__ void e4m3x16_to_f16x16(const uint4 v, uint4& o0, uint4& o1) {
-  asm("{\n"
-      ".reg .b16 c0, c1, c2, c3, c4, c5, c6, c7;\n"
-      "mov.b32 {c0, c1}, %8;\n"
-      "mov.b32 {c2, c3}, %9;\n"
-      "mov.b32 {c4, c5}, %10;\n"
-      "mov.b32 {c6, c7}, %11;\n"
-      "cvt.rn.f16x2.e4m3x2 %0, c0;\n"
-      "cvt.rn.f16x2.e4m3x2 %1, c1;\n"
-      "cvt.rn.f16x2.e4m3x2 %2, c2;\n"
-      "cvt.rn.f16x2.e4m3x2 %3, c3;\n"
-      "cvt.rn.f16x2.e4m3x2 %4, c4;\n"
-      "cvt.rn.f16x2.e4m3x2 %5, c5;\n"
-      "cvt.rn.f16x2.e4m3x2 %6, c6;\n"
-      "cvt.rn.f16x2.e4m3x2 %7, c7;\n"
-      "}\n"
-      : "=r"(o0.x), "=r"(o0.y), "=r"(o0.z), "=r"(o0.w), "=r"(o1.x), "=r"(o1.y), "=r"(o1.z),
-        "=r"(o1.w)
-      : "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
-}
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

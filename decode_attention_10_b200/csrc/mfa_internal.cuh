@@ -77,6 +77,8 @@ struct WsLayout {
   size_t xproj_part;   // fp32 [kXProjSplits][batch][kXProjCols]
   size_t c_hat;        // bf16 [batch][kRank]
   size_t oproj_part;   // fp32 [kOProjSplits][batch][kHidden]
+  size_t x8, x8_scale;        // FP8 path: x as e4m3 [batch][7168] + scales [batch][56]
+  size_t chat8, chat8_scale;  // FP8 path: c_hat as e4m3 [batch][2048] + scales [batch][16]
   size_t total;
   int attn_slots;
   int attn_grid;
@@ -106,6 +108,14 @@ inline WsLayout ws_layout(int batch, int num_sms) {
   off = align_up(off + sizeof(uint16_t) * (size_t)batch * kRank, 256);
   L.oproj_part = off;
   off = align_up(off + sizeof(float) * kOProjSplits * (size_t)batch * kHidden, 256);
+  L.x8 = off;
+  off = align_up(off + (size_t)batch * kHidden, 256);
+  L.x8_scale = off;
+  off = align_up(off + sizeof(float) * (size_t)batch * (kHidden / 128), 256);
+  L.chat8 = off;
+  off = align_up(off + (size_t)batch * kRank, 256);
+  L.chat8_scale = off;
+  off = align_up(off + sizeof(float) * (size_t)batch * (kRank / 128), 256);
   L.total = off;
   return L;
 }
@@ -148,14 +158,23 @@ struct WGemmArgs {
   uint16_t* out_bf16;   // bf16 [batch][out_ld] (when out_f32 is null)
   int out_ld;
   uint32_t* err;
-  int n_box, stages, tmem_cols;  // filled in by launch_wgemm
+  // block-FP8 weights: per weight its scales [N_out / 128][wscale_ld] (row-major, one per
+  // 128 x 128 block); null = bf16 weights
+  const float* wscale[3];
+  int wscale_ld[3];
+  // FP8 path: X is e4m3 codes [batch, K] with scales [batch][xscale_ld] (one per 128 k)
+  const float* xscale;
+  int xscale_ld;
+  int n_box, stages, tmem_cols, dbufs;  // filled in by launch_wgemm
 };
-// w: 3 tensor maps over row-major [K, N_out] bf16 weights, boxes [128 k x 64 features];
+// w: 3 tensor maps over row-major [K, N_out] bf16 weights, boxes [128 k x 64 features], or
+// for block-FP8 weights over [N_out, K] e4m3 codes, boxes [128 features x 128 k];
 // xmap over X [batch, K] bf16, boxes [wgemm_n_box(batch) x 64 k]; all with 128-byte swizzle.
 // kblocks_per_cta counts blocks of 128 k.
 cudaError_t launch_wgemm(const CUtensorMap* w, const CUtensorMap& xmap, WGemmArgs p,
                          int m_tiles, int splits, cudaStream_t s);
 int wgemm_n_box(int batch);
+int wgemm_n_box_fp8(int batch);  // the FP8 path's X box rows (at most 128 rows per CTA)
 
 struct FinishArgs {
   const float* part;  // x-projection partials
@@ -164,6 +183,8 @@ struct FinishArgs {
   const uint16_t* gamma;  // null = skip the query half
   float eps;
   uint16_t* c_hat;  // [batch, 2048]
+  uint8_t* chat8;        // FP8 path: c_hat also as e4m3 [batch, 2048] (null = bf16 path)
+  float* chat8_scale;    // FP8 path: its scales [batch, 16], one per 128 columns
   // K/V half: append bf16 / e4m3 rows
   const KvSeq* kv;  // null = skip the K/V half
   int kv_dtype;
@@ -179,6 +200,11 @@ struct FinishArgs {
   int attn_grid;
 };
 cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s);
+
+// The FP8 path's activations: a [rows, k] bf16 -> e4m3 codes [rows, k] and float32 scales
+// [rows, k / 128], per row and group of 128 values (query_path.cu).
+cudaError_t launch_quantize_rows(const uint16_t* a, int rows, int k, uint8_t* codes,
+                                 float* scales, cudaStream_t s);
 
 // y = bf16(partial[0] + partial[1]) over batch x 7168 fp32 partials (out_proj.cu).
 cudaError_t launch_oproj_finish(const float* part, uint16_t* y, int batch, cudaStream_t s);
@@ -211,11 +237,17 @@ size_t attention_tc_smem_bytes();
 // dependent.
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s);
 
+// A projection weight: bf16 stored [in, out] (scales null), or block-FP8 e4m3 codes stored
+// [out, in] with one float32 scale per 128 x 128 block ([out / 128, in / 128]).
+struct WRef {
+  const void* ptr;
+  const float* scales;
+};
+
 // The query path (x-projection onto W_qdown, finish with RMSNorm, q_up) on `s`, using the
 // x-projection partials, c_hat and error word at the offsets of L inside `ws`.
-mfa_status run_query_proj(const void* x, const void* w_qdown, const void* gamma,
-                          const void* w_qup, float eps, void* q_out, int batch, void* ws,
-                          const WsLayout& L, cudaStream_t s);
+mfa_status run_query_proj(const void* x, WRef w_qdown, const void* gamma, WRef w_qup, float eps,
+                          void* q_out, int batch, void* ws, const WsLayout& L, cudaStream_t s);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable).
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -83,5 +83,6 @@ extern "C" MFA_API mfa_status mfa_query_proj_noalloc(const void* x, const void* 
   if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + L.err, 0, sizeof(uint32_t), s) !=
       cudaSuccess)
     return MFA_ERR_CUDA;
-  return run_query_proj(x, w_qdown, gamma, w_qup, eps, q_out, batch, scratch, L, s);
+  return run_query_proj(x, WRef{w_qdown, nullptr}, gamma, WRef{w_qup, nullptr}, eps, q_out,
+                        batch, scratch, L, s);
 }

@@ -84,9 +84,40 @@ __global__ void __launch_bounds__(kFinishThreads) xproj_finish_kernel(FinishArgs
     const float ss = block_sum_1024(fmaf(c0, c0, c1 * c1), red);
     const float r = rsqrtf(ss * (1.0f / kRank) + a.eps);
     uint16_t* ch = a.c_hat + (size_t)b * kRank;
-    ch[tid] = f32_to_bf16_bits(c0 * r * bf16_bits_to_f32(a.gamma[tid]));
-    ch[tid + kFinishThreads] =
+    const uint16_t h0 = f32_to_bf16_bits(c0 * r * bf16_bits_to_f32(a.gamma[tid]));
+    const uint16_t h1 =
         f32_to_bf16_bits(c1 * r * bf16_bits_to_f32(a.gamma[tid + kFinishThreads]));
+    ch[tid] = h0;
+    ch[tid + kFinishThreads] = h1;
+    if (a.chat8 != nullptr) {
+      // the FP8 path: c_hat (as stored, bf16) quantized per group of 128 columns -- group g
+      // is the columns of warps 4 (g mod 8) .. 4 (g mod 8) + 3, in the first half for g < 8
+      __shared__ float gmax[32][2];
+      const float v0 = bf16_bits_to_f32(h0), v1 = bf16_bits_to_f32(h1);
+      float m0 = fabsf(v0), m1 = fabsf(v1);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      }
+      const int warp = tid >> 5, gw = warp & ~3;
+      if ((tid & 31) == 0) {
+        gmax[warp][0] = m0;
+        gmax[warp][1] = m1;
+      }
+      __syncthreads();
+      const float a0 = fmaxf(fmaxf(gmax[gw][0], gmax[gw + 1][0]), fmaxf(gmax[gw + 2][0], gmax[gw + 3][0]));
+      const float a1 = fmaxf(fmaxf(gmax[gw][1], gmax[gw + 1][1]), fmaxf(gmax[gw + 2][1], gmax[gw + 3][1]));
+      const float s0 = a0 > 0.f ? __fdiv_rn(a0, 448.f) : 1.f;
+      const float s1 = a1 > 0.f ? __fdiv_rn(a1, 448.f) : 1.f;
+      uint8_t* q8 = a.chat8 + (size_t)b * kRank;
+      q8[tid] = f32_to_e4m3(__fdiv_rn(v0, s0));
+      q8[tid + kFinishThreads] = f32_to_e4m3(__fdiv_rn(v1, s1));
+      if ((tid & 127) == 0) {
+        a.chat8_scale[(size_t)b * (kRank / 128) + (tid >> 7)] = s0;
+        a.chat8_scale[(size_t)b * (kRank / 128) + 8 + (tid >> 7)] = s1;
+      }
+    }
   }
   if (!do_kv) return;
   const int row = a.pos[b] - (a.pos_from_len ? 1 : 0);
@@ -117,7 +148,42 @@ __global__ void __launch_bounds__(kFinishThreads) xproj_finish_kernel(FinishArgs
   }
 }
 
+// The FP8 path's activations: one warp per (row, group of 128 values); lane l holds values
+// 4 l .. 4 l + 3. scale = max |a| / 448 (1 for an all-zero group), code = e4m3(a / scale),
+// both float32 operations rounded to nearest even, the code saturating.
+__global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* __restrict__ a,
+                                                           int rows, int k,
+                                                           uint8_t* __restrict__ codes,
+                                                           float* __restrict__ scales) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int groups = k / 128;
+  const int task = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (task >= rows * groups) return;
+  const int r = task / groups, g = task % groups;
+  const size_t off = (size_t)r * k + 128 * g + 4 * lane;
+  const uint2 raw = *reinterpret_cast<const uint2*>(a + off);
+  const float v[4] = {bf16_bits_to_f32(raw.x & 0xFFFFu), bf16_bits_to_f32(raw.x >> 16),
+                      bf16_bits_to_f32(raw.y & 0xFFFFu), bf16_bits_to_f32(raw.y >> 16)};
+  float m = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  const float sc = m > 0.f ? __fdiv_rn(m, 448.f) : 1.f;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) packed |= static_cast<uint32_t>(f32_to_e4m3(__fdiv_rn(v[i], sc))) << (8 * i);
+  *reinterpret_cast<uint32_t*>(codes + off) = packed;
+  if (lane == 0) scales[(size_t)r * groups + g] = sc;
+}
+
 }  // namespace
+
+cudaError_t launch_quantize_rows(const uint16_t* a, int rows, int k, uint8_t* codes,
+                                 float* scales, cudaStream_t s) {
+  const int tasks = rows * (k / 128);
+  return launch_pdl(quantize_rows_kernel, dim3((tasks + 7) / 8), dim3(256), 0, s, a, rows, k,
+                    codes, scales);
+}
 
 cudaError_t launch_xproj_finish(const FinishArgs& a, cudaStream_t s) {
   const int blocks = a.batch + (a.plan != nullptr ? 1 : 0);

@@ -172,6 +172,29 @@ __device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// 16 e4m3 codes (one uint4, code 0 in the low byte) -> 16 f16 values, exactly (every e4m3
+// value is an f16 value): o0 holds codes 0..7, o1 codes 8..15, two per 32-bit word.
+__device__ __forceinline__ void e4m3x16_to_f16x16(const uint4 v, uint4& o0, uint4& o1) {
+  asm("{\n"
+      ".reg .b16 c0, c1, c2, c3, c4, c5, c6, c7;\n"
+      "mov.b32 {c0, c1}, %8;\n"
+      "mov.b32 {c2, c3}, %9;\n"
+      "mov.b32 {c4, c5}, %10;\n"
+      "mov.b32 {c6, c7}, %11;\n"
+      "cvt.rn.f16x2.e4m3x2 %0, c0;\n"
+      "cvt.rn.f16x2.e4m3x2 %1, c1;\n"
+      "cvt.rn.f16x2.e4m3x2 %2, c2;\n"
+      "cvt.rn.f16x2.e4m3x2 %3, c3;\n"
+      "cvt.rn.f16x2.e4m3x2 %4, c4;\n"
+      "cvt.rn.f16x2.e4m3x2 %5, c5;\n"
+      "cvt.rn.f16x2.e4m3x2 %6, c6;\n"
+      "cvt.rn.f16x2.e4m3x2 %7, c7;\n"
+      "}\n"
+      : "=r"(o0.x), "=r"(o0.y), "=r"(o0.z), "=r"(o0.w), "=r"(o1.x), "=r"(o1.y), "=r"(o1.z),
+        "=r"(o1.w)
+      : "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w));
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -274,6 +297,20 @@ __device__ __forceinline__ void umma_f16_ss(uint32_t d_tmem, uint64_t adesc, uin
       ".reg .pred p;\n"
       "setp.ne.b32 p, %4, 0;\n"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem] for 8-bit e4m3 operands (K = 32 per instruction; the
+// instruction descriptor's A and B format fields are 0 for e4m3), single CTA, one thread.
+__device__ __forceinline__ void umma_f8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      ".reg .pred p;\n"
+      "setp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n"
       "}\n" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");

@@ -22,6 +22,11 @@ STATUS = {0: "MFA_OK", 1: "MFA_ERR_INVALID_ARG", 2: "MFA_ERR_UNSUPPORTED",
           3: "MFA_ERR_CAPACITY", 4: "MFA_ERR_WORKSPACE", 5: "MFA_ERR_CUDA",
           6: "MFA_ERR_EMPTY", 7: "MFA_ERR_TIMEOUT"}
 
+class W8(ctypes.Structure):
+    """mfa_w8: a block-FP8 weight (device pointers to codes and scales)."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
 # name -> (restype, argtypes), mirroring include/mfa.h
 _P = ctypes.c_void_p
 _SIGNATURES = {
@@ -44,6 +49,10 @@ _SIGNATURES = {
     "mfa_decode_layer": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
                                         ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
     "mfa_o_proj": (ctypes.c_int, [_P, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "mfa_query_proj_w8": (ctypes.c_int, [_P, W8, _P, W8, ctypes.c_float, _P, ctypes.c_int32,
+                                         _P, ctypes.c_size_t, _P]),
+    "mfa_decode_layer_w8": (ctypes.c_int, [_P, W8, _P, W8, W8, W8, ctypes.c_float, _P, _P,
+                                           ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]),
     "mfa_query_proj_noalloc": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_float, _P,
                                               ctypes.c_int32, _P]),
     "mfa_wait_selftest": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_uint32, _P]),
@@ -198,6 +207,23 @@ class PagedKVCache:
                                 self.table.data_ptr(), self.page_size)
 
 
+class BlockFP8Weight:
+    """A block-FP8 projection weight for the library: e4m3 codes [out, in] (a CUDA uint8 or
+    float8_e4m3fn tensor) and one float32 scale per 128 x 128 block ([out / 128, in / 128]);
+    the layer multiplies with bf16(code * scale)."""
+
+    def __init__(self, codes: torch.Tensor, scales: torch.Tensor):
+        if codes.dim() != 2 or codes.element_size() != 1 or not codes.is_contiguous():
+            raise ValueError("codes must be a contiguous [out, in] tensor of one-byte codes")
+        out_dim, in_dim = int(codes.shape[0]), int(codes.shape[1])
+        if (scales.dtype != torch.float32 or not scales.is_contiguous()
+                or tuple(scales.shape) != (-(-out_dim // 128), -(-in_dim // 128))):
+            raise ValueError("scales must be contiguous float32 [out / 128, in / 128]")
+        _ptr(codes), _ptr(scales)
+        self.codes, self.scales = codes, scales
+        self.struct = W8(codes.data_ptr(), scales.data_ptr())
+
+
 class Workspace:
     """Device workspace for `batch` sequences (allocated by torch, zeroed by the library)."""
 
@@ -288,6 +314,20 @@ def o_proj(out, w_o, y=None, ws=None, stream=None) -> torch.Tensor:
     return y
 
 
+def query_proj_w8(x, w_qdown: "BlockFP8Weight", gamma, w_qup: "BlockFP8Weight",
+                  eps: float = 1e-6, q_out=None, ws=None, stream=None) -> torch.Tensor:
+    """mfa_query_proj with block-FP8 weights."""
+    lib = load()
+    bsz = int(x.shape[0])
+    if q_out is None:
+        q_out = torch.empty(bsz, N_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=x.device)
+    ws = ws if ws is not None else Workspace(bsz, x.device)
+    _check(lib.mfa_query_proj_w8(_ptr(x), w_qdown.struct, _ptr(gamma), w_qup.struct,
+                                 float(eps), _ptr(q_out), bsz, ws.ptr, ws.nbytes,
+                                 _stream(stream)), "mfa_query_proj_w8")
+    return q_out
+
+
 def query_proj_noalloc(x, w_qdown, gamma, w_qup, eps: float = 1e-6, q_out=None, stream=None):
     """mfa_query_proj without a workspace: the library's built-in scratch (batch <= 32)."""
     lib = load()
@@ -318,13 +358,16 @@ class DecodeStep:
                  stream=None):
         self._lib = load()
         self._keep = (x, w_qdown, gamma, w_qup, w_k, w_v, cache, seq_lens, q_out, out, ws)
-        self._args = (_P(_ptr(x)), _P(_ptr(w_qdown)), _P(_ptr(gamma)), _P(_ptr(w_qup)),
-                      _P(_ptr(w_k)), _P(_ptr(w_v)), ctypes.c_float(eps),
-                      ctypes.byref(cache.desc), _P(_ptr(seq_lens)), ctypes.c_float(scale),
-                      _P(_ptr(q_out)), _P(_ptr(out)), _P(ws.ptr), ctypes.c_size_t(ws.nbytes),
-                      _P(_stream(stream)))
+        # weights: bf16 tensors, or BlockFP8Weight (then mfa_decode_layer_w8)
+        self._w8 = isinstance(w_qdown, BlockFP8Weight)
+        wa = (lambda w: w.struct) if self._w8 else (lambda w: _P(_ptr(w)))
+        self._fn = self._lib.mfa_decode_layer_w8 if self._w8 else self._lib.mfa_decode_layer
+        self._args = (_P(_ptr(x)), wa(w_qdown), _P(_ptr(gamma)), wa(w_qup), wa(w_k), wa(w_v),
+                      ctypes.c_float(eps), ctypes.byref(cache.desc), _P(_ptr(seq_lens)),
+                      ctypes.c_float(scale), _P(_ptr(q_out)), _P(_ptr(out)), _P(ws.ptr),
+                      ctypes.c_size_t(ws.nbytes), _P(_stream(stream)))
 
     def __call__(self):
-        st = self._lib.mfa_decode_layer(*self._args)
+        st = self._fn(*self._args)
         if st != 0:
-            raise MfaError(st, "mfa_decode_layer")
+            raise MfaError(st, "mfa_decode_layer_w8" if self._w8 else "mfa_decode_layer")

@@ -214,6 +214,24 @@ def generate_layer_on_device(seq_lens: Sequence[int], kv_dtype: str, seed: int, 
     return d
 
 
+def quantize_w8(w: torch.Tensor, block: int = 128):
+    """A bf16 weight [in, out] drawn by ``generate``, stored as block FP8 in the checkpoints'
+    order: e4m3 codes [out, in] (uint8) and one float32 scale per block x block tile (its
+    largest |w| / 448; 1 for an all-zero tile), the values w / scale rounded to nearest even
+    and kept within +-448. Returns (codes, scales) on w's device."""
+    wt = w.t().float()
+    o, i = wt.shape
+    bo, bi = -(-o // block), -(-i // block)
+    pad = torch.zeros(bo * block, bi * block, dtype=torch.float32, device=w.device)
+    pad[:o, :i] = wt
+    tiles = pad.view(bo, block, bi, block)
+    amax = tiles.abs().amax(dim=(1, 3))
+    scales = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax)).float()
+    q = (tiles / scales[:, None, :, None]).clamp(-448.0, 448.0).to(torch.float8_e4m3fn)
+    codes = q.view(bo * block, bi * block)[:o, :i].contiguous().view(torch.uint8)
+    return codes, scales.contiguous()
+
+
 def to_paged(k_cache: Sequence[torch.Tensor], v_cache: Sequence[torch.Tensor], page_size: int,
              seed: int, spare_pages: int = 0, shuffle: bool = True):
     """The per-sequence caches ([capacity_b, 256] tensors, on any device) copied into K and V

@@ -205,6 +205,40 @@ MFA_API mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const vo
                             const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
                             void* q_out, void* out, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Block-FP8 weights
+ * ------------------------------------------------------------------------------------- */
+
+/* A block-FP8 projection weight (step3-fp8 model page, "Deployment": the checkpoints are
+ * stored in bf16 and in block-fp8; the Step-3 pages: the whole model runs in FP8). The pages
+ * give neither block size nor arithmetic; the library's reading: e4m3 codes in the
+ * checkpoints' [out, in] order (row-major, out rows of `in` codes) with one float32 scale per
+ * 128 x 128 block, and the projection runs in FP8: its input row is quantized per group of
+ * 128 values (scale = max |a| / 448, code = e4m3(a / scale), both float32 operations rounded
+ * to nearest even, the code saturating), the tensor cores multiply codes (e4m3 x e4m3, float32
+ * accumulation), and each 128-wide block of the sum is scaled by its weight and activation
+ * scales: y = sum over blocks of s_w s_a sum(code_w code_a). The RMSNorm, the K/V cache and the
+ * attention are as in the bf16 calls. The weights stream from HBM as codes (half the bytes). */
+typedef struct {
+  const void* codes;    /* device uint8 [out, in], 16-byte aligned */
+  const float* scales;  /* device float32 [out / 128, in / 128] (row-major), 4-byte aligned */
+} mfa_w8;
+
+/* mfa_query_proj on the FP8 path: block-FP8 W_qdown (codes [2048, 7168], scales [16, 56])
+ * and W_qup (codes [16384, 2048], scales [128, 16]); x and c_hat quantized as above.
+ * Errors as mfa_query_proj. */
+MFA_API mfa_status mfa_query_proj_w8(const void* x, mfa_w8 w_qdown, const void* gamma,
+                                     mfa_w8 w_qup, float eps, void* q_out, int32_t batch,
+                                     void* ws, size_t ws_bytes, void* stream);
+
+/* mfa_decode_layer on the FP8 path: W_qdown and W_qup as in mfa_query_proj_w8, W_k and W_v
+ * codes [256, 7168] with scales [2, 56]. Errors as mfa_decode_layer. */
+MFA_API mfa_status mfa_decode_layer_w8(const void* x, mfa_w8 w_qdown, const void* gamma,
+                                       mfa_w8 w_qup, mfa_w8 w_k, mfa_w8 w_v, float eps,
+                                       const mfa_kv_cache* kv, const int32_t* seq_lens,
+                                       float scale, void* q_out, void* out, void* ws,
+                                       size_t ws_bytes, void* stream);
+
 /* Output projection of the attention (pages: bud-325 "Method" -- the per-token decoding
  * cost counts the linear projections around attention, and each layer's attention hands a
  * hidden-width vector to the FFN; the 16384 -> 7168 shape is the reading that the 64 x 256

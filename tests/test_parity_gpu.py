@@ -572,3 +572,79 @@ def test_cache_description_contradicting_its_table_is_reported():
     out = mfa.decode_attn(q, step.cache, seq_lens, ws=ws)
     assert mfa.get_error(ws) == 0
     assert np.isfinite(bf16_np(out)).all()
+
+
+# ----------------------------------------------------------------------------------------
+# the FP8 path: block-FP8 weights (e4m3 codes [out, in], one float32 scale per 128 x 128
+# block) and FP8 activations (per row and 128 values)
+# ----------------------------------------------------------------------------------------
+
+
+def _q_close_fp8(q_gpu, q_ref):
+    # The FP8 path decides integer codes from float inputs twice: x's codes are computed
+    # identically on both sides, but c_hat comes from float32 (GPU) and float64 (oracle) sums,
+    # so a one-ulp difference in a group's largest |c_hat| moves that group's scale and can
+    # move every code in it by one e4m3 step (up to 2^-3 relative). Each moved code shifts q
+    # by about 0.0625 |c_hat| |W_qup| (~1.4e-3); a group's 128 codes move with random signs,
+    # so a few 1e-2 at most. Bound: rel-L2 1e-3, max-abs 5e-2, and at most 0.1 % of the
+    # elements beyond the two-ulp bf16 bound of the bf16 path.
+    ulp = np.ldexp(1.0, np.frexp(np.abs(q_ref))[1] - 8)
+    off = np.abs(q_gpu - q_ref) > 2 * ulp + 1e-3
+    assert off.mean() <= 1e-3, f"{off.sum()} q elements beyond two ulps"
+    assert max_abs(q_gpu, q_ref) <= 5e-2
+    assert rel_l2(q_gpu, q_ref) <= 1e-3
+
+
+def _w8(w_bf16):
+    from decode_attention_10_b200 import mfa
+    codes, scales = W.quantize_w8(w_bf16)
+    return mfa.BlockFP8Weight(codes.cuda(), scales.cuda()), codes.numpy(), scales.numpy()
+
+
+@pytest.mark.parametrize("bsz", [1, 32, 300])
+def test_query_proj_w8_matches_oracle(bsz):
+    from decode_attention_10_b200 import mfa
+    inp = W.generate([1] * bsz, W.KV_BF16, seed=110 + bsz)
+    wq, cq, sq = _w8(inp.w_qdown)
+    wu, cu, su = _w8(inp.w_qup)
+    q = mfa.query_proj_w8(inp.x.cuda(), wq, inp.gamma.cuda(), wu)
+    torch.cuda.synchronize()
+    ow = oracle_weights(inp)
+    _, q_ref = omfa.query_proj_fp8(ow["x"], cq, sq, ow["gamma"], cu, su)
+    _q_close_fp8(bf16_np(q), q_ref)
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_layer_w8_matches_oracle(kv_dtype):
+    from decode_attention_10_b200 import mfa
+    lens = [1, 130, 300, 129, 64]
+    inp = W.generate(lens, kv_dtype, seed=120)
+    step = GpuStep(inp)
+    k_before = [codes_np(t) for t in step.k]
+    v_before = [codes_np(t) for t in step.v]
+    w8s = [_w8(w) for w in (inp.w_qdown, inp.w_qup, inp.w_k, inp.w_v)]
+    q = torch.empty(len(lens), 64, 256, dtype=torch.bfloat16, device="cuda")
+    out = torch.empty_like(q)
+    run = mfa.DecodeStep(step.x, w8s[0][0], step.gamma, w8s[1][0], w8s[2][0], w8s[3][0],
+                         step.cache, step.seq_lens, q, out, step.ws)
+    run()
+    torch.cuda.synchronize()
+    assert mfa.get_error(step.ws) == 0
+    od = oracle_dtype(kv_dtype)
+    ow = oracle_weights(inp)
+    (_, cq, sq), (_, cu, su), (_, ck, sk), (_, cv, sv) = w8s
+    _, q_ref = omfa.query_proj_fp8(ow["x"], cq, sq, ow["gamma"], cu, su)
+    _q_close_fp8(bf16_np(q), q_ref)
+    # the appended rows: one code apart at most from the oracle's (fp32 vs float64 sums)
+    k_new, v_new = omfa.fp8_project(ow["x"], ck, sk), omfa.fp8_project(ow["x"], cv, sv)
+    for b, n in enumerate(lens):
+        for t, want in ((step.k[b], omfa.kv_store(k_new[b], od, inp.k_scale)),
+                        (step.v[b], omfa.kv_store(v_new[b], od, inp.v_scale))):
+            got = codes_np(t)[n - 1].astype(np.int64)
+            assert np.abs(got - want.astype(np.int64)).max() <= 1
+    # end to end: the oracle's own chain (its q, its appended rows, its attention)
+    k_codes = omfa.kv_store(k_new, od, inp.k_scale)
+    v_codes = omfa.kv_store(v_new, od, inp.v_scale)
+    k2, v2 = omfa.kv_append(k_before, v_before, [n - 1 for n in lens], k_codes, v_codes)
+    ref = omfa.decode_attn(q_ref, k2, v2, lens, od, inp.k_scale, inp.v_scale)
+    assert_close(bf16_np(out), ref, kv_dtype, "FP8-path layer (end to end)")
