@@ -132,7 +132,7 @@ def test_layer_per_sequence_buffers_with_spare_capacity():
     _check_layer(inp)
 
 
-def _attn_case(lens, kv_dtype, seed, caps=None, nan_tail=False, q_scale=1.0):
+def _attn_case(lens, kv_dtype, seed, caps=None, nan_tail=False, q_scale=1.0, ws=None):
     from decode_attention_10_b200 import mfa
     inp = W.generate(lens, kv_dtype, seed=seed, contiguous=False, capacity=caps)
     g = torch.Generator().manual_seed(seed + 7)
@@ -146,7 +146,7 @@ def _attn_case(lens, kv_dtype, seed, caps=None, nan_tail=False, q_scale=1.0):
     kd = [t.cuda() for t in k]
     vd = [t.cuda() for t in v]
     cache = mfa.KVCache(kd, vd, inp.k_scale, inp.v_scale)
-    out = mfa.decode_attn(q.cuda(), cache, inp.seq_lens.cuda())
+    out = mfa.decode_attn(q.cuda(), cache, inp.seq_lens.cuda(), ws=ws)
     torch.cuda.synchronize()
     ref = omfa.decode_attn(bf16_np(q), [codes_np(t) for t in k], [codes_np(t) for t in v],
                            lens, oracle_dtype(kv_dtype), inp.k_scale, inp.v_scale)
@@ -177,12 +177,33 @@ def test_attention_rows_past_length_are_ignored(kv_dtype):
     assert_close(out, ref, kv_dtype, "NaN past length")
 
 
-def test_attention_long_sequence_split_over_many_ctas():
-    # one 40,000-position sequence spans ~313 tiles, more than one per SM: split-K + merge
-    out, ref, _ = _attn_case([40000], W.KV_BF16, seed=23)
-    assert_close(out, ref, W.KV_BF16, "long single sequence")
-    out, ref, _ = _attn_case([65536, 3, 20000], W.KV_BF16, seed=24)
-    assert_close(out, ref, W.KV_BF16, "mixed long")
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_attention_long_sequence_split_over_many_ctas(kv_dtype):
+    # one 40,000-position sequence spans ~313 tiles, more than one per SM: it is split over
+    # every CTA, and the merge takes the path for more than 8 splits
+    out, ref, _ = _attn_case([40000], kv_dtype, seed=23)
+    assert_close(out, ref, kv_dtype, "long single sequence")
+    out, ref, _ = _attn_case([65536, 3, 20000], kv_dtype, seed=24)
+    assert_close(out, ref, kv_dtype, "mixed long")
+
+
+def test_attention_one_workspace_across_differently_split_calls():
+    # One workspace across calls whose sequences split differently (2 to 148 CTAs per
+    # sequence, sequences finished by one CTA alone, lengths of 1 and 5). Each call rewrites
+    # the per-sequence split information and the partial slots in the workspace; nothing an
+    # earlier call left there may reach a later call's merge.
+    from decode_attention_10_b200 import mfa
+    ws = mfa.Workspace(16)
+    cases = [[9000, 300, 20000], [40000], [700] * 16, [5, 4096, 1, 65, 12000],
+             [9000, 300, 20000]]
+    outs = []
+    for i, lens in enumerate(cases):
+        out, ref, _ = _attn_case(lens, W.KV_BF16, seed=60 + (i % 4), ws=ws)
+        assert mfa.get_error(ws) == 0
+        assert_close(out, ref, W.KV_BF16, f"call {i} on one workspace")
+        outs.append(out)
+    # the combine adds the splits in a fixed order: the same call gives the same bits
+    assert np.array_equal(outs[0], outs[4])
 
 
 def test_attention_sharp_softmax():
