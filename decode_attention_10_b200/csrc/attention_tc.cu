@@ -28,16 +28,19 @@
 //   Tiles are windows of 128 positions; the last window of a work item ends at the item's
 //   end (it may start before the item or at a negative position, which TMA zero-fills), so
 //   rows past a sequence's length are never read. Positions outside the item are masked.
-// FP8 caches: TMA brings raw e4m3 boxes of [128 positions x 128 dims], and the eight
-// softmax warps convert them (e4m3 -> f16 is exact). A K tile (two boxes through a 2-slot raw
-// ring) goes straight into tensor memory (two 128-column buffers), where the S^T product
-// reads it as its A operand. A V box lands in the upper half of a 32 KB V slot and is
-// converted in place into the slot's two swizzled 16 KB chunks, the layout the bf16 path
-// streams; four slots hold two V tiles, so converting V(t) never waits for PV(t - 1). Per
-// tile the softmax warps do K(t + 1), V(t), then the softmax of t. Both products run with f16
-// operands: Q is converted to f16 in place once per item (scaled by a power of two if its
-// magnitude could overflow f16), P is written as f16. The K and V scales fold into the
-// softmax scale and the output scale.
+// FP8 caches: the e4m3 codes go to the tensor cores as they are (tcgen05 kind::f8f6f4; e4m3
+// values times the power-of-two scales below are exact, and so are the products). The ring
+// holds raw boxes of [128 positions x 128 dims] (128 bytes a row, the same swizzle), two per
+// K or V tile, ten in flight. The other operand must be e4m3 too, so Q and P each become a
+// pair of e4m3 matrices with one common scale, a high part and the rounded remainder (hi +
+// lo keeps 7 to 8 significant bits, about what bf16 keeps), stacked along N:
+//   S^T(t)[128 pos x 128] = K(t) . [Q_hi ; Q_lo]^T        (M=128, N=128: hi heads, lo heads)
+//   O^T[256 x 128]     += V(t)^T . [P_hi | P_lo]^T(t)  (2 x M=128, N=128)
+// and the softmax adds the two halves of S, the epilogue those of O. Q is split once per
+// work item (scaled by 2^-e so that its largest magnitude is in [128, 256)); P is computed as
+// 2^(s - m + 4) and raised m only when a tile's max exceeds it by more than 4, so P stays
+// below 2^8 and its useful values clear e4m3's subnormal range. The K and V scales fold into
+// the softmax scale and the output scale.
 // The split plan (which CTA streams which tiles) is computed on chip: see attn_plan.cuh.
 // A sequence covered by one CTA is finished in place; the items of a sequence split over
 // several CTAs leave (m, l, acc) partials that attention_combine_kernel merges.
@@ -57,40 +60,44 @@ constexpr int kThreads = 320;
 constexpr int kSoftmaxWarps = 8;        // warps 2..9
 constexpr int kGroupThreads = 128;      // one softmax group = four warps = the 128 lanes
 constexpr int kGroupHeads = 32;         // heads per group
-constexpr int kChunkBytes = 16384;      // [128 positions x 64 dims] 16-bit, 128-byte swizzle
+// a ring box: [128 positions x 128 bytes] (64 bf16 dims, or 128 e4m3 dims), 128-byte swizzle
+constexpr int kChunkBytes = 16384;
 constexpr int kRingBytes = 10 * kChunkBytes;
-constexpr int kRawBytes = 16384;         // FP8: a raw e4m3 box [128 positions x 128 dims]
-constexpr int kKRawSlots = 2;           // FP8: raw K boxes (one K tile)
-constexpr int kVSlots = 4;              // FP8: V slots of 32 KB (two V tiles)
-constexpr int kVSlotBytes = 2 * kChunkBytes;
-constexpr int kKRawOff = kVSlots * kVSlotBytes;
 constexpr int kMaxSlots = 10;
-constexpr int kQChunkBytes = 8192;      // [64 heads x 64 dims] 16-bit
-constexpr int kPBytes = 16384;          // P^T: [128 positions x 64 heads] 16-bit
-constexpr uint32_t kTmemS = 0;          // S^T buffers: columns [0, 64) and [64, 128)
-constexpr uint32_t kTmemO = 128;        // O^T halves: columns [128, 192) and [192, 256)
-constexpr uint32_t kTmemK = 256;        // FP8: f16 K tiles (A operand), [256, 384), [384, 512)
+constexpr int kQChunkBytes = 8192;      // bf16 Q box: [64 heads x 64 dims]
+constexpr int kQ8ChunkBytes = 16384;    // FP8 Q: [128 rows (hi, then lo) x 128 dims] e4m3
+constexpr int kPBytes = 16384;          // P^T: [128 positions x 128 bytes]
+constexpr uint32_t kTmemS = 0;          // S^T buffers from column 0 (see Cfg::kSCols)
 constexpr int kPageIds = 128;          // paged caches: page ids held per work item
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // named barriers: 1 + group among one softmax group, 3 among all eight softmax warps
 constexpr uint32_t kBarAllSoftmax = 3;
 
-// Per cache type: the ring area's use, the number of Q buffers, the tensor memory used, and
-// the operand type. bf16 caches: a 6-slot ring of 16-bit chunks ([128 positions x 64 dims],
-// K and V) and the second Q buffer. FP8 caches: 4 V slots of 32 KB (a raw V box lands in a
-// slot's upper half and is converted in place into the slot's two f16 chunks; two V tiles
-// in flight) and 2 raw K boxes (converted K tiles go to tensor memory).
+// Per cache type. bf16 caches: a 6-slot ring of [128 positions x 64 dims] boxes (four per K
+// or V tile) and a second Q buffer in the rest of the ring area; S^T and each O^T half are
+// 64 columns (N = 64 heads). FP8 caches: a 10-slot ring of [128 positions x 128 dims] e4m3
+// boxes (two per K or V tile) and one Q buffer; S^T and each O^T half are 128 columns (the
+// hi parts of the 64 heads, then the lo parts), and P = 2^(s - m + kPExp).
 template <bool kFp8>
 struct Cfg {
-  static constexpr int kSlots = 6;  // bf16 ring: even, so a V half-tile's 2 chunks are adjacent
+  // bf16 ring: even, so a V half-tile's 2 chunks are adjacent
+  static constexpr int kSlots = kFp8 ? 10 : 6;
+  static constexpr int kTileBoxes = kFp8 ? 2 : 4;   // ring boxes per K (or V) tile
+  static constexpr int kBoxDims = kFp8 ? 128 : 64;  // head dims per box
+  static constexpr int kMmaK = kFp8 ? 32 : 16;      // K of one MMA instruction
   static constexpr uint32_t kTmemCols = kFp8 ? 512 : 256;
+  static constexpr uint32_t kSCols = kFp8 ? 128 : 64;  // S^T buffer, or O^T half, columns
+  static constexpr uint32_t kTmemO = 2 * kSCols;       // O^T halves follow the S^T buffers
   static constexpr int kQBufs = kFp8 ? 1 : 2;
-  static constexpr bool kBf16 = !kFp8;           // operands: bf16, or f16 for FP8 caches
-  static constexpr uint32_t kIdescS = idesc_f16(128, 64, kBf16, false, false);  // K x Q^T
-  static constexpr uint32_t kIdescPV = idesc_f16(128, 64, kBf16, true, true);   // V^T x P^T
+  static constexpr float kRescaleThreshold = kFp8 ? 4.0f : 8.0f;  // log2 units
+  static constexpr float kPExp = kFp8 ? 4.0f : 0.0f;  // P = 2^(s - m + kPExp)
+  // operand formats: bf16 (kind::f16), or e4m3 (kind::f8f6f4, whose format code is 0)
+  static constexpr uint32_t kIdescS = idesc_f16(128, kSCols, !kFp8, false, false);  // K x Q^T
+  static constexpr uint32_t kIdescPV = idesc_f16(128, kSCols, !kFp8, true, true);   // V^T x P^T
 };
-static_assert(kKRawOff + kKRawSlots * kRawBytes <= kRingBytes, "FP8 ring");
+static_assert(Cfg<true>::kSlots <= kMaxSlots && Cfg<false>::kSlots <= kMaxSlots, "ring");
+static_assert(Cfg<true>::kSlots * kChunkBytes <= kRingBytes, "FP8 ring");
+static_assert(2 * kQ8ChunkBytes == 4 * kQChunkBytes, "FP8 Q is converted in place");
 constexpr int kQ1Off = Cfg<false>::kSlots * kChunkBytes;  // bf16: the second Q buffer
 static_assert(kQ1Off + 4 * kQChunkBytes <= kRingBytes, "second Q buffer");
 
@@ -106,11 +113,8 @@ struct __align__(1024) TcSmem {
   float qmax[kSoftmaxWarps];
   uint64_t kv_full[kMaxSlots];
   uint64_t kv_empty[kMaxSlots];
-  uint64_t raw_full[kKRawSlots];   // FP8: raw K box landed
-  uint64_t raw_empty[kKRawSlots];  // FP8: raw K box converted
-  uint64_t vraw_full[kVSlots];     // FP8: raw V box landed in a V slot
-  uint64_t q_full[2], q_empty[2], q_ready;
-  uint64_t k_full[2];  // FP8: K tile converted into tensor memory buffer 0 / 1
+  uint64_t q_full[2], q_empty[2];
+  uint64_t q_ready;  // FP8: Q split into its e4m3 hi and lo parts
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, p_free;
   uint64_t o_free;
@@ -124,19 +128,12 @@ struct __align__(1024) TcSmem {
 // 227 KB a block may have
 static_assert(sizeof(TcSmem) + 1024 <= 232448, "shared memory per CTA");
 
-// bf16: ring chunk `slot`
+// ring box `slot`
 __device__ __forceinline__ uint8_t* ring_chunk(TcSmem& S, uint32_t slot) {
   return S.ring_area + slot * kChunkBytes;
 }
-// FP8: V slot `slot` (its f16 chunks at +0 and +16 KB; the raw box lands at +16 KB)
-__device__ __forceinline__ uint8_t* v_slot(TcSmem& S, uint32_t slot) {
-  return S.ring_area + slot * kVSlotBytes;
-}
-// FP8: raw K box slot
-__device__ __forceinline__ uint8_t* k_raw(TcSmem& S, uint32_t slot) {
-  return S.ring_area + kKRawOff + slot * kRawBytes;
-}
-// Q buffer qb: [4 chunks of 64 heads x 64 dims]
+// Q buffer qb: [4 boxes of 64 heads x 64 dims] bf16 as loaded (for FP8 caches then split in
+// place into 2 chunks of [128 rows x 128 dims] e4m3)
 __device__ __forceinline__ uint8_t* q_buf(TcSmem& S, int qb) {
   return qb == 0 ? S.q[0] : S.ring_area + kQ1Off;
 }
@@ -195,8 +192,6 @@ __device__ __forceinline__ float f16_hi(uint32_t w) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
 }
 
-// sixteen e4m3 codes (lowest byte first) -> sixteen f16 values in two 16-byte words, exact:
-// each 16-bit pair of codes becomes one f16x2 word (low byte -> low half)
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -255,8 +250,8 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   const int page_size = kPaged ? S.plan.page_size : 1;  // read only by the paged code
   const int page_shift = 31 - __clz(page_size);         // page sizes are powers of two
   const int box_rows = kPaged ? paged_box_rows(page_size) : kTile;
-  uint32_t chunk = 0, issued = 0;                 // bf16: ring chunks
-  uint32_t kb = 0, kb_issued = 0, vb = 0, vb_issued = 0;  // FP8: raw K and V boxes
+  constexpr int kC = C::kTileBoxes;
+  uint32_t chunk = 0, issued = 0;  // ring boxes
   int item = 0, q_issued = 0;
   if (leader) prefetch_tensormap(q_map);
   // every K/V byte is read once: keep it from evicting q and the split partials from L2
@@ -272,11 +267,10 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     prefetch_tensormap(&a.kv[it.b].tmap_k);
     prefetch_tensormap(&a.kv[it.b].tmap_v);
   }
-  // bf16: the boxes of one item in the order the MMA consumes them -- K(0), then K(t+1),
-  // V(t) for each t, then V(n-1) -- as four [128 positions x 64 dims] boxes per K or V tile,
-  // straight into the ring. FP8: per tile K(t) (two raw [128 x 128] e4m3 boxes into the K
-  // raw slots), then V(t) (two raw boxes into the upper halves of two V slots).
-  constexpr int kBoxesPerTile = kFp8 ? 4 : 8;
+  // The boxes of one item in the order the MMA consumes them -- K(0), then K(t+1), V(t) for
+  // each t, then V(n-1) -- as kC boxes of [128 positions x 128 bytes] per K or V tile,
+  // straight into the ring.
+  constexpr int kBoxesPerTile = 2 * kC;
   // Paged caches: the page ids of work item k, pages [p0, p_last] of its sequence (p_last =
   // the page of its last position), sit in S.page_ids[k & 1] (the first kPageIds of them; the
   // leader reads any further id straight from the table). Each lane fetches its share of the
@@ -326,56 +320,31 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   auto issue_box = [&](const WorkItem& w, int j) {
     const KvSeq* seq = a.kv + w.b;
     int y, a0, e0;
-    if constexpr (kFp8) {
-      const int t = j >> 2, r = j & 3;
-      tile_window(w, t, paged, y, a0, e0);
-      if (r < 2) {
-        const uint32_t slot = kb % kKRawSlots, use = kb / kKRawSlots;
-        if (use > 0) mbar_wait(&S.raw_empty[slot], (use - 1) & 1, abort);
-        const bool ok = !*abort;
-        if (leader && ok) mbar_arrive_expect_tx(&S.raw_full[slot], kRawBytes);
-        load_rows(k_raw(S, slot), &seq->tmap_k, 128 * r, w, y, &S.raw_full[slot],
-                  evict_first, ok);
-        if (ok) kb_issued = kb + 1;
-        ++kb;
-      } else {
-        const uint32_t slot = vb % kVSlots, use = vb / kVSlots;
-        if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);  // PV(t - 2) done
-        const bool ok = !*abort;
-        if (leader && ok) mbar_arrive_expect_tx(&S.vraw_full[slot], kRawBytes);
-        load_rows(v_slot(S, slot) + kChunkBytes, &seq->tmap_v, 128 * (r - 2), w, y,
-                  &S.vraw_full[slot], evict_first, ok);
-        if (ok) vb_issued = vb + 1;
-        ++vb;
-      }
+    const int n = num_tiles(w);
+    bool is_v;
+    int t, c;
+    if (j < kC) {
+      is_v = false, t = 0, c = j;
     } else {
-      const int n = num_tiles(w);
-      bool is_v;
-      int t, c;
-      if (j < 4) {
-        is_v = false, t = 0, c = j;
-      } else {
-        const int rr0 = j - 4, tt = rr0 / 8, rr = rr0 % 8;
-        if (tt < n - 1)
-          is_v = rr >= 4, t = is_v ? tt : tt + 1, c = is_v ? rr - 4 : rr;
-        else
-          is_v = true, t = n - 1, c = rr;
-      }
-      tile_window(w, t, paged, y, a0, e0);
-      const uint32_t slot = chunk % kN, use = chunk / kN;
-      if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);
-      const bool ok = !*abort;
-      if (leader && ok) mbar_arrive_expect_tx(&S.kv_full[slot], kChunkBytes);
-      load_rows(ring_chunk(S, slot), is_v ? &seq->tmap_v : &seq->tmap_k, 64 * c, w, y,
-                &S.kv_full[slot], evict_first, ok);
-      if (ok) issued = chunk + 1;
-      ++chunk;
+      const int rr0 = j - kC, tt = rr0 / (2 * kC), rr = rr0 % (2 * kC);
+      if (tt < n - 1)
+        is_v = rr >= kC, t = is_v ? tt : tt + 1, c = is_v ? rr - kC : rr;
+      else
+        is_v = true, t = n - 1, c = rr;
     }
+    tile_window(w, t, paged, y, a0, e0);
+    const uint32_t slot = chunk % kN, use = chunk / kN;
+    if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);
+    const bool ok = !*abort;
+    if (leader && ok) mbar_arrive_expect_tx(&S.kv_full[slot], kChunkBytes);
+    load_rows(ring_chunk(S, slot), is_v ? &seq->tmap_v : &seq->tmap_k, C::kBoxDims * c, w, y,
+              &S.kv_full[slot], evict_first, ok);
+    if (ok) issued = chunk + 1;
+    ++chunk;
   };
   // The K/V rows (and the split plan) were written by kernels that completed before this one
-  // launched, so the first boxes of the first item -- those that need no free slot: a
-  // ring-full for bf16, K(0) and V(0) for FP8 -- stream in while the previous kernel (which
-  // writes q) finishes.
+  // launched, so the first boxes of the first item -- a ring-full, which needs no free slot
+  // -- stream in while the previous kernel (which writes q) finishes.
   int first_done = 0;
   if constexpr (kPaged) {
     if (has) {
@@ -386,7 +355,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   }
   if (has) {
     const int total = kBoxesPerTile * num_tiles(it);
-    const int pre = kFp8 ? 4 : static_cast<int>(kN);
+    const int pre = static_cast<int>(kN);
     first_done = total < pre ? total : pre;
     for (int j = 0; j < first_done; ++j) issue_box(it, j);
   }
@@ -422,15 +391,8 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   }
   // Before the CTA may exit, every copy it started must have landed.
   if (*abort) {
-    if constexpr (kFp8) {
-      for (uint32_t c = (kb_issued > kKRawSlots ? kb_issued - kKRawSlots : 0); c < kb_issued; ++c)
-        mbar_wait_drain(&S.raw_full[c % kKRawSlots], (c / kKRawSlots) & 1);
-      for (uint32_t c = (vb_issued > kVSlots ? vb_issued - kVSlots : 0); c < vb_issued; ++c)
-        mbar_wait_drain(&S.vraw_full[c % kVSlots], (c / kVSlots) & 1);
-    } else {
-      for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
-        mbar_wait_drain(&S.kv_full[c % kN], (c / kN) & 1);
-    }
+    for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
+      mbar_wait_drain(&S.kv_full[c % kN], (c / kN) & 1);
     for (int i = (q_issued > C::kQBufs ? q_issued - C::kQBufs : 0); i < q_issued; ++i)
       mbar_wait_drain(&S.q_full[i % C::kQBufs], (i / C::kQBufs) & 1);
   }
@@ -443,6 +405,7 @@ template <bool kFp8, bool kPaged>
 __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool leader) {
   using C = Cfg<kFp8>;
   constexpr uint32_t kSlots = C::kSlots;
+  constexpr int kC = C::kTileBoxes;
   volatile int* abort = &S.abort_flag;
   const int lane = threadIdx.x & 31;
   constexpr bool paged = kPaged;
@@ -462,45 +425,42 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
     tc_fence_after();
     const uint32_t q_base = smem_u32(q_buf(S, qb));
 
+    // one MMA: kind::f16 (bf16) or kind::f8f6f4 (e4m3)
+    auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
+      if constexpr (kFp8)
+        umma_f8_ss(d, ad, bd, idesc, acc);
+      else
+        umma_f16_ss(d, ad, bd, idesc, acc);
+    };
+    // 128-byte rows: an MMA's K step is 32 bytes of a K-major row, or kMmaK rows (kMmaK / 8
+    // swizzle atoms of 1024 bytes) of an MN-major operand
+    constexpr int kStepsPerBox = 128 / (C::kMmaK * (kFp8 ? 1 : 2));  // 4
+    constexpr uint32_t kMnStep = C::kMmaK / 8 * 1024;
+    constexpr int kQStride = kFp8 ? kQ8ChunkBytes : kQChunkBytes;
+
     auto issue_s = [&](uint32_t tile) {
       const uint32_t j = tile & 1, k = tile >> 1;
       if (k > 0) mbar_wait(&S.s_free[j], (k - 1) & 1, abort);
       tc_fence_after();
-      const uint32_t d = tmem + kTmemS + 64 * j;
-      if constexpr (kFp8) {
-        // K(tile) in tensor memory buffer j (converted by the softmax warps)
-        mbar_wait(&S.k_full[j], k & 1, abort);
+      const uint32_t d = tmem + kTmemS + C::kSCols * j;
+      // K(tile): kC ring boxes, each used as soon as TMA has landed it
+      for (int c = 0; c < kC; ++c) {
+        const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
+        mbar_wait(&S.kv_full[slot], use & 1, abort);
         tc_fence_after();
-        if (!*abort) {
-          const uint32_t a_tm = tmem + kTmemK + 128 * j;
+        if (!*abort && leader) {
+          const uint32_t a_base = smem_u32(ring_chunk(S, slot));
 #pragma unroll
-          for (int kk = 0; kk < kHeadDim / 16; ++kk) {
-            const uint64_t bd =
-                sdesc_sw128(q_base + (kk >> 2) * kQChunkBytes + 32 * (kk & 3), 16, 1024);
-            if (leader) umma_f16_ts(d, a_tm + 8 * kk, bd, C::kIdescS, kk != 0);
+          for (int kk = 0; kk < kStepsPerBox; ++kk) {
+            const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
+            const uint64_t bd = sdesc_sw128(q_base + c * kQStride + 32 * kk, 16, 1024);
+            mma(d, ad, bd, C::kIdescS, (c | kk) != 0);
           }
-          if (leader) umma_commit(&S.s_full[j]);
+          umma_commit(&S.kv_empty[slot]);
         }
-      } else {
-        // K(tile): four ring chunks of 64 dims, each used as soon as TMA has landed it
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
-          mbar_wait(&S.kv_full[slot], use & 1, abort);
-          tc_fence_after();
-          if (!*abort && leader) {
-            const uint32_t a_base = smem_u32(ring_chunk(S, slot));
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
-              const uint64_t bd = sdesc_sw128(q_base + c * kQChunkBytes + 32 * kk, 16, 1024);
-              umma_f16_ss(d, ad, bd, C::kIdescS, (c | kk) != 0);
-            }
-            umma_commit(&S.kv_empty[slot]);
-          }
-          ++chunk;
-        }
-        if (!*abort && leader) umma_commit(&S.s_full[j]);
+        ++chunk;
       }
+      if (!*abort && leader) umma_commit(&S.s_full[j]);
     };
 
     auto issue_pv = [&](uint32_t tile, bool first, int keep) {
@@ -508,67 +468,43 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       if (first && item > 0) mbar_wait(&S.o_free, (item - 1) & 1, abort);
       tc_fence_after();
       const uint32_t p_base = smem_u32(S.p);
-      if constexpr (!kFp8) {
-        // bf16: each half of V^T (two chunks) is used as soon as TMA has landed it
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t c0 = chunk + 2 * h;
-          const uint32_t s0 = c0 % kSlots, s1 = (c0 + 1) % kSlots;
-          mbar_wait(&S.kv_full[s0], (c0 / kSlots) & 1, abort);
-          mbar_wait(&S.kv_full[s1], ((c0 + 1) / kSlots) & 1, abort);
-          tc_fence_after();
-          if (kPaged && keep < kTile && __shfl_sync(0xffffffffu, *abort, 0) == 0) {
-            // paged cache, the sequence's last window: V rows past its end may hold any
-            // bytes (NaN too) and meet a zero weight, so they are zeroed before PV (the
-            // whole warp runs this loop; the abort flag is read once for all its lanes)
-            zero_chunk_rows(ring_chunk(S, s0), keep, lane);
-            zero_chunk_rows(ring_chunk(S, s1), keep, lane);
-            fence_proxy_async_smem();
-            __syncwarp();
-          }
-          if (!*abort && leader) {
-            const uint32_t d = tmem + kTmemO + 64 * h;
-            const uint32_t a_base = smem_u32(ring_chunk(S, s0));
+      // each half of V^T (the 128 dims of one M=128 product: two bf16 boxes, or one FP8 box)
+      // is used as soon as TMA has landed it
+      constexpr int kPerHalf = kC / 2;
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t c0 = chunk + kPerHalf * h;
+        uint32_t sl[kPerHalf];
 #pragma unroll
-            for (int kt = 0; kt < kTile / 16; ++kt) {
-              const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
-              const uint64_t bd = sdesc_sw128(p_base + 2048 * kt, kPBytes, 1024);
-              umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
-            }
-            umma_commit(&S.kv_empty[s0]);
-            umma_commit(&S.kv_empty[s1]);
-          }
-        }
-        chunk += 4;
-        if (!*abort && leader) umma_commit(&S.p_free);
-      } else {
-        // FP8: V(t) sits in two V slots (one per half of the head dimension, two chunks
-        // each), converted in one step, so both are waited for first and the 16 MMAs issue
-        // back to back (a wait or commit between MMAs stalls the issue stream)
-        uint32_t slot[2];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          slot[h] = (chunk + h) % kVSlots;
-          mbar_wait(&S.kv_full[slot[h]], ((chunk + h) / kVSlots) & 1, abort);
+        for (int i = 0; i < kPerHalf; ++i) {
+          sl[i] = (c0 + i) % kSlots;
+          mbar_wait(&S.kv_full[sl[i]], ((c0 + i) / kSlots) & 1, abort);
         }
         tc_fence_after();
-        if (!*abort && leader) {
+        if (kPaged && keep < kTile && __shfl_sync(0xffffffffu, *abort, 0) == 0) {
+          // paged cache, the sequence's last window: V rows past its end may hold any
+          // bytes (NaN too) and meet a zero weight, so they are zeroed before PV (the
+          // whole warp runs this loop; the abort flag is read once for all its lanes)
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t d = tmem + kTmemO + 64 * h;
-            const uint32_t a_base = smem_u32(v_slot(S, slot[h]));
-#pragma unroll
-            for (int kt = 0; kt < kTile / 16; ++kt) {
-              const uint64_t ad = sdesc_sw128(a_base + 2048 * kt, kChunkBytes, 1024);
-              const uint64_t bd = sdesc_sw128(p_base + 2048 * kt, kPBytes, 1024);
-              umma_f16_ss(d, ad, bd, C::kIdescPV, !(first && kt == 0));
-            }
-          }
-          umma_commit(&S.kv_empty[slot[0]]);
-          umma_commit(&S.kv_empty[slot[1]]);
-          umma_commit(&S.p_free);
+          for (int i = 0; i < kPerHalf; ++i) zero_chunk_rows(ring_chunk(S, sl[i]), keep, lane);
+          fence_proxy_async_smem();
+          __syncwarp();
         }
-        chunk += 2;
+        if (!*abort && leader) {
+          const uint32_t d = tmem + C::kTmemO + C::kSCols * h;
+          const uint32_t a_base = smem_u32(ring_chunk(S, sl[0]));
+#pragma unroll
+          for (int kt = 0; kt < kTile / C::kMmaK; ++kt) {
+            // bf16: the half's two boxes are adjacent slots, kChunkBytes apart along M
+            const uint64_t ad = sdesc_sw128(a_base + kMnStep * kt, kChunkBytes, 1024);
+            const uint64_t bd = sdesc_sw128(p_base + kMnStep * kt, kPBytes, 1024);
+            mma(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+          }
+#pragma unroll
+          for (int i = 0; i < kPerHalf; ++i) umma_commit(&S.kv_empty[sl[i]]);
+        }
       }
+      chunk += kC;
+      if (!*abort && leader) umma_commit(&S.p_free);
     };
 
     for (int t = 0; t < n; ++t) {
@@ -586,99 +522,62 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
 }
 
 // ---------------------------------------------------------------------------------------
-// FP8 conversions, run by the eight softmax warps (256 threads, st = 0..255)
+// FP8 caches: e4m3 pairs, and the split of Q (run by the eight softmax warps)
 // ---------------------------------------------------------------------------------------
 
-// K(t) of an FP8 cache -> tensor memory buffer `buf` as the A operand of S^T = K . Q^T:
-// lane = position, 64 columns of f16 pairs per half of the 256 dims. Softmax group g
-// converts raw box `rbox + g` (dims 128 g .. 128 g + 127); thread = its TMEM lane = row of
-// the box. Each row is read as eight 16-byte pieces (128-byte swizzle: piece j of row r sits
-// at 16 (j ^ (r mod 8)), so the eight rows of a quarter warp hit distinct banks).
-__device__ void convert_k_tmem(TcSmem& S, uint32_t rbox, uint32_t tmem, uint32_t buf, int group,
-                               int row, uint32_t lane_addr, int lane, volatile int* abort) {
-  const uint32_t b = rbox + group, rslot = b % kKRawSlots;
-  mbar_wait(&S.raw_full[rslot], (b / kKRawSlots) & 1, abort);
-  const uint8_t* raw = k_raw(S, rslot) + row * 128;
-  const uint32_t dst = tmem + lane_addr + kTmemK + 128 * buf + 64 * group;
-  const int sw = row & 7;
-  uint4 v[8];  // all loads first: each tensor-memory store is a compiler barrier
-#pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(raw + ((j ^ sw) << 4));
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    uint4 o0, o1;
-    e4m3x16_to_f16x16(v[j], o0, o1);
-    tmem_st_32x32b_x8(dst + 8 * j, o0, o1);
-  }
-  tmem_wait_st();
-  tc_fence_before();
-  __syncwarp();
-  if (lane == 0) {
-    mbar_arrive_cnt(&S.raw_empty[rslot], 2);  // four warps per box, eight arrivals expected
-    mbar_arrive(&S.k_full[buf]);
-  }
+// f16x2 -> two e4m3 codes (round to nearest even, saturating at 448), low half -> low byte
+__device__ __forceinline__ uint16_t f16x2_to_e4m3x2(uint32_t v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(v));
+  return r;
 }
 
-// V(t) of an FP8 cache, in place: its two raw boxes (e4m3, [128 positions x 128 dims],
-// 128-byte swizzle) sit in the upper halves of V slots vbox and vbox + 1 (mod 4); box b
-// becomes the two f16 chunks ([128 positions x 64 dims], same swizzle) of its slot. Every
-// thread first loads all eight of its 16-byte pieces (16 codes of one position each), then
-// the eight warps synchronize, and only then is any slot overwritten: a thread's output
-// covers other threads' input. One proxy fence covers the whole tile.
-__device__ void convert_v_inplace(TcSmem& S, uint32_t vbox, int st, int lane, int keep,
-                                  volatile int* abort) {
-  uint32_t slot[2];
-#pragma unroll
-  for (int bx = 0; bx < 2; ++bx) {
-    slot[bx] = (vbox + bx) % kVSlots;
-    mbar_wait(&S.vraw_full[slot[bx]], ((vbox + bx) / kVSlots) & 1, abort);
-  }
-  uint4 v[2][2][2];
-#pragma unroll
-  for (int bx = 0; bx < 2; ++bx)
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int pc = st + 256 * i, r = pc >> 2, j = 4 * cc + (pc & 3);
-        v[bx][cc][i] = *reinterpret_cast<const uint4*>(v_slot(S, slot[bx]) + kChunkBytes +
-                                                       r * 128 + ((j ^ (r & 7)) << 4));
-      }
-  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);
-#pragma unroll
-  for (int bx = 0; bx < 2; ++bx)
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      uint8_t* dst = v_slot(S, slot[bx]) + cc * kChunkBytes;
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int pc = st + 256 * i, r = pc >> 2, jj = pc & 3, sw = r & 7;
-        uint4 o0, o1;
-        e4m3x16_to_f16x16(v[bx][cc][i], o0, o1);
-        if (r >= keep) o0 = o1 = make_uint4(0u, 0u, 0u, 0u);  // paged: past the sequence
-        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj) ^ sw) << 4)) = o0;
-        *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * jj + 1) ^ sw) << 4)) = o1;
-      }
-    }
-  fence_proxy_async_smem();
-  __syncwarp();
-  if (lane == 0) {
-    mbar_arrive(&S.kv_full[slot[0]]);
-    mbar_arrive(&S.kv_full[slot[1]]);
-  }
+// two e4m3 codes -> f16x2 (exact)
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
 }
 
-// Q of the current item (bf16, loaded by TMA) -> f16 in place, scaled by 2^-e where e >= 0
-// is the smallest exponent that keeps every |q| below 2^15. Returns e.
-__device__ int convert_q(TcSmem& S, int item, int st, int swarp, int lane, volatile int* abort) {
+__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// A pair of values (f16x2, |v| <= 256) as e4m3 hi and lo parts: hi = e4m3(v), lo =
+// e4m3(v - hi); returns hi + lo (f16x2, exact: both parts and their sum fit f16).
+__device__ __forceinline__ uint32_t split_e4m3x2(uint32_t v, uint16_t& hi, uint16_t& lo) {
+  hi = f16x2_to_e4m3x2(v);
+  const uint32_t hf = e4m3x2_to_f16x2(hi);
+  lo = f16x2_to_e4m3x2(hsub2_u32(v, hf));
+  return hadd2_u32(hf, e4m3x2_to_f16x2(lo));
+}
+
+// Q of the current item (bf16, four TMA boxes of [64 heads x 64 dims]) -> in place, two
+// chunks of [128 rows x 128 dims] e4m3 (row h: the hi part of head h; row 64 + h: its lo
+// part; 128-byte swizzle), scaled by 2^-e with e chosen so that the largest |q| maps into
+// [128, 256). Returns e. Thread st takes head st / 4 and dims [64 (st % 4), +64): the eight
+// 16-byte pieces of one raw box row in, four pieces of the hi row and four of the lo row out.
+// Every thread has read its input before any thread writes: outputs overlap inputs.
+// (Not inlined: runs once per work item, and inlined it pushed the softmax loop to spill.)
+__device__ __noinline__ int convert_q8(TcSmem& S, int item, int st, int swarp, int lane, volatile int* abort) {
   mbar_wait(&S.q_full[0], item & 1, abort);
-  uint4* q = reinterpret_cast<uint4*>(S.q[0]);
-  constexpr int kPieces = kHeads * kHeadDim / 8 / (32 * kSoftmaxWarps);  // 8 per thread
+  const int h = st >> 2, qd = st & 3;
+  const uint8_t* src = S.q[qd] + h * 128;
+  uint4 v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (h & 7)) << 4));
   float mx = 0.f;
 #pragma unroll
-  for (int i = 0; i < kPieces; ++i) {
-    const uint4 v = q[st + 256 * i];
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[k] << 16)),
@@ -686,22 +585,38 @@ __device__ int convert_q(TcSmem& S, int item, int st, int swarp, int lane, volat
   }
   mx = warp_max_f32(mx);
   if (lane == 0) S.qmax[swarp] = mx;
-  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);
+  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);  // also: every raw row has been read
   float m = 0.f;
 #pragma unroll
   for (int w = 0; w < kSoftmaxWarps; ++w) m = fmaxf(m, S.qmax[w]);
-  const int e = (m >= 32768.f && m <= 3.0e38f) ? ilogbf(m) - 14 : 0;
+  // m * 2^-e in [128, 256); bf16 values times a power of two in [2^-24, 256] are exact in f16
+  const int e = (m > 0.f && m <= 3.0e38f) ? ilogbf(m) - 7 : 0;
   const float sc = ldexpf(1.f, -e);
+  uint32_t hi[16], lo[16];  // 64 codes each, four per word
 #pragma unroll
-  for (int i = 0; i < kPieces; ++i) {
-    uint4& ref = q[st + 256 * i];
-    const uint4 v = ref;
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-    uint32_t o[4];
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      o[k] = pack_f16x2(__uint_as_float(w[k] << 16) * sc, __uint_as_float(w[k] & 0xFFFF0000u) * sc);
-    ref = make_uint4(o[0], o[1], o[2], o[3]);
+    for (int k = 0; k < 4; k += 2) {
+      uint16_t h0, l0, h1, l1;
+      split_e4m3x2(pack_f16x2(__uint_as_float(w[k] << 16) * sc,
+                              __uint_as_float(w[k] & 0xFFFF0000u) * sc), h0, l0);
+      split_e4m3x2(pack_f16x2(__uint_as_float(w[k + 1] << 16) * sc,
+                              __uint_as_float(w[k + 1] & 0xFFFF0000u) * sc), h1, l1);
+      hi[2 * j + k / 2] = static_cast<uint32_t>(h0) | (static_cast<uint32_t>(h1) << 16);
+      lo[2 * j + k / 2] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
+    }
+  }
+  uint8_t* chunk = S.q[0] + (qd >> 1) * kQ8ChunkBytes;
+  const int piece0 = 4 * (qd & 1);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int pj = piece0 + j;
+    *reinterpret_cast<uint4*>(chunk + h * 128 + ((pj ^ (h & 7)) << 4)) =
+        make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
+    const int r = 64 + h;
+    *reinterpret_cast<uint4*>(chunk + r * 128 + ((pj ^ (r & 7)) << 4)) =
+        make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
   }
   fence_proxy_async_smem();
   named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);  // qmax is read before it is reused
@@ -726,11 +641,11 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
   const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
   const int row = quad * 32 + lane;          // tile position / O^T row of this thread
   const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
+  using C = Cfg<kFp8>;
   const float s_mul0 = a.scale * kLog2e * (kFp8 ? a.k_scale : 1.f);
   const float v_mul = kFp8 ? a.v_scale : 1.f;
   constexpr bool paged = kPaged;
   uint32_t gt = 0;
-  uint32_t kbox = 0, vbox = 0;  // FP8: raw K and V boxes converted so far
   int item = 0;
   uint8_t* const p_row = S.p + row * 128;
 
@@ -738,54 +653,45 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     const int n = num_tiles(it);
     float lsum_w = 0.f;  // this warp's running row sum of head h0 + lane
     float s_mul = s_mul0;
-    // FP8: a V tile is two raw boxes -> converted in place in two V slots; a K tile is two
-    // raw boxes -> tensor memory buffer (tile mod 2). Tensor memory buffer j was last read by
-    // S(tile - 2), whose completion this warp has already waited for.
-    auto convert_v = [&](int keep) {
-      convert_v_inplace(S, vbox, st, lane, keep, abort);
-      vbox += 2;
-    };
-    auto convert_k = [&](uint32_t tile) {
-      convert_k_tmem(S, kbox, tmem, tile & 1, group, row, lane_addr, lane, abort);
-      kbox += 2;
-    };
-    if constexpr (kFp8) {
-      s_mul = s_mul0 * ldexpf(1.f, convert_q(S, item, st, swarp, lane, abort));
-      convert_k(gt);  // K(0)
-    }
+    // FP8: Q split into e4m3 hi and lo parts scaled by 2^-e, so the scores carry 2^e
+    if constexpr (kFp8) s_mul = s_mul0 * ldexpf(1.f, convert_q8(S, item, st, swarp, lane, abort));
 
-    // FP8 order within a tile: K(t + 1), V(t), then the softmax of t. V(t)'s slots were last
-    // read by PV(t - 2), so neither conversion waits for the tensor core's current work, and
-    // PV(t) can issue as soon as P(t) is stored.
     for (int t = 0; t < n; ++t) {
       int y, a0, e0;
       tile_window(it, t, paged, y, a0, e0);
-      if constexpr (kFp8) {
-        if (t + 1 < n) convert_k(gt + t + 1);      // consumed by S(t + 1)
-        convert_v(window_rows_kept(paged, y, e0));  // V(t), consumed by PV(t)
-      }
       const uint32_t tile = gt + t, j = tile & 1, k = tile >> 1;
       const int pos = y + row;
       const bool valid = pos >= a0 && pos < e0;
 
       mbar_wait(&S.s_full[j], k & 1, abort);
       tc_fence_after();
-      uint32_t sr[kGroupHeads];
-      tmem_ld_32x32b_x32(tmem + lane_addr + kTmemS + 64 * j + h0, sr);
-      tmem_wait_ld();
+      float s[kGroupHeads];
+      {
+        const uint32_t sa = tmem + lane_addr + kTmemS + C::kSCols * j + h0;
+        uint32_t sr[kGroupHeads];
+        tmem_ld_32x32b_x32(sa, sr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < kGroupHeads; ++h) s[h] = __uint_as_float(sr[h]);
+        if constexpr (kFp8) {  // plus the lo parts' scores, 64 columns on
+          tmem_ld_32x32b_x32(sa + 64, sr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < kGroupHeads; ++h) s[h] += __uint_as_float(sr[h]);
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.s_free[j]);
 
-      float s[kGroupHeads];
 #pragma unroll
-      for (int h = 0; h < kGroupHeads; ++h)
-        s[h] = valid ? __uint_as_float(sr[h]) * s_mul : -INFINITY;
+      for (int h = 0; h < kGroupHeads; ++h) s[h] = valid ? s[h] * s_mul : -INFINITY;
 
       bool need = (t == 0);
       if (!need) {
 #pragma unroll
-        for (int h = 0; h < kGroupHeads; ++h) need |= s[h] > S.m_used[h0 + h] + kRescaleThreshold;
+        for (int h = 0; h < kGroupHeads; ++h)
+          need |= s[h] > S.m_used[h0 + h] + C::kRescaleThreshold;
       }
       if (named_bar_or(gbar, kGroupThreads, need)) {
         // exact per-head max of this tile across the 128 positions
@@ -809,10 +715,12 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
           // O must hold PV(t-1) before it is rescaled
           mbar_wait(&S.p_free, (tile - 1) & 1, abort);
           tc_fence_after();
+          // each O^T half (FP8: its hi and its lo columns)
 #pragma unroll 1
-          for (int hf = 0; hf < 2; ++hf) {
+          for (int hp = 0; hp < (kFp8 ? 4 : 2); ++hp) {
             uint32_t o[kGroupHeads];
-            const uint32_t addr = tmem + lane_addr + kTmemO + 64 * hf + h0;
+            const uint32_t addr =
+                tmem + lane_addr + C::kTmemO + C::kSCols * (hp & 1) + 64 * (hp >> 1) + h0;
             tmem_ld_32x32b_x32(addr, o);
             tmem_wait_ld();
 #pragma unroll
@@ -824,17 +732,24 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
         }
       }
 
-      // probabilities (rounded to the operand type the tensor core reads: bf16, or f16
-      // for FP8 caches), this group's half of the P^T row, and the row sums of the rounded
+      // probabilities, rounded to what the tensor core reads (bf16; for FP8 caches e4m3 hi
+      // and lo parts), this group's share of the P^T row, and the row sums of the rounded
       // values
-      uint32_t pk[kGroupHeads / 2];
+      uint32_t pk[kGroupHeads / 2];  // bf16: 32 values; FP8: 32 hi codes, then 32 lo codes
 #pragma unroll
       for (int h = 0; h < kGroupHeads; h += 2) {
-        const float p0 = ex2(s[h] - S.m_used[h0 + h]);
-        const float p1 = ex2(s[h + 1] - S.m_used[h0 + h + 1]);
+        const float p0 = ex2(s[h] - (S.m_used[h0 + h] - C::kPExp));
+        const float p1 = ex2(s[h + 1] - (S.m_used[h0 + h + 1] - C::kPExp));
         if constexpr (kFp8) {
-          const uint32_t w = pack_f16x2(p0, p1);
-          pk[h / 2] = w;
+          uint16_t hi, lo;
+          const uint32_t w = split_e4m3x2(pack_f16x2(p0, p1), hi, lo);
+          if ((h & 2) == 0) {
+            pk[h / 4] = hi;
+            pk[8 + h / 4] = lo;
+          } else {
+            pk[h / 4] |= static_cast<uint32_t>(hi) << 16;
+            pk[8 + h / 4] |= static_cast<uint32_t>(lo) << 16;
+          }
           s[h] = f16_lo(w);
           s[h + 1] = f16_hi(w);
         } else {
@@ -849,7 +764,9 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       if (tile >= 1) mbar_wait(&S.p_free, (tile - 1) & 1, abort);
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const int cl = 4 * group + c;  // logical 16-byte chunk of the 128-byte row
+        // logical 16-byte piece of the 128-byte row: bf16, heads 8 c' .. 8 c' + 7 in piece c';
+        // FP8, hi codes of heads 16 c' .. in piece c' < 4, lo codes in piece 4 + c'
+        const int cl = kFp8 ? (c < 2 ? 2 * group + c : 4 + 2 * group + (c - 2)) : 4 * group + c;
         uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         *reinterpret_cast<uint4*>(p_row + ((cl ^ (row & 7)) << 4)) = v;
       }
@@ -877,8 +794,17 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
 #pragma unroll 1
     for (int hf = 0; hf < 2; ++hf) {
       uint32_t o[kGroupHeads];
-      tmem_ld_32x32b_x32(tmem + lane_addr + kTmemO + 64 * hf + h0, o);
+      const uint32_t oa = tmem + lane_addr + C::kTmemO + C::kSCols * hf + h0;
+      tmem_ld_32x32b_x32(oa, o);
       tmem_wait_ld();
+      if constexpr (kFp8) {  // O = (V . P_hi) + (V . P_lo)
+        uint32_t ol[kGroupHeads];
+        tmem_ld_32x32b_x32(oa + 64, ol);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < kGroupHeads; ++h)
+          o[h] = __float_as_uint(__uint_as_float(o[h]) + __uint_as_float(ol[h]));
+      }
       const int d = hf * 128 + row;
       if (ok) {
         if (it.slot < 0) {
@@ -917,20 +843,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < Cfg<kFp8>::kSlots; ++i) {
-      mbar_init(&S.kv_full[i], kFp8 ? kSoftmaxWarps : 1);  // FP8: the converting warps arrive
+      mbar_init(&S.kv_full[i], 1);
       mbar_init(&S.kv_empty[i], 1);
     }
-    for (int i = 0; i < kKRawSlots; ++i) {
-      mbar_init(&S.raw_full[i], 1);
-      mbar_init(&S.raw_empty[i], kSoftmaxWarps);
-    }
-    for (int i = 0; i < kVSlots; ++i) mbar_init(&S.vraw_full[i], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
     }
     mbar_init(&S.q_ready, kSoftmaxWarps);
-    for (int i = 0; i < 2; ++i) mbar_init(&S.k_full[i], kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
       mbar_init(&S.s_free[i], kSoftmaxWarps);
