@@ -56,10 +56,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 320;
-constexpr int kSoftmaxWarps = 8;        // warps 2..9
 constexpr int kGroupThreads = 128;      // one softmax group = four warps = the 128 lanes
-constexpr int kGroupHeads = 32;         // heads per group
+constexpr int kMaxSoftmaxWarps = 16;
 // a ring box: [128 positions x 128 bytes] (64 bf16 dims, or 128 e4m3 dims), 128-byte swizzle
 constexpr int kChunkBytes = 16384;
 constexpr int kRingBytes = 10 * kChunkBytes;
@@ -70,25 +68,34 @@ constexpr int kPBytes = 16384;          // P^T: [128 positions x 128 bytes]
 constexpr uint32_t kTmemS = 0;          // S^T buffers from column 0 (see Cfg::kSCols)
 constexpr int kPageIds = 128;          // paged caches: page ids held per work item
 constexpr float kLog2e = 1.4426950408889634f;
-// named barriers: 1 + group among one softmax group, 3 among all eight softmax warps
-constexpr uint32_t kBarAllSoftmax = 3;
+// named barriers: 1 + group among one softmax group, Cfg::kBarAll among all softmax warps
 
 // Per cache type. bf16 caches: a 6-slot ring of [128 positions x 64 dims] boxes (four per K
-// or V tile) and a second Q buffer in the rest of the ring area; S^T and each O^T half are
-// 64 columns (N = 64 heads). FP8 caches: a 10-slot ring of [128 positions x 128 dims] e4m3
-// boxes (two per K or V tile) and one Q buffer; S^T and each O^T half are 128 columns (the
-// hi parts of the 64 heads, then the lo parts), and P = 2^(s - m + kPExp).
+// or V tile); S^T and each O^T half are 64 columns (N = 64 heads). FP8 caches: an 8-slot
+// ring of [128 positions x 128 dims] e4m3 boxes (two per K or V tile); S^T and each O^T half
+// are 128 columns (the hi parts of the 64 heads, then the lo parts), and P =
+// 2^(s - m + kPExp). Both: a second Q buffer in the rest of the ring area, and two softmax
+// groups of 32 heads (four groups of 16 heads were measured slower for FP8: the extra warps
+// slowed the MMA warp's issue more than they sped up the softmax). A softmax group is four
+// warps, one per tensor-memory lane quadrant, so that together they hold the 128 positions
+// of a tile.
 template <bool kFp8>
 struct Cfg {
+  static constexpr int kGroups = 2;
+  static constexpr int kSoftmaxWarps = 4 * kGroups;     // warps 2 .. 2 + kSoftmaxWarps - 1
+  static constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
+  static constexpr int kGroupHeads = kHeads / kGroups;  // heads per group
+  static constexpr uint32_t kBarAll = 1 + kGroups;      // named barrier of all softmax warps
   // bf16 ring: even, so a V half-tile's 2 chunks are adjacent
-  static constexpr int kSlots = kFp8 ? 10 : 6;
+  static constexpr int kSlots = kFp8 ? 8 : 6;
   static constexpr int kTileBoxes = kFp8 ? 2 : 4;   // ring boxes per K (or V) tile
   static constexpr int kBoxDims = kFp8 ? 128 : 64;  // head dims per box
   static constexpr int kMmaK = kFp8 ? 32 : 16;      // K of one MMA instruction
   static constexpr uint32_t kTmemCols = kFp8 ? 512 : 256;
   static constexpr uint32_t kSCols = kFp8 ? 128 : 64;  // S^T buffer, or O^T half, columns
   static constexpr uint32_t kTmemO = 2 * kSCols;       // O^T halves follow the S^T buffers
-  static constexpr int kQBufs = kFp8 ? 1 : 2;
+  static constexpr int kQBufs = 2;
+  static constexpr int kQ1Off = kSlots * kChunkBytes;  // the second Q buffer in the ring area
   static constexpr float kRescaleThreshold = kFp8 ? 4.0f : 8.0f;  // log2 units
   static constexpr float kPExp = kFp8 ? 4.0f : 0.0f;  // P = 2^(s - m + kPExp)
   // operand formats: bf16 (kind::f16), or e4m3 (kind::f8f6f4, whose format code is 0)
@@ -96,10 +103,13 @@ struct Cfg {
   static constexpr uint32_t kIdescPV = idesc_f16(128, kSCols, !kFp8, true, true);   // V^T x P^T
 };
 static_assert(Cfg<true>::kSlots <= kMaxSlots && Cfg<false>::kSlots <= kMaxSlots, "ring");
-static_assert(Cfg<true>::kSlots * kChunkBytes <= kRingBytes, "FP8 ring");
 static_assert(2 * kQ8ChunkBytes == 4 * kQChunkBytes, "FP8 Q is converted in place");
-constexpr int kQ1Off = Cfg<false>::kSlots * kChunkBytes;  // bf16: the second Q buffer
-static_assert(kQ1Off + 4 * kQChunkBytes <= kRingBytes, "second Q buffer");
+static_assert(Cfg<true>::kSoftmaxWarps <= kMaxSoftmaxWarps &&
+                  Cfg<false>::kSoftmaxWarps <= kMaxSoftmaxWarps,
+              "softmax warps");
+static_assert(Cfg<true>::kBarAll < 16 && Cfg<false>::kBarAll < 16, "named barrier ids");
+static_assert(Cfg<false>::kQ1Off + 4 * kQChunkBytes <= kRingBytes, "second Q buffer (bf16)");
+static_assert(Cfg<true>::kQ1Off + 4 * kQChunkBytes <= kRingBytes, "second Q buffer (FP8)");
 
 struct __align__(1024) TcSmem {
   uint8_t ring_area[kRingBytes];
@@ -110,7 +120,7 @@ struct __align__(1024) TcSmem {
   float alpha[kHeads];
   float red[4][kHeads];
   float lsum[kHeads];
-  float qmax[kSoftmaxWarps];
+  float qmax[kMaxSoftmaxWarps];
   uint64_t kv_full[kMaxSlots];
   uint64_t kv_empty[kMaxSlots];
   uint64_t q_full[2], q_empty[2];
@@ -134,8 +144,9 @@ __device__ __forceinline__ uint8_t* ring_chunk(TcSmem& S, uint32_t slot) {
 }
 // Q buffer qb: [4 boxes of 64 heads x 64 dims] bf16 as loaded (for FP8 caches then split in
 // place into 2 chunks of [128 rows x 128 dims] e4m3)
+template <bool kFp8>
 __device__ __forceinline__ uint8_t* q_buf(TcSmem& S, int qb) {
-  return qb == 0 ? S.q[0] : S.ring_area + kQ1Off;
+  return qb == 0 ? S.q[0] : S.ring_area + Cfg<kFp8>::kQ1Off;
 }
 
 __device__ __forceinline__ int num_tiles(const WorkItem& it) {
@@ -198,42 +209,47 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Sum 32 per-lane values over the 32 lanes of the warp: afterwards lane l holds the sum of
-// entry l in v[0]. Each step exchanges half of the live entries with the partner lane (bit
-// 4, 3, 2, 1, 0 of the lane id) and keeps the half it owns.
-__device__ __forceinline__ float warp_transpose_sum32(float (&v)[32], int lane) {
+// Sum N (32 or 16) per-lane values over the 32 lanes of the warp. Each step exchanges half
+// of the live entries with the partner lane (bit 4, 3, ... of the lane id) and keeps the
+// half it owns; once one entry is left, the remaining steps are plain sums. Afterwards lane
+// l holds the sum of entry l (N = 32) or of entry l / 2 (N = 16, lanes l and l ^ 1 alike).
+template <int N>
+__device__ __forceinline__ float warp_transpose_sum(float (&v)[N], int lane) {
+  static_assert(N == 32 || N == 16, "entries");
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const bool up = lane & 16;
-    const float send = up ? v[i] : v[i + 16];
-    const float keep = up ? v[i + 16] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-  }
+  for (int step = 0; step < 5; ++step) {
+    const int bit = 16 >> step;
+    const int live = N >> step;  // entries still live before this step (>= 1)
+    if (live >= 2) {
+      const int half = live / 2;
+      const bool up = lane & bit;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const bool up = lane & 8;
-    const float send = up ? v[i] : v[i + 8];
-    const float keep = up ? v[i + 8] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      for (int i = 0; i < half; ++i) {
+        const float send = up ? v[i] : v[i + half];
+        const float keep = up ? v[i + half] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+      }
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], bit);
+    }
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const bool up = lane & 4;
-    const float send = up ? v[i] : v[i + 4];
-    const float keep = up ? v[i + 4] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-  }
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const bool up = lane & 2;
-    const float send = up ? v[i] : v[i + 2];
-    const float keep = up ? v[i + 2] : v[i];
-    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-  }
-  const bool up = lane & 1;
-  const float send = up ? v[0] : v[1];
-  const float keep = up ? v[1] : v[0];
-  return keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  return v[0];
+}
+
+// tensor memory: N = 32 or 16 consecutive columns of this warp's 32 lanes
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+  if constexpr (N == 32)
+    tmem_ld_32x32b_x32(taddr, r);
+  else
+    tmem_ld_32x32b_x16(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&r)[N]) {
+  if constexpr (N == 32)
+    tmem_st_32x32b_x32(taddr, r);
+  else
+    tmem_st_32x32b_x16(taddr, r);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -376,7 +392,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     if (!*abort) {
       if (leader) {
         mbar_arrive_expect_tx(&S.q_full[qb], 4 * kQChunkBytes);
-        uint8_t* qd = q_buf(S, qb);
+        uint8_t* qd = q_buf<kFp8>(S, qb);
         for (int c = 0; c < 4; ++c)
           tma_load_2d(qd + c * kQChunkBytes, q_map, 64 * c, it.b * kHeads, &S.q_full[qb]);
       }
@@ -421,9 +437,10 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       return window_rows_kept(paged, y, e0);
     };
     const int qb = item % C::kQBufs, qu = item / C::kQBufs;
-    mbar_wait(kFp8 ? &S.q_ready : &S.q_full[qb], qu & 1, abort);
+    // FP8: q_ready completes once per item (the split of its Q)
+    mbar_wait(kFp8 ? &S.q_ready : &S.q_full[qb], (kFp8 ? item : qu) & 1, abort);
     tc_fence_after();
-    const uint32_t q_base = smem_u32(q_buf(S, qb));
+    const uint32_t q_base = smem_u32(q_buf<kFp8>(S, qb));
 
     // one MMA: kind::f16 (bf16) or kind::f8f6f4 (e4m3)
     auto mma = [&](uint32_t d, uint64_t ad, uint64_t bd, uint32_t idesc, uint32_t acc) {
@@ -443,24 +460,50 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       if (k > 0) mbar_wait(&S.s_free[j], (k - 1) & 1, abort);
       tc_fence_after();
       const uint32_t d = tmem + kTmemS + C::kSCols * j;
-      // K(tile): kC ring boxes, each used as soon as TMA has landed it
-      for (int c = 0; c < kC; ++c) {
-        const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
-        mbar_wait(&S.kv_full[slot], use & 1, abort);
+      if constexpr (kFp8) {
+        // K(tile): both boxes, then the 8 MMAs back to back. FP8 tiles are consumed slower
+        // than they stream, so the ring runs ahead and the boxes have landed; a wait or a
+        // commit between MMAs would stall the issue stream.
+        const uint32_t s0 = chunk % kSlots, s1 = (chunk + 1) % kSlots;
+        mbar_wait(&S.kv_full[s0], (chunk / kSlots) & 1, abort);
+        mbar_wait(&S.kv_full[s1], ((chunk + 1) / kSlots) & 1, abort);
         tc_fence_after();
         if (!*abort && leader) {
-          const uint32_t a_base = smem_u32(ring_chunk(S, slot));
 #pragma unroll
-          for (int kk = 0; kk < kStepsPerBox; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
-            const uint64_t bd = sdesc_sw128(q_base + c * kQStride + 32 * kk, 16, 1024);
-            mma(d, ad, bd, C::kIdescS, (c | kk) != 0);
+          for (int c = 0; c < 2; ++c) {
+            const uint32_t a_base = smem_u32(ring_chunk(S, c == 0 ? s0 : s1));
+#pragma unroll
+            for (int kk = 0; kk < kStepsPerBox; ++kk) {
+              const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
+              const uint64_t bd = sdesc_sw128(q_base + c * kQStride + 32 * kk, 16, 1024);
+              mma(d, ad, bd, C::kIdescS, (c | kk) != 0);
+            }
           }
-          umma_commit(&S.kv_empty[slot]);
+          umma_commit(&S.kv_empty[s0]);
+          umma_commit(&S.kv_empty[s1]);
+          umma_commit(&S.s_full[j]);
         }
-        ++chunk;
+        chunk += 2;
+      } else {
+        // K(tile): kC ring boxes, each used as soon as TMA has landed it
+        for (int c = 0; c < kC; ++c) {
+          const uint32_t slot = chunk % kSlots, use = chunk / kSlots;
+          mbar_wait(&S.kv_full[slot], use & 1, abort);
+          tc_fence_after();
+          if (!*abort && leader) {
+            const uint32_t a_base = smem_u32(ring_chunk(S, slot));
+#pragma unroll
+            for (int kk = 0; kk < kStepsPerBox; ++kk) {
+              const uint64_t ad = sdesc_sw128(a_base + 32 * kk, 16, 1024);
+              const uint64_t bd = sdesc_sw128(q_base + c * kQStride + 32 * kk, 16, 1024);
+              mma(d, ad, bd, C::kIdescS, (c | kk) != 0);
+            }
+            umma_commit(&S.kv_empty[slot]);
+          }
+          ++chunk;
+        }
+        if (!*abort && leader) umma_commit(&S.s_full[j]);
       }
-      if (!*abort && leader) umma_commit(&S.s_full[j]);
     };
 
     auto issue_pv = [&](uint32_t tile, bool first, int keep) {
@@ -468,43 +511,77 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       if (first && item > 0) mbar_wait(&S.o_free, (item - 1) & 1, abort);
       tc_fence_after();
       const uint32_t p_base = smem_u32(S.p);
-      // each half of V^T (the 128 dims of one M=128 product: two bf16 boxes, or one FP8 box)
-      // is used as soon as TMA has landed it
-      constexpr int kPerHalf = kC / 2;
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t c0 = chunk + kPerHalf * h;
-        uint32_t sl[kPerHalf];
-#pragma unroll
-        for (int i = 0; i < kPerHalf; ++i) {
-          sl[i] = (c0 + i) % kSlots;
-          mbar_wait(&S.kv_full[sl[i]], ((c0 + i) / kSlots) & 1, abort);
-        }
+      if constexpr (kFp8) {
+        // V(tile): both boxes (one per half of V^T: 128 dims, one M=128 product each), then
+        // the 8 MMAs back to back, as for S
+        const uint32_t s0 = chunk % kSlots, s1 = (chunk + 1) % kSlots;
+        mbar_wait(&S.kv_full[s0], (chunk / kSlots) & 1, abort);
+        mbar_wait(&S.kv_full[s1], ((chunk + 1) / kSlots) & 1, abort);
         tc_fence_after();
         if (kPaged && keep < kTile && __shfl_sync(0xffffffffu, *abort, 0) == 0) {
-          // paged cache, the sequence's last window: V rows past its end may hold any
-          // bytes (NaN too) and meet a zero weight, so they are zeroed before PV (the
-          // whole warp runs this loop; the abort flag is read once for all its lanes)
-#pragma unroll
-          for (int i = 0; i < kPerHalf; ++i) zero_chunk_rows(ring_chunk(S, sl[i]), keep, lane);
+          // paged cache, the sequence's last window: V rows past its end are zeroed (see
+          // the bf16 branch below)
+          zero_chunk_rows(ring_chunk(S, s0), keep, lane);
+          zero_chunk_rows(ring_chunk(S, s1), keep, lane);
           fence_proxy_async_smem();
           __syncwarp();
         }
         if (!*abort && leader) {
-          const uint32_t d = tmem + C::kTmemO + C::kSCols * h;
-          const uint32_t a_base = smem_u32(ring_chunk(S, sl[0]));
 #pragma unroll
-          for (int kt = 0; kt < kTile / C::kMmaK; ++kt) {
-            // bf16: the half's two boxes are adjacent slots, kChunkBytes apart along M
-            const uint64_t ad = sdesc_sw128(a_base + kMnStep * kt, kChunkBytes, 1024);
-            const uint64_t bd = sdesc_sw128(p_base + kMnStep * kt, kPBytes, 1024);
-            mma(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t d = tmem + C::kTmemO + C::kSCols * h;
+            const uint32_t a_base = smem_u32(ring_chunk(S, h == 0 ? s0 : s1));
+#pragma unroll
+            for (int kt = 0; kt < kTile / C::kMmaK; ++kt) {
+              const uint64_t ad = sdesc_sw128(a_base + kMnStep * kt, kChunkBytes, 1024);
+              const uint64_t bd = sdesc_sw128(p_base + kMnStep * kt, kPBytes, 1024);
+              mma(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+            }
           }
-#pragma unroll
-          for (int i = 0; i < kPerHalf; ++i) umma_commit(&S.kv_empty[sl[i]]);
+          umma_commit(&S.kv_empty[s0]);
+          umma_commit(&S.kv_empty[s1]);
+          umma_commit(&S.p_free);
         }
+        chunk += 2;
+      } else {
+        // each half of V^T (the 128 dims of one M=128 product: two bf16 boxes) is used as soon
+        // as TMA has landed it
+        constexpr int kPerHalf = kC / 2;
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t c0 = chunk + kPerHalf * h;
+          uint32_t sl[kPerHalf];
+#pragma unroll
+          for (int i = 0; i < kPerHalf; ++i) {
+            sl[i] = (c0 + i) % kSlots;
+            mbar_wait(&S.kv_full[sl[i]], ((c0 + i) / kSlots) & 1, abort);
+          }
+          tc_fence_after();
+          if (kPaged && keep < kTile && __shfl_sync(0xffffffffu, *abort, 0) == 0) {
+            // paged cache, the sequence's last window: V rows past its end may hold any
+            // bytes (NaN too) and meet a zero weight, so they are zeroed before PV (the
+            // whole warp runs this loop; the abort flag is read once for all its lanes)
+#pragma unroll
+            for (int i = 0; i < kPerHalf; ++i) zero_chunk_rows(ring_chunk(S, sl[i]), keep, lane);
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+          if (!*abort && leader) {
+            const uint32_t d = tmem + C::kTmemO + C::kSCols * h;
+            const uint32_t a_base = smem_u32(ring_chunk(S, sl[0]));
+#pragma unroll
+            for (int kt = 0; kt < kTile / C::kMmaK; ++kt) {
+              // bf16: the half's two boxes are adjacent slots, kChunkBytes apart along M
+              const uint64_t ad = sdesc_sw128(a_base + kMnStep * kt, kChunkBytes, 1024);
+              const uint64_t bd = sdesc_sw128(p_base + kMnStep * kt, kPBytes, 1024);
+              mma(d, ad, bd, C::kIdescPV, !(first && kt == 0));
+            }
+#pragma unroll
+            for (int i = 0; i < kPerHalf; ++i) umma_commit(&S.kv_empty[sl[i]]);
+          }
+        }
+        chunk += kC;
+        if (!*abort && leader) umma_commit(&S.p_free);
       }
-      chunk += kC;
-      if (!*abort && leader) umma_commit(&S.p_free);
     };
 
     for (int t = 0; t < n; ++t) {
@@ -560,23 +637,33 @@ __device__ __forceinline__ uint32_t split_e4m3x2(uint32_t v, uint16_t& hi, uint1
   return hadd2_u32(hf, e4m3x2_to_f16x2(lo));
 }
 
-// Q of the current item (bf16, four TMA boxes of [64 heads x 64 dims]) -> in place, two
+// Q of work item `item` (bf16, four TMA boxes of [64 heads x 64 dims]) -> in place, two
 // chunks of [128 rows x 128 dims] e4m3 (row h: the hi part of head h; row 64 + h: its lo
 // part; 128-byte swizzle), scaled by 2^-e with e chosen so that the largest |q| maps into
-// [128, 256). Returns e. Thread st takes head st / 4 and dims [64 (st % 4), +64): the eight
-// 16-byte pieces of one raw box row in, four pieces of the hi row and four of the lo row out.
-// Every thread has read its input before any thread writes: outputs overlap inputs.
-// (Not inlined: runs once per work item, and inlined it pushed the softmax loop to spill.)
-__device__ __noinline__ int convert_q8(TcSmem& S, int item, int st, int swarp, int lane, volatile int* abort) {
-  mbar_wait(&S.q_full[0], item & 1, abort);
-  const int h = st >> 2, qd = st & 3;
-  const uint8_t* src = S.q[qd] + h * 128;
-  uint4 v[8];
+// [128, 256). Returns e. Each of the softmax threads takes kPer consecutive dims of one head:
+// kPer / 8 16-byte pieces of one raw box row in, kPer / 16 pieces of the hi row and as many
+// of the lo row out. Every thread has read its input before any thread writes: outputs
+// overlap inputs. (Not inlined: it runs once per work item, and inlined it pushed the
+// softmax loop to spill.)
+__device__ __noinline__ int convert_q8(TcSmem& S, int item, int st, int swarp, int lane,
+                                      volatile int* abort) {
+  using C = Cfg<true>;
+  constexpr int kPer = kHeads * kHeadDim / (32 * C::kSoftmaxWarps);  // dims per thread
+  constexpr int kParts = kHeadDim / kPer;                             // threads per head
+  static_assert(kPer % 16 == 0 && 64 % kPer == 0, "Q split shares");
+  const int qb = item & 1;  // two Q buffers
+  mbar_wait(&S.q_full[qb], (item >> 1) & 1, abort);
+  uint8_t* const qbuf = q_buf<true>(S, qb);
+  const int h = st / kParts, d0 = (st % kParts) * kPer;  // head, first dim
+  const uint8_t* src = qbuf + (d0 / 64) * kQChunkBytes + h * 128;
+  const int rp0 = (d0 % 64) / 8;  // first raw piece of the row
+  uint4 v[kPer / 8];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) v[j] = *reinterpret_cast<const uint4*>(src + ((j ^ (h & 7)) << 4));
+  for (int j = 0; j < kPer / 8; ++j)
+    v[j] = *reinterpret_cast<const uint4*>(src + (((rp0 + j) ^ (h & 7)) << 4));
   float mx = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < kPer / 8; ++j) {
     const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
     for (int k = 0; k < 4; ++k)
@@ -585,16 +672,16 @@ __device__ __noinline__ int convert_q8(TcSmem& S, int item, int st, int swarp, i
   }
   mx = warp_max_f32(mx);
   if (lane == 0) S.qmax[swarp] = mx;
-  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);  // also: every raw row has been read
+  named_bar_sync(C::kBarAll, 32 * C::kSoftmaxWarps);  // also: every raw row has been read
   float m = 0.f;
 #pragma unroll
-  for (int w = 0; w < kSoftmaxWarps; ++w) m = fmaxf(m, S.qmax[w]);
+  for (int w = 0; w < C::kSoftmaxWarps; ++w) m = fmaxf(m, S.qmax[w]);
   // m * 2^-e in [128, 256); bf16 values times a power of two in [2^-24, 256] are exact in f16
   const int e = (m > 0.f && m <= 3.0e38f) ? ilogbf(m) - 7 : 0;
   const float sc = ldexpf(1.f, -e);
-  uint32_t hi[16], lo[16];  // 64 codes each, four per word
+  uint32_t hi[kPer / 4], lo[kPer / 4];  // kPer codes each, four per word
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < kPer / 8; ++j) {
     const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
     for (int k = 0; k < 4; k += 2) {
@@ -607,11 +694,11 @@ __device__ __noinline__ int convert_q8(TcSmem& S, int item, int st, int swarp, i
       lo[2 * j + k / 2] = static_cast<uint32_t>(l0) | (static_cast<uint32_t>(l1) << 16);
     }
   }
-  uint8_t* chunk = S.q[0] + (qd >> 1) * kQ8ChunkBytes;
-  const int piece0 = 4 * (qd & 1);
+  uint8_t* chunk = qbuf + (d0 / 128) * kQ8ChunkBytes;
+  const int op0 = (d0 % 128) / 16;  // first output piece of the rows
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int pj = piece0 + j;
+  for (int j = 0; j < kPer / 16; ++j) {
+    const int pj = op0 + j;
     *reinterpret_cast<uint4*>(chunk + h * 128 + ((pj ^ (h & 7)) << 4)) =
         make_uint4(hi[4 * j], hi[4 * j + 1], hi[4 * j + 2], hi[4 * j + 3]);
     const int r = 64 + h;
@@ -619,42 +706,54 @@ __device__ __noinline__ int convert_q8(TcSmem& S, int item, int st, int swarp, i
         make_uint4(lo[4 * j], lo[4 * j + 1], lo[4 * j + 2], lo[4 * j + 3]);
   }
   fence_proxy_async_smem();
-  named_bar_sync(kBarAllSoftmax, 32 * kSoftmaxWarps);  // qmax is read before it is reused
+  named_bar_sync(C::kBarAll, 32 * C::kSoftmaxWarps);  // qmax is read before it is reused
   __syncwarp();
   if (lane == 0) mbar_arrive(&S.q_ready);
   return e;
 }
 
 // ---------------------------------------------------------------------------------------
-// warps 2..9: softmax, rescale, epilogue (and the FP8 conversions)
+// warps 2 ..: softmax, rescale, epilogue (and the FP8 split of Q)
 // ---------------------------------------------------------------------------------------
 template <bool kFp8, bool kPaged>
 __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) {
+  using C = Cfg<kFp8>;
+  constexpr int GH = C::kGroupHeads;  // heads of this thread's group
   volatile int* abort = &S.abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int swarp = warp - 2;                // 0..7
-  const int group = swarp >> 2;              // 0: heads 0..31, 1: heads 32..63
-  const int st = threadIdx.x - 64;           // 0..255 (conversions)
+  const int swarp = warp - 2;                // 0 .. kSoftmaxWarps - 1
+  const int group = swarp >> 2;              // heads [GH group, GH (group + 1))
+  const int st = threadIdx.x - 64;           // 0 .. 32 kSoftmaxWarps - 1
   const int gt_id = st & 127;                // thread within the group
   const uint32_t gbar = 1 + group;           // the group's named barrier
-  const int h0 = group * kGroupHeads;
+  const int h0 = group * GH;
   const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
   const int row = quad * 32 + lane;          // tile position / O^T row of this thread
   const uint32_t lane_addr = static_cast<uint32_t>(quad * 32) << 16;
-  using C = Cfg<kFp8>;
+  // the head whose row sum this lane holds after a transpose-sum (see warp_transpose_sum)
+  const int sum_head = GH == 32 ? lane : lane >> 1;
+  const bool sum_owner = GH == 32 || (lane & 1) == 0;
   const float s_mul0 = a.scale * kLog2e * (kFp8 ? a.k_scale : 1.f);
   const float v_mul = kFp8 ? a.v_scale : 1.f;
   constexpr bool paged = kPaged;
   uint32_t gt = 0;
   int item = 0;
   uint8_t* const p_row = S.p + row * 128;
+  // FP8: the next item's Q is split at the end of the current item, before its epilogue, so
+  // that the tensor core can start on it while the epilogue runs
+  int n_items = 0;
+  if constexpr (kFp8) plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem&) { ++n_items; });
+  int q_e = 0;  // FP8: the scale exponent of the current item's Q
 
   plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem& it) {
     const int n = num_tiles(it);
-    float lsum_w = 0.f;  // this warp's running row sum of head h0 + lane
+    float lsum_w = 0.f;  // this warp's running row sum of head h0 + sum_head
     float s_mul = s_mul0;
-    // FP8: Q split into e4m3 hi and lo parts scaled by 2^-e, so the scores carry 2^e
-    if constexpr (kFp8) s_mul = s_mul0 * ldexpf(1.f, convert_q8(S, item, st, swarp, lane, abort));
+    if constexpr (kFp8) {
+      // Q split into e4m3 hi and lo parts scaled by 2^-e, so the scores carry 2^e
+      if (item == 0) q_e = convert_q8(S, item, st, swarp, lane, abort);
+      s_mul = s_mul0 * ldexpf(1.f, q_e);
+    }
 
     for (int t = 0; t < n; ++t) {
       int y, a0, e0;
@@ -665,19 +764,19 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
 
       mbar_wait(&S.s_full[j], k & 1, abort);
       tc_fence_after();
-      float s[kGroupHeads];
+      float s[GH];
       {
         const uint32_t sa = tmem + lane_addr + kTmemS + C::kSCols * j + h0;
-        uint32_t sr[kGroupHeads];
-        tmem_ld_32x32b_x32(sa, sr);
+        uint32_t sr[GH];
+        tmem_ld_cols<GH>(sa, sr);
         tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < kGroupHeads; ++h) s[h] = __uint_as_float(sr[h]);
+        for (int h = 0; h < GH; ++h) s[h] = __uint_as_float(sr[h]);
         if constexpr (kFp8) {  // plus the lo parts' scores, 64 columns on
-          tmem_ld_32x32b_x32(sa + 64, sr);
+          tmem_ld_cols<GH>(sa + 64, sr);
           tmem_wait_ld();
 #pragma unroll
-          for (int h = 0; h < kGroupHeads; ++h) s[h] += __uint_as_float(sr[h]);
+          for (int h = 0; h < GH; ++h) s[h] += __uint_as_float(sr[h]);
         }
       }
       tc_fence_before();
@@ -685,23 +784,22 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       if (lane == 0) mbar_arrive(&S.s_free[j]);
 
 #pragma unroll
-      for (int h = 0; h < kGroupHeads; ++h) s[h] = valid ? s[h] * s_mul : -INFINITY;
+      for (int h = 0; h < GH; ++h) s[h] = valid ? s[h] * s_mul : -INFINITY;
 
       bool need = (t == 0);
       if (!need) {
 #pragma unroll
-        for (int h = 0; h < kGroupHeads; ++h)
-          need |= s[h] > S.m_used[h0 + h] + C::kRescaleThreshold;
+        for (int h = 0; h < GH; ++h) need |= s[h] > S.m_used[h0 + h] + C::kRescaleThreshold;
       }
       if (named_bar_or(gbar, kGroupThreads, need)) {
         // exact per-head max of this tile across the 128 positions
 #pragma unroll
-        for (int h = 0; h < kGroupHeads; ++h) {
+        for (int h = 0; h < GH; ++h) {
           const float r = warp_max_f32(s[h]);
           if (lane == 0) S.red[quad][h0 + h] = r;
         }
         named_bar_sync(gbar, kGroupThreads);
-        if (gt_id < kGroupHeads) {
+        if (gt_id < GH) {
           const int hh = h0 + gt_id;
           const float mt = fmaxf(fmaxf(S.red[0][hh], S.red[1][hh]), fmaxf(S.red[2][hh], S.red[3][hh]));
           const float mo = t == 0 ? -INFINITY : S.m_used[hh];
@@ -711,22 +809,22 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
         }
         named_bar_sync(gbar, kGroupThreads);
         if (t > 0) {
-          lsum_w *= S.alpha[h0 + lane];
+          lsum_w *= S.alpha[h0 + sum_head];
           // O must hold PV(t-1) before it is rescaled
           mbar_wait(&S.p_free, (tile - 1) & 1, abort);
           tc_fence_after();
           // each O^T half (FP8: its hi and its lo columns)
 #pragma unroll 1
           for (int hp = 0; hp < (kFp8 ? 4 : 2); ++hp) {
-            uint32_t o[kGroupHeads];
+            uint32_t o[GH];
             const uint32_t addr =
                 tmem + lane_addr + C::kTmemO + C::kSCols * (hp & 1) + 64 * (hp >> 1) + h0;
-            tmem_ld_32x32b_x32(addr, o);
+            tmem_ld_cols<GH>(addr, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < kGroupHeads; ++h)
+            for (int h = 0; h < GH; ++h)
               o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h0 + h]);
-            tmem_st_32x32b_x32(addr, o);
+            tmem_st_cols<GH>(addr, o);
           }
           tmem_wait_st();
         }
@@ -735,9 +833,9 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       // probabilities, rounded to what the tensor core reads (bf16; for FP8 caches e4m3 hi
       // and lo parts), this group's share of the P^T row, and the row sums of the rounded
       // values
-      uint32_t pk[kGroupHeads / 2];  // bf16: 32 values; FP8: 32 hi codes, then 32 lo codes
+      uint32_t pk[GH / 2];  // bf16: GH values; FP8: GH hi codes, then GH lo codes
 #pragma unroll
-      for (int h = 0; h < kGroupHeads; h += 2) {
+      for (int h = 0; h < GH; h += 2) {
         const float p0 = ex2(s[h] - (S.m_used[h0 + h] - C::kPExp));
         const float p1 = ex2(s[h + 1] - (S.m_used[h0 + h + 1] - C::kPExp));
         if constexpr (kFp8) {
@@ -745,10 +843,10 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
           const uint32_t w = split_e4m3x2(pack_f16x2(p0, p1), hi, lo);
           if ((h & 2) == 0) {
             pk[h / 4] = hi;
-            pk[8 + h / 4] = lo;
+            pk[GH / 4 + h / 4] = lo;
           } else {
             pk[h / 4] |= static_cast<uint32_t>(hi) << 16;
-            pk[8 + h / 4] |= static_cast<uint32_t>(lo) << 16;
+            pk[GH / 4 + h / 4] |= static_cast<uint32_t>(lo) << 16;
           }
           s[h] = f16_lo(w);
           s[h + 1] = f16_hi(w);
@@ -759,14 +857,17 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
           s[h + 1] = __uint_as_float(w & 0xFFFF0000u);
         }
       }
-      lsum_w += warp_transpose_sum32(s, lane);
+      lsum_w += warp_transpose_sum<GH>(s, lane);
       // the P^T buffer is free once PV(t-1) has read it
       if (tile >= 1) mbar_wait(&S.p_free, (tile - 1) & 1, abort);
+      // logical 16-byte pieces of the 128-byte row: bf16, heads 8 c .. 8 c + 7 in piece c;
+      // FP8, the hi codes of heads 16 c .. 16 c + 15 in piece c < 4, their lo codes in 4 + c
+      constexpr int kPieces = GH / 8;  // of this group
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        // logical 16-byte piece of the 128-byte row: bf16, heads 8 c' .. 8 c' + 7 in piece c';
-        // FP8, hi codes of heads 16 c' .. in piece c' < 4, lo codes in piece 4 + c'
-        const int cl = kFp8 ? (c < 2 ? 2 * group + c : 4 + 2 * group + (c - 2)) : 4 * group + c;
+      for (int c = 0; c < kPieces; ++c) {
+        const int cl = kFp8 ? (c < kPieces / 2 ? group * (kPieces / 2) + c
+                                               : 4 + group * (kPieces / 2) + (c - kPieces / 2))
+                            : group * kPieces + c;
         uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
         *reinterpret_cast<uint4*>(p_row + ((cl ^ (row & 7)) << 4)) = v;
       }
@@ -776,11 +877,16 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       if (lane == 0) mbar_arrive(&S.p_full);
     }
     gt += n;
+    if constexpr (kFp8) {
+      // every S of this item has completed (its scores were read above), and the next Q
+      // sits in the other buffer
+      if (item + 1 < n_items) q_e = convert_q8(S, item + 1, st, swarp, lane, abort);
+    }
 
     // ---- epilogue of the item (each group for its heads) ----
-    S.red[quad][h0 + lane] = lsum_w;
+    if (sum_owner) S.red[quad][h0 + sum_head] = lsum_w;
     named_bar_sync(gbar, kGroupThreads);
-    if (gt_id < kGroupHeads) {
+    if (gt_id < GH) {
       const int hh = h0 + gt_id;
       S.lsum[hh] = S.red[0][hh] + S.red[1][hh] + S.red[2][hh] + S.red[3][hh];
     }
@@ -793,28 +899,28 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     float* pacc = it.slot >= 0 ? partial_acc(a.partials, it.slot) : nullptr;
 #pragma unroll 1
     for (int hf = 0; hf < 2; ++hf) {
-      uint32_t o[kGroupHeads];
+      uint32_t o[GH];
       const uint32_t oa = tmem + lane_addr + C::kTmemO + C::kSCols * hf + h0;
-      tmem_ld_32x32b_x32(oa, o);
+      tmem_ld_cols<GH>(oa, o);
       tmem_wait_ld();
       if constexpr (kFp8) {  // O = (V . P_hi) + (V . P_lo)
-        uint32_t ol[kGroupHeads];
-        tmem_ld_32x32b_x32(oa + 64, ol);
+        uint32_t ol[GH];
+        tmem_ld_cols<GH>(oa + 64, ol);
         tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < kGroupHeads; ++h)
+        for (int h = 0; h < GH; ++h)
           o[h] = __float_as_uint(__uint_as_float(o[h]) + __uint_as_float(ol[h]));
       }
       const int d = hf * 128 + row;
       if (ok) {
         if (it.slot < 0) {
 #pragma unroll
-          for (int h = 0; h < kGroupHeads; ++h)
+          for (int h = 0; h < GH; ++h)
             out[(h0 + h) * kHeadDim + d] =
                 f32_to_bf16_bits(__uint_as_float(o[h]) * (v_mul / S.lsum[h0 + h]));
         } else {
 #pragma unroll
-          for (int h = 0; h < kGroupHeads; ++h) pacc[(h0 + h) * kHeadDim + d] = __uint_as_float(o[h]);
+          for (int h = 0; h < GH; ++h) pacc[(h0 + h) * kHeadDim + d] = __uint_as_float(o[h]);
         }
       }
     }
@@ -822,7 +928,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.o_free);
 
-    if (it.slot >= 0 && ok && gt_id < kGroupHeads) {
+    if (it.slot >= 0 && ok && gt_id < GH) {
       partial_m(a.partials, it.slot)[h0 + gt_id] = S.m_used[h0 + gt_id];
       partial_l(a.partials, it.slot)[h0 + gt_id] = S.lsum[h0 + gt_id];
     }
@@ -833,7 +939,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
 }
 
 template <bool kFp8, bool kPaged>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap q_map, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   TcSmem& S = *reinterpret_cast<TcSmem*>(
@@ -850,14 +956,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&S.q_full[i], 1);
       mbar_init(&S.q_empty[i], 1);
     }
-    mbar_init(&S.q_ready, kSoftmaxWarps);
+    mbar_init(&S.q_ready, Cfg<kFp8>::kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&S.s_full[i], 1);
-      mbar_init(&S.s_free[i], kSoftmaxWarps);
+      mbar_init(&S.s_free[i], Cfg<kFp8>::kSoftmaxWarps);
     }
-    mbar_init(&S.p_full, kSoftmaxWarps);
+    mbar_init(&S.p_full, Cfg<kFp8>::kSoftmaxWarps);
     mbar_init(&S.p_free, 1);
-    mbar_init(&S.o_free, kSoftmaxWarps);
+    mbar_init(&S.o_free, Cfg<kFp8>::kSoftmaxWarps);
     mbar_init(&S.mma_done, 1);
     S.abort_flag = 0;
     fence_mbar_init();
@@ -1024,7 +1130,7 @@ static cudaError_t launch_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaSt
   cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<kFp8, kPaged>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attention_tc_kernel<kFp8, kPaged>, dim3(a.grid), dim3(kThreads), smem, s,
+  return launch_pdl(attention_tc_kernel<kFp8, kPaged>, dim3(a.grid), dim3(Cfg<kFp8>::kThreads), smem, s,
                     q_map, a);
 }
 
