@@ -9,9 +9,9 @@
 //
 // Design (one persistent CTA per SM, warp-specialized, 320 threads):
 //   warp 0      TMA producer: Q of each work item (4 boxes of [64 heads x 64 dims]; two Q
-//               buffers for bf16 caches, so the next item's Q loads while this one streams),
-//               then K and V tiles of 128 positions as 16 KB boxes of [128 positions x 64
-//               dims] into a 6-slot shared-memory ring (128-byte swizzle).
+//               buffers, so the next item's Q loads while this one streams), then K and V
+//               tiles of 128 positions as 16 KB boxes of [128 positions x 64 dims] into a
+//               6-slot shared-memory ring (128-byte swizzle).
 //   warp 1      TMEM owner and MMA issuer (one elected lane; the warp runs converged). Per
 //               tile t:
 //                 S^T(t)[128 pos x 64 heads] = K(t)[128 x 256] . Q^T        (M=128, N=64)
@@ -31,13 +31,15 @@
 // FP8 caches: the e4m3 codes go to the tensor cores as they are (tcgen05 kind::f8f6f4; e4m3
 // values times the power-of-two scales below are exact, and so are the products). The ring
 // holds raw boxes of [128 positions x 128 dims] (128 bytes a row, the same swizzle), two per
-// K or V tile, ten in flight. The other operand must be e4m3 too, so Q and P each become a
+// K or V tile, eight in flight; each S and each PV is issued as 8 MMAs back to back once
+// both of its boxes have landed (at this byte rate the ring runs ahead of the tensor core). The other operand must be e4m3 too, so Q and P each become a
 // pair of e4m3 matrices with one common scale, a high part and the rounded remainder (hi +
 // lo keeps 7 to 8 significant bits, about what bf16 keeps), stacked along N:
 //   S^T(t)[128 pos x 128] = K(t) . [Q_hi ; Q_lo]^T        (M=128, N=128: hi heads, lo heads)
 //   O^T[256 x 128]     += V(t)^T . [P_hi | P_lo]^T(t)  (2 x M=128, N=128)
 // and the softmax adds the two halves of S, the epilogue those of O. Q is split once per
-// work item (scaled by 2^-e so that its largest magnitude is in [128, 256)); P is computed as
+// work item by the softmax warps (scaled by 2^-e so that its largest magnitude is in
+// [128, 256)), the next item's at the end of the current one; P is computed as
 // 2^(s - m + 4) and raised m only when a tile's max exceeds it by more than 4, so P stays
 // below 2^8 and its useful values clear e4m3's subnormal range. The K and V scales fold into
 // the softmax scale and the output scale.
