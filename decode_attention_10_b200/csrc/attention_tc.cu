@@ -105,7 +105,7 @@ struct Cfg {
   static constexpr uint32_t kIdescPV = idesc_f16(128, kSCols, !kFp8, true, true);   // V^T x P^T
 };
 static_assert(Cfg<true>::kSlots <= kMaxSlots && Cfg<false>::kSlots <= kMaxSlots, "ring");
-static_assert(2 * kQ8ChunkBytes == 4 * kQChunkBytes, "FP8 Q is converted in place");
+static_assert(2 * kQ8ChunkBytes == 4 * kQChunkBytes, "FP8 Q is split in place");
 static_assert(Cfg<true>::kSoftmaxWarps <= kMaxSoftmaxWarps &&
                   Cfg<false>::kSoftmaxWarps <= kMaxSoftmaxWarps,
               "softmax warps");
