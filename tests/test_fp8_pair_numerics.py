@@ -6,8 +6,8 @@ are used as they are, while Q and P (values that carry more precision) are writt
 of e4m3 values with one common power-of-two scale: hi = e4m3(x), lo = e4m3(x - hi). The
 kernel computes in f16x2: x is first rounded to f16, the remainder x - hi and the sum hi + lo
 are taken in f16. This file checks that those steps are exact where the kernel needs them
-exact, and that hi + lo is within 2^-8 |x| of x (for |x| >= 1/4; within 2^-10 below), the
-size of a bf16 rounding. Q is scaled so that
+exact, that hi + lo is within 2^-8 |x| of x (for |x| >= 1/4; within 2^-10 below), the
+size of a bf16 rounding, and that for bf16 inputs (Q) the pair is exact. Q is scaled so that
 its largest magnitude lies in [128, 256). P = 2^(s - m + 4), with the running max m raised
 once a score exceeds it by more than 4, so P <= 2^8. Neither ever reaches e4m3's largest
 value, 448.
@@ -89,3 +89,17 @@ def test_p_stays_below_2_pow_8_under_the_rescale_threshold():
     # weights down to 2^-10 of the largest possible stay out of e4m3's subnormal range once
     # scaled: 2^-10 * 2^4 (the smallest largest weight) = 2^-6, e4m3's smallest normal
     assert np.exp2(-10.0 + 4.0) == 2.0 ** -6
+
+
+def test_q_pair_is_exact_for_bf16_values():
+    # q arrives in bf16 (8 significant bits): hi takes the top 4 (rounded), and the remainder
+    # always fits e4m3's 4 significant bits, so hi + lo is q itself as long as the remainder's
+    # last bit (2^-7 of |q|) is not below e4m3's subnormal step 2^-9, i.e. |q| >= 2^-2 once
+    # scaled (q's largest magnitude sits in [128, 256), so that is every q within 2^-10 of it)
+    bits = np.arange(0, 0x7F80, dtype=np.uint32).astype(np.uint16)
+    x = codecs.bf16_decode(bits)
+    x = x[(x >= 0.25) & (x <= 256.0)]
+    assert len(x) > 1000
+    hi, r, lo = _split(x)
+    assert np.array_equal(hi + lo, x)
+    assert np.array_equal(lo, r)  # the remainder is itself an e4m3 value
