@@ -678,8 +678,9 @@ __device__ __noinline__ int convert_q8(TcSmem& S, int item, int st, int swarp, i
   float m = 0.f;
 #pragma unroll
   for (int w = 0; w < C::kSoftmaxWarps; ++w) m = fmaxf(m, S.qmax[w]);
-  // m * 2^-e in [128, 256); bf16 values times a power of two in [2^-24, 256] are exact in f16
-  const int e = (m > 0.f && m <= 3.0e38f) ? ilogbf(m) - 7 : 0;
+  // m * 2^-e in [128, 256); bf16 values times a power of two in [2^-24, 256] are exact in f16.
+  // e >= -100 keeps 2^-e finite (a Q whose largest |q| is below 2^-93 is scaled less).
+  const int e = (m > 0.f && m <= 3.0e38f) ? max(ilogbf(m) - 7, -100) : 0;
   const float sc = ldexpf(1.f, -e);
   uint32_t hi[kPer / 4], lo[kPer / 4];  // kPer codes each, four per word
 #pragma unroll

@@ -67,9 +67,15 @@ def test_q_scale_maps_the_largest_magnitude_into_128_256_and_keeps_bf16_values_e
     # every positive finite bf16 value as the largest |q| of an item
     bits = np.arange(1, 0x7F80, dtype=np.uint32)
     m = codecs.bf16_decode(bits.astype(np.uint16))
-    e = np.floor(np.log2(m)).astype(np.int64) - 7
+    # the kernel's rule: e = floor(log2 m) - 7, but at least -100, so that 2^-e stays a
+    # finite float32 even for bf16 subnormals
+    e = np.maximum(np.floor(np.log2(m)).astype(np.int64) - 7, -100)
+    assert np.isfinite(np.float32(np.ldexp(1.0, 100)))
     scaled = np.ldexp(m, -e)
-    assert ((scaled >= 128.0) & (scaled < 256.0)).all()
+    regular = m >= 2.0 ** -93
+    assert ((scaled[regular] >= 128.0) & (scaled[regular] < 256.0)).all()
+    assert (scaled[~regular] < 128.0).all() and (scaled[~regular] > 0).all()
+    m, e = m[regular], e[regular]
     # any bf16 value up to the largest, times the same power of two, is exact in f16 unless it
     # falls below f16's normal range (2^-14 of a maximum in [128, 256): no contribution)
     rng = np.random.default_rng(5)
