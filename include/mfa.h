@@ -187,9 +187,10 @@ MFA_API mfa_status mfa_kv_append(const void* x, const void* w_k, const void* w_v
  * "Method"; the cost is max(attention compute, KV memory access)):
  *   out[b][h] = sum_{j < L_b} softmax_j(scale * q[b][h] . K_b[j]) V_b[j],  L_b = seq_lens[b],
  * with K_b, V_b the cache rows (e4m3 codes times their scale for FP8 caches). For FP8 caches
- * the products run on e4m3 tensor cores: the cached codes are used exactly, q is written as
- * an exact pair of e4m3 values (hi + lo, one power-of-two scale per sequence), and the
- * softmax weights as such a pair within 2^-8 of their value (a bf16 rounding's size).
+ * the products run on e4m3 tensor cores: the cached codes are used exactly; q is written as
+ * a pair of e4m3 values (hi + lo, one power-of-two scale per sequence), exact for every
+ * element within 2^-10 of the sequence's largest |q|; the softmax weights as such a pair
+ * within 2^-8 of their value (a bf16 rounding's size).
  * q: device bf16 [kv->batch, 64, 256]; seq_lens: device int32 [kv->batch]; out: device
  * bf16 [kv->batch, 64, 256]; scale > 0 (1/16 for the layer). The work is split over the
  * GPU's SMs by length (split-K over the cache; a second kernel on the same stream merges
