@@ -347,7 +347,9 @@ def a8_dequantize(codes, scales, group=A8_GROUP):
 def fp8_project(a, w_codes, w_scales):
     """A projection on the FP8 path: the activation rows quantized by ``a8_quantize``, the
     weight block-FP8; the products of the real values, summed in float64. Returns [rows,
-    out]."""
+    out].
+
+    Pinned by: ``math.fsum`` of the decoded codes times their scales, element by element."""
     ac, asc = a8_quantize(a)
     return a8_dequantize(ac, asc) @ w8_dequantize(w_codes, w_scales)
 
@@ -356,7 +358,13 @@ def query_proj_fp8(x, wq_codes, wq_scales, gamma, wu_codes, wu_scales, eps=RMS_E
                    n_heads=N_HEADS, emulate=True):
     """The query path on the FP8 path: c = fp8_project(x, W_qdown), RMSNorm as ever, then
     q = fp8_project(c_hat, W_qup) (c_hat rounded to bf16 first with ``emulate``, as stored).
-    Returns (c_hat, q)."""
+    Returns (c_hat, q).
+
+    Pinned by: a pure-Python brute force of the whole chain at small sizes (exact ``fsum``
+    sums of decoded codes times block scales, the bf16 rounding of c_hat before it is
+    quantized, head-major output columns), one-hot routing of chosen inputs to chosen
+    (head, dim) slots, and two planted mistakes (quantizing c_hat before its bf16 rounding;
+    a dim-major reshape) that the brute force rejects."""
     c_hat = rms_norm(fp8_project(x, wq_codes, wq_scales), gamma, eps)
     if emulate:
         c_hat = codecs.bf16_round(c_hat)

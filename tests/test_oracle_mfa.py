@@ -526,3 +526,136 @@ def test_fp8_project_is_the_sum_of_real_products():
 def _f32_rne(x):
     import struct
     return struct.unpack("<f", struct.pack("<f", x))[0]
+
+
+# ----------------------------------------------------------------------------------------
+# the whole FP8 query chain (step3-fp8 model card: block-fp8 checkpoints; bud-325 "Key
+# claims": the model runs in FP8), brute force at tiny sizes
+# ----------------------------------------------------------------------------------------
+
+
+def _brute_quantize_row(row):
+    """One activation row in groups of 128: (codes, scales) by the reading's rule, written
+    out element by element (float32 scale and quotient, e4m3 nearest-even saturating)."""
+    codes, scales = [], []
+    for g0 in range(0, len(row), 128):
+        grp = [float(v) for v in row[g0:g0 + 128]]
+        amax = max(abs(v) for v in grp)
+        sc = _f32_rne(_f32_rne(amax) / 448.0) if amax > 0 else 1.0
+        scales.append(sc)
+        codes.extend(int(codecs.e4m3_encode(_f32_rne(v / sc))) for v in grp)
+    return codes, scales
+
+
+def _brute_fp8_dot(a_codes, a_scales, w_codes, w_scales, o):
+    """sum_k a_k w[o, k] over the real values code * scale, as one exact-rounded fsum."""
+    return math.fsum(float(codecs.e4m3_decode(a_codes[k])) * a_scales[k // 128]
+                     * float(codecs.e4m3_decode(w_codes[o, k])) * float(w_scales[o // 128, k // 128])
+                     for k in range(len(a_codes)))
+
+
+def _brute_query_proj_fp8(x, wq_codes, wq_scales, gamma, wu_codes, wu_scales, n_heads, eps):
+    """The FP8 query path in pure Python: x quantized per group, c by exact sums, RMSNorm,
+    c_hat rounded to bf16 (as stored) and only then quantized, q by exact sums, rounded to
+    bf16, and q[b][h][d] taken from output column h * head_dim + d (head-major)."""
+    rank = wq_codes.shape[0]
+    width = wu_codes.shape[0]
+    hd = width // n_heads
+    c_hat_all, q_all = [], []
+    for row in x:
+        xc, xs = _brute_quantize_row(row)
+        c = [_brute_fp8_dot(xc, xs, wq_codes, wq_scales, r) for r in range(rank)]
+        inv = 1.0 / math.sqrt(math.fsum(v * v for v in c) / rank + eps)
+        c_hat = [float(codecs.bf16_round(v * inv * float(gamma[j]))) for j, v in enumerate(c)]
+        cc, cs = _brute_quantize_row(c_hat)
+        q = [[float(codecs.bf16_round(_brute_fp8_dot(cc, cs, wu_codes, wu_scales, h * hd + d)))
+              for d in range(hd)] for h in range(n_heads)]
+        c_hat_all.append(c_hat)
+        q_all.append(q)
+    return np.array(c_hat_all), np.array(q_all)
+
+
+def _fp8_chain_inputs(seed=21, bsz=2, din=256, rank=256, n_heads=3, hd=64):
+    rng = np.random.default_rng(seed)
+    x = codecs.bf16_round(rng.standard_normal((bsz, din)) * rng.uniform(0.2, 5.0, (bsz, 1)))
+    wq = rng.standard_normal((rank, din)) / math.sqrt(din)          # [out, in]
+    wu = rng.standard_normal((n_heads * hd, rank)) / math.sqrt(rank)
+    # block scales of different sizes per 128 x 128 block (the output side of W_qup ends in a
+    # ragged block of 64)
+    wq_s = np.array([[0.004, 0.003], [0.005, 0.0035]], np.float32)
+    wu_s = np.array([[0.006, 0.0045], [0.005, 0.007]], np.float32)
+    wq_c = codecs.e4m3_encode(wq / np.repeat(np.repeat(wq_s, 128, 0), 128, 1)[:rank, :din])
+    wu_c = codecs.e4m3_encode(wu / np.repeat(np.repeat(wu_s, 128, 0), 128, 1)[:n_heads * hd, :rank])
+    gamma = codecs.bf16_round(rng.uniform(0.5, 1.5, rank))
+    return x, wq_c, wq_s, gamma, wu_c, wu_s, n_heads
+
+
+_BRUTE_FP8 = {}
+
+
+def _brute_fp8_chain():
+    """The brute force of the default chain inputs, computed once for the tests below."""
+    if not _BRUTE_FP8:
+        x, wq_c, wq_s, gamma, wu_c, wu_s, nh = _fp8_chain_inputs()
+        _BRUTE_FP8["r"] = _brute_query_proj_fp8(x, wq_c, wq_s, gamma, wu_c, wu_s, nh,
+                                                mfa.RMS_EPS)
+    return _BRUTE_FP8["r"]
+
+
+def test_query_proj_fp8_matches_pure_python_brute_force():
+    x, wq_c, wq_s, gamma, wu_c, wu_s, nh = _fp8_chain_inputs()
+    c_hat, q = mfa.query_proj_fp8(x, wq_c, wq_s, gamma, wu_c, wu_s, n_heads=nh)
+    bc, bq = _brute_fp8_chain()
+    assert q.shape == bq.shape == (2, 3, 64)
+    # both sides round the same real numbers to bf16: equal unless a float64 sum sits within
+    # 1e-16 of a rounding midpoint
+    assert np.array_equal(c_hat, bc)
+    assert np.array_equal(q, bq)
+
+
+def test_query_proj_fp8_one_hot_routes_to_the_head_major_slot():
+    # W_qup with one nonzero code per output column: column h * 64 + d reads input j(h, d),
+    # so q[b, h, d] must be (the e4m3 code of c_hat[j] in its group) * scales, rounded to bf16
+    x, wq_c, wq_s, gamma, _, _, nh = _fp8_chain_inputs(seed=5)
+    hd, rank = 64, 256
+    wu_c = np.zeros((nh * hd, rank), np.uint8)
+    wu_s = np.array([[0.25, 0.5], [2.0, 1.0]], np.float32)
+    one = int(codecs.e4m3_encode(1.0))
+    src = {}
+    for h in range(nh):
+        for d in range(hd):
+            j = (7 * h + 3 * d + 11) % rank
+            wu_c[h * hd + d, j] = one
+            src[h, d] = j
+    c_hat, q = mfa.query_proj_fp8(x, wq_c, wq_s, gamma, wu_c, wu_s, n_heads=nh)
+    for b in range(2):
+        cc, cs = _brute_quantize_row(c_hat[b])
+        for (h, d), j in src.items():
+            o = h * hd + d
+            want = codecs.bf16_round(float(codecs.e4m3_decode(cc[j])) * cs[j // 128]
+                                     * float(wu_s[o // 128, j // 128]))
+            assert q[b, h, d] == want
+
+
+def test_planted_fp8_quantize_before_bf16_rounding_is_caught():
+    # a chain that quantizes the float64 c_hat (before its storage rounding to bf16) differs
+    # from the stated order; the brute-force pin must reject it
+    x, wq_c, wq_s, gamma, wu_c, wu_s, nh = _fp8_chain_inputs()
+
+    def wrong_order(x, wq_c, wq_s, gamma, wu_c, wu_s, n_heads):
+        c_hat = mfa.rms_norm(mfa.fp8_project(x, wq_c, wq_s), gamma)
+        q = codecs.bf16_round(mfa.fp8_project(c_hat, wu_c, wu_s))
+        return q.reshape(q.shape[0], n_heads, -1)
+
+    _, bq = _brute_fp8_chain()
+    assert not np.array_equal(wrong_order(x, wq_c, wq_s, gamma, wu_c, wu_s, nh), bq)
+
+
+def test_planted_fp8_dim_major_reshape_is_caught():
+    # q taken dim-major ([b, head_dim, heads] then transposed) instead of head-major
+    x, wq_c, wq_s, gamma, wu_c, wu_s, nh = _fp8_chain_inputs()
+    _, q = mfa.query_proj_fp8(x, wq_c, wq_s, gamma, wu_c, wu_s, n_heads=nh)
+    flat = q.reshape(q.shape[0], -1)
+    wrong = flat.reshape(q.shape[0], -1, nh).transpose(0, 2, 1)
+    _, bq = _brute_fp8_chain()
+    assert np.array_equal(q, bq) and not np.array_equal(wrong, bq)
