@@ -360,10 +360,28 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     if (ok) issued = chunk + 1;
     ++chunk;
   };
-  // The K/V rows (and the split plan) were written by kernels that completed before this one
-  // launched, so the first boxes of the first item -- a ring-full, which needs no free slot
-  // -- stream in while the previous kernel (which writes q) finishes.
+  // Q of work item `item` into its buffer (after the previous user of the buffer is done).
+  auto issue_q = [&](int item_no, const WorkItem& w) {
+    const int qb = item_no % C::kQBufs, qu = item_no / C::kQBufs;
+    if (qu > 0) mbar_wait(&S.q_empty[qb], (qu - 1) & 1, abort);
+    if (!*abort) {
+      if (leader) {
+        mbar_arrive_expect_tx(&S.q_full[qb], 4 * kQChunkBytes);
+        uint8_t* qd = q_buf<kFp8>(S, qb);
+        for (int c = 0; c < 4; ++c)
+          tma_load_2d(qd + c * kQChunkBytes, q_map, 64 * c, w.b * kHeads, &S.q_full[qb]);
+      }
+      q_issued = item_no + 1;
+    }
+  };
+  // In a layer step the K/V rows (and the split plan) were written by kernels that completed
+  // before this one launched, so the first boxes of the first item -- a ring-full, which
+  // needs no free slot -- stream in while the previous kernel (which writes q) finishes. In a
+  // standalone call the CTA has already waited (it built the plan), so the first item's Q,
+  // which its first product needs, goes out ahead of the ring.
   int first_done = 0;
+  const bool q0_early = !a.plan_early;
+  if (has && q0_early) issue_q(0, it);
   if constexpr (kPaged) {
     if (has) {
       fetch_ids(it);
@@ -389,17 +407,7 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
       prefetch_tensormap(&a.kv[nx.b].tmap_k);
       prefetch_tensormap(&a.kv[nx.b].tmap_v);
     }
-    const int qb = item % C::kQBufs, qu = item / C::kQBufs;
-    if (qu > 0) mbar_wait(&S.q_empty[qb], (qu - 1) & 1, abort);
-    if (!*abort) {
-      if (leader) {
-        mbar_arrive_expect_tx(&S.q_full[qb], 4 * kQChunkBytes);
-        uint8_t* qd = q_buf<kFp8>(S, qb);
-        for (int c = 0; c < 4; ++c)
-          tma_load_2d(qd + c * kQChunkBytes, q_map, 64 * c, it.b * kHeads, &S.q_full[qb]);
-      }
-      q_issued = item + 1;
-    }
+    if (!(item == 0 && q0_early)) issue_q(item, it);
     const int total = kBoxesPerTile * num_tiles(it);
     for (int j = (item == 0 ? first_done : 0); j < total; ++j) issue_box(it, j);
     ++item;
@@ -976,6 +984,14 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     tmem_relinquish();
   }
   pdl_launch_dependents();  // the combine kernel may start launching; it waits for us
+  if (!a.plan_early && threadIdx.x == 0 && a.batch > 0) {
+    // The tensor maps of the sequence this CTA most likely starts in (where it would with
+    // equal lengths), fetched while the plan is built; the KV table is written only by the
+    // host-side table set-up, never by a kernel, so this needs no wait.
+    const KvSeq* kv = a.kv + min(a.batch - 1, static_cast<int>((int64_t)g * a.batch / gridDim.x));
+    prefetch_tensormap(&kv->tmap_k);
+    prefetch_tensormap(&kv->tmap_v);
+  }
   if (a.plan_early) {
     // the split plan, computed during the layer step's x-projection by an extra block of
     // the x-projection's finish kernel
@@ -1025,7 +1041,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 // ---------------------------------------------------------------------------------------
 constexpr int kCombineHeads = 4;
 constexpr int kCombineOnePass = 8;      // up to this many splits: the one-pass merge
-constexpr int kCombineMaxSplits = 256;  // above it: the one-pass merge (never with <= 256 SMs)
+constexpr int kCombineMaxSplits = kMaxAttnGrid;  // a sequence has at most grid splits
 
 __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
   pdl_wait();

@@ -21,7 +21,6 @@ struct PlanSmem {
   int32_t tile_start[kMaxBatch + 1];  // exclusive prefix of tiles per sequence
   int32_t slot_base[kMaxBatch];       // exclusive prefix of partial slots per sequence
   int32_t len[kMaxBatch];             // attended positions (0 for rejected sequences)
-  int32_t scan_tmp[33];
   int32_t grid;  // CTAs that get work: min(G, total tiles), so none of them is empty
   int32_t flag;
   int32_t page_size;  // the KV table's layout: 0 contiguous, else rows per page
@@ -36,55 +35,27 @@ __device__ __forceinline__ int plan_cta_of(int t, int G, int NT) {
   return static_cast<int>((static_cast<int64_t>(t + 1) * G - 1) / NT);
 }
 
-// Block-wide exclusive scan of v[0, n) in place; returns the total. Every thread of the
-// block must call it (blockDim.x a multiple of 32).
-__device__ inline int block_exclusive_scan(int32_t* v, int n, int32_t* tmp) {
-  const int tid = threadIdx.x, nt = blockDim.x;
-  const int per = (n + nt - 1) / nt;
-  const int lo = min(n, tid * per), hi = min(n, lo + per);
-  int local = 0;
-  for (int i = lo; i < hi; ++i) local += v[i];
-  const int lane = tid & 31, warp = tid >> 5, nwarps = nt >> 5;
-  int incl = local;
+// Inclusive sum over the lanes of a warp (lane l gets the sum of lanes 0..l).
+__device__ __forceinline__ int warp_inclusive_sum(int v, int lane) {
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
   }
-  if (lane == 31) tmp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < nwarps ? tmp[lane] : 0;
-    int wi = w;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += y;
-    }
-    if (lane < nwarps) tmp[lane] = wi - w;  // exclusive warp offsets
-    if (lane == 31) tmp[32] = wi;          // total
-  }
-  __syncthreads();
-  int run = tmp[warp] + incl - local;
-  for (int i = lo; i < hi; ++i) {
-    const int x = v[i];
-    v[i] = run;
-    run += x;
-  }
-  const int total = tmp[32];
-  __syncthreads();
-  return total;
+  return v;
 }
 
 // Build the plan for `batch` sequences over a grid of G CTAs. Lengths outside
 // [1, capacity] are rejected (length 0; the output is zero-filled) and, if `report`, flagged.
+// Every thread of the block calls it. The lengths are read by all threads at once (one
+// round trip to memory); warp 0 then scans the tile counts and the split slots, each lane
+// over a contiguous run of sequences, so the block meets at two barriers only.
 __device__ inline void plan_build(PlanSmem& P, const int32_t* __restrict__ seq_lens,
                                   const KvSeq* __restrict__ kv, int batch, int G,
                                   uint32_t* err, bool report) {
   for (int b = threadIdx.x; b < batch; b += blockDim.x) {
     const int L = seq_lens[b];
     const int cap = kv[b].capacity;
-    if (b == 0) P.page_size = kv[0].page_size;  // the same in every entry
     int len = L;
     if (L <= 0) {
       len = 0;
@@ -94,27 +65,51 @@ __device__ inline void plan_build(PlanSmem& P, const int32_t* __restrict__ seq_l
       if (report) atomicOr(err, kErrCapacity);
     }
     P.len[b] = len;
-    P.tile_start[b] = (len + kTile - 1) / kTile;
+    P.tile_start[b] = (len + kTile - 1) / kTile;  // the tile count; scanned below
   }
+  if (threadIdx.x == 0) P.page_size = kv[0].page_size;  // the same in every entry
   __syncthreads();
-  const int NT = block_exclusive_scan(P.tile_start, batch, P.scan_tmp);
-  const int Ge = min(G, NT);
-  if (threadIdx.x == 0) {
-    P.tile_start[batch] = NT;
-    P.grid = Ge;
-  }
-  __syncthreads();
-  for (int b = threadIdx.x; b < batch; b += blockDim.x) {
-    const int ts = P.tile_start[b], te = P.tile_start[b + 1];
-    int slots = 0;
-    if (te > ts) {
-      const int n = plan_cta_of(te - 1, Ge, NT) - plan_cta_of(ts, Ge, NT) + 1;
-      slots = n > 1 ? n : 0;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const int per = (batch + 31) / 32;
+    const int b0 = min(batch, lane * per), b1 = min(batch, b0 + per);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) sum += P.tile_start[b];
+    int incl = warp_inclusive_sum(sum, lane);
+    const int NT = __shfl_sync(0xffffffffu, incl, 31);
+    int run = incl - sum;
+    for (int b = b0; b < b1; ++b) {
+      const int n = P.tile_start[b];
+      P.tile_start[b] = run;
+      run += n;
     }
-    P.slot_base[b] = slots;
+    const int Ge = min(G, NT);  // CTAs that get work, so none of them is empty
+    if (lane == 0) {
+      P.tile_start[batch] = NT;
+      P.grid = Ge;
+    }
+    __syncwarp();
+    // partial slots: a sequence whose tiles fall in n > 1 CTAs' ranges gets n of them
+    sum = 0;
+    for (int b = b0; b < b1; ++b) {
+      const int ts = P.tile_start[b], te = P.tile_start[b + 1];
+      int slots = 0;
+      if (te > ts) {
+        const int n = plan_cta_of(te - 1, Ge, NT) - plan_cta_of(ts, Ge, NT) + 1;
+        slots = n > 1 ? n : 0;
+      }
+      P.slot_base[b] = slots;
+      sum += slots;
+    }
+    incl = warp_inclusive_sum(sum, lane);
+    run = incl - sum;
+    for (int b = b0; b < b1; ++b) {
+      const int n = P.slot_base[b];
+      P.slot_base[b] = run;
+      run += n;
+    }
   }
   __syncthreads();
-  block_exclusive_scan(P.slot_base, batch, P.scan_tmp);
 }
 
 // The plan in global memory: tile_start[batch + 1], slot_base[batch], len[batch], grid,
@@ -160,6 +155,7 @@ struct WorkItem {
   int tok1;     // one past the last
   int slot;     // partial slot, or -1 if the sequence is finished by this item alone
   int nsplit;   // CTAs sharing the sequence
+  int split;    // this item's index among them (its slot is slot_base[b] + split)
 };
 
 // Walk over the work items of CTA g, in order: begin, then get until it returns false.
@@ -200,7 +196,8 @@ __device__ inline bool plan_get(const PlanSmem& P, int batch, PlanCursor& c, Wor
     it.tok1 = min(P.len[b], (a1 - ts) * kTile);
     const int gf = plan_cta_of(ts, G, NT);
     it.nsplit = plan_cta_of(te - 1, G, NT) - gf + 1;
-    it.slot = it.nsplit > 1 ? P.slot_base[b] + (c.g - gf) : -1;
+    it.split = c.g - gf;
+    it.slot = it.nsplit > 1 ? P.slot_base[b] + it.split : -1;
     ++c.b;
     return true;
   }

@@ -86,8 +86,10 @@ struct WsLayout {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// Persistent attention grid: one CTA per SM.
-inline int attn_grid_for(int num_sms) { return num_sms; }
+// Persistent attention grid: one CTA per SM, at most kMaxAttnGrid (the combine kernel merges
+// at most that many splits of one sequence).
+constexpr int kMaxAttnGrid = 256;
+inline int attn_grid_for(int num_sms) { return num_sms < kMaxAttnGrid ? num_sms : kMaxAttnGrid; }
 
 inline WsLayout ws_layout(int batch, int num_sms) {
   WsLayout L{};
