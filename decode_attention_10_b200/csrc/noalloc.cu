@@ -11,8 +11,14 @@
 // The scratch -- the split-K partials of x W_qdown, the normalized low-rank query and the
 // error word -- lives in one file-scope __device__ array of fixed size, sized for at most
 // MFA_NOALLOC_MAX_BATCH token rows. The CUDA runtime reserves it on every GPU that loads
-// the library, for the life of the process. Host code cannot use the array's name as a
-// device address, so its address is looked up per device with cudaGetSymbolAddress.
+// the library, for the life of the process, and zeroes it when it loads the module. Host
+// code cannot use the array's name as a device address, so its address is looked up per
+// device with cudaGetSymbolAddress (once per device: a device reset, which unloads the
+// module, leaves that address stale for the rest of the process).
+//
+// The partials and c_hat are written before they are read in every call, so only the error
+// word must start at zero: it is zero at load, the kernels only OR bits into it, and
+// mfa_query_proj_noalloc_get_error reads and clears it.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -78,11 +84,35 @@ extern "C" MFA_API mfa_status mfa_query_proj_noalloc(const void* x, const void* 
   L.xproj_part = kNoAllocPart;
   L.c_hat = kNoAllocChat;
   L.total = kNoAllocBytes;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the error word is the only part of the scratch that must start at zero
-  if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + L.err, 0, sizeof(uint32_t), s) !=
-      cudaSuccess)
-    return MFA_ERR_CUDA;
   return run_query_proj(x, WRef{w_qdown, nullptr}, gamma, WRef{w_qup, nullptr}, eps, q_out,
-                        batch, scratch, L, s);
+                        batch, scratch, L, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" MFA_API mfa_status mfa_query_proj_noalloc_get_error(void* stream) {
+  void* scratch = nullptr;
+  mfa_status st = scratch_address(&scratch);
+  if (st != MFA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MFA_ERR_CUDA;
+  uint32_t bits = 0;
+  uint8_t* word = static_cast<uint8_t*>(scratch) + kNoAllocErr;
+  if (cudaMemcpy(&bits, word, sizeof(bits), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  if (bits == 0) return MFA_OK;
+  if (cudaMemsetAsync(word, 0, sizeof(bits), s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return MFA_ERR_CUDA;
+  return status_of_error_bits(bits);
+}
+
+extern "C" MFA_API mfa_status mfa_query_proj_noalloc_wait_selftest(uint32_t limit_us,
+                                                                   void* stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return MFA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  mfa_status st = scratch_address(&scratch);
+  if (st != MFA_OK) return st;
+  uint32_t* word = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(scratch) + kNoAllocErr);
+  return launch_wait_selftest(word, limit_us, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MFA_OK
+             : MFA_ERR_CUDA;
 }

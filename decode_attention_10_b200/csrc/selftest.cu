@@ -37,13 +37,18 @@ __global__ void __launch_bounds__(32) wait_selftest_kernel(uint32_t* err, uint64
 
 using namespace mfa;
 
+cudaError_t mfa::launch_wait_selftest(uint32_t* err, uint32_t limit_us, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(err, static_cast<uint64_t>(limit_us) * 1000u);
+  return cudaGetLastError();
+}
+
 extern "C" MFA_API mfa_status mfa_wait_selftest(void* ws, size_t ws_bytes, uint32_t limit_us,
                                                 void* stream) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < 256)
     return MFA_ERR_INVALID_ARG;
   if (limit_us == 0 || limit_us > 1000000u) return MFA_ERR_INVALID_ARG;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  wait_selftest_kernel<<<1, 32, 0, s>>>(static_cast<uint32_t*>(ws),
-                                       static_cast<uint64_t>(limit_us) * 1000u);
-  return cudaGetLastError() == cudaSuccess ? MFA_OK : MFA_ERR_CUDA;
+  return launch_wait_selftest(static_cast<uint32_t*>(ws), limit_us,
+                              static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? MFA_OK
+             : MFA_ERR_CUDA;
 }
