@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libmfa.so")
 SOURCES = ["abi.cu", "query_path.cu", "gemm_tc.cu", "attention_tc.cu", "out_proj.cu", "noalloc.cu",
-           "selftest.cu"]
+           "selftest.cu", "split_plan.cu"]
 HEADERS = ["mfa_internal.cuh", "attn_plan.cuh", "sm100.cuh"]
 
 

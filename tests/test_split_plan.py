@@ -1,62 +1,100 @@
-"""Properties of the attention's split plan that the workspace and the kernels rely on,
-checked on the host over many length mixes.
+"""The attention's length-aware split plan, read back from the device (mfa_split_plan runs
+the same plan_build / plan_get the attention kernels run), checked over many length mixes
+for what the kernels and the workspace rely on:
+- every accepted sequence (1 <= length <= capacity) is covered by its items exactly once,
+  in whole 128-position tiles; rejected sequences get no items;
+- G = min(grid, NT) CTAs get work, none of them empty, and their tile counts differ by at
+  most one (NT counted here from the lengths);
+- a sequence with n > 1 items has split indices 0 .. n-1 in CTA order and n partial slots,
+  distinct over all sequences and inside the workspace's grid + batch slots; a sequence with
+  one item has no slot."""
 
-The plan (decode_attention_10_b200/csrc/attn_plan.cuh) lays every sequence's 128-position
-tiles end to end (NT tiles in all) and gives CTA g of a grid of G = min(grid, NT) CTAs the
-tiles [bound(g), bound(g + 1)), bound(g) = floor(g NT / G). The owner of tile t is
-cta_of(t) = floor(((t + 1) G - 1) / NT). A sequence whose tiles fall to n > 1 CTAs gets n
-partial slots. The two formulas are restated below, and the test checks:
-- every tile belongs to exactly one CTA, and cta_of agrees with bound;
-- no CTA is empty, and tile counts differ by at most one;
-- the slots of all sequences fit the workspace's grid + batch slots, since the workspace is
-  sized for exactly that many.
-"""
+import ctypes
 
 import numpy as np
 import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
 
 TILE = 128
 
 
-def bound(g, G, NT):
-    return (g * NT) // G
+@pytest.fixture(scope="module")
+def lib():
+    from decode_attention_10_b200 import build, mfa
+    build.build()
+    return mfa.load()
 
 
-def cta_of(t, G, NT):
-    return ((t + 1) * G - 1) // NT
+class _Table:
+    """A KV table with the given capacities. Only mfa_split_plan reads it (the capacities):
+    every entry points at one small buffer, so no attention may ever run on it."""
+
+    def __init__(self, lib, caps):
+        from decode_attention_10_b200 import mfa
+        self.batch = len(caps)
+        self.buf = torch.zeros(4096, dtype=torch.bfloat16, device="cuda")
+        nbytes = lib.mfa_kv_table_bytes(self.batch)
+        self.table = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+        arr = ctypes.c_void_p * self.batch
+        ptrs = arr(*([self.buf.data_ptr()] * self.batch))
+        cp = (ctypes.c_int32 * self.batch)(*caps)
+        assert lib.mfa_kv_table_init(self.table.data_ptr(), nbytes, self.batch, 0,
+                                     ctypes.cast(ptrs, ctypes.c_void_p),
+                                     ctypes.cast(ptrs, ctypes.c_void_p),
+                                     ctypes.cast(cp, ctypes.c_void_p), None) == 0
+        self.desc = mfa.KvCacheDesc(self.batch, 0, 1.0, 1.0, self.table.data_ptr(), 0)
 
 
-def plan(lens, grid):
-    tiles = [(L + TILE - 1) // TILE if L > 0 else 0 for L in lens]
-    start = np.concatenate([[0], np.cumsum(tiles)]).astype(np.int64)
-    NT = int(start[-1])
-    G = min(grid, NT)
-    return tiles, start, NT, G
-
-
-def _check(lens, grid):
-    tiles, start, NT, G = plan(lens, grid)
-    if NT == 0:
+def _check(lib, lens, grid, caps=None):
+    from decode_attention_10_b200 import mfa
+    batch = len(lens)
+    caps = caps or [max(1, L) for L in lens]
+    tab = _Table(lib, caps)
+    G, NT, items = mfa.split_plan(tab, torch.tensor(lens, dtype=torch.int32, device="cuda"),
+                                  grid)
+    items = items.numpy()
+    accepted = [1 <= L <= c for L, c in zip(lens, caps)]
+    nt = sum((L + TILE - 1) // TILE for L, ok in zip(lens, accepted) if ok)
+    assert NT == nt and G == min(grid, nt)
+    if nt == 0:
+        assert len(items) == 0
         return
-    owner = np.array([cta_of(t, G, NT) for t in range(NT)])
-    for g in range(G):
-        lo, hi = bound(g, G, NT), bound(g + 1, G, NT)
-        assert hi > lo, "empty CTA"
-        assert (owner[lo:hi] == g).all()
-    counts = np.bincount(owner, minlength=G)
-    assert counts.sum() == NT and counts.max() - counts.min() <= 1
-    slots = 0
-    for b, n in enumerate(tiles):
-        if n == 0:
+    assert len(items) <= grid + batch
+    ctas = items[:, 0]
+    assert (np.diff(ctas) >= 0).all(), "items listed CTA by CTA"
+    assert set(ctas.tolist()) == set(range(G)), "every CTA of the plan has work, no other"
+    # tiles per CTA differ by at most one
+    tiles = np.zeros(G, np.int64)
+    for cta, b, t0, t1, slot, ns, sp in items:
+        assert t0 % TILE == 0 and t1 > t0
+        tiles[cta] += (t1 + TILE - 1) // TILE - t0 // TILE
+    assert tiles.sum() == nt and tiles.max() - tiles.min() <= 1
+    # coverage, splits and slots per sequence
+    slots = []
+    for b in range(batch):
+        mine = items[items[:, 1] == b]
+        if not accepted[b]:
+            assert len(mine) == 0
             continue
-        ns = cta_of(int(start[b + 1]) - 1, G, NT) - cta_of(int(start[b]), G, NT) + 1
-        assert ns >= 1
-        slots += ns if ns > 1 else 0
-    assert slots <= grid + len(lens)
+        pos = 0
+        for k, (cta, _, t0, t1, slot, ns, sp) in enumerate(mine):
+            assert t0 == pos, f"sequence {b}: gap or overlap at {pos}"
+            pos = t1
+            assert ns == len(mine) and sp == k
+            if ns == 1:
+                assert slot == -1
+            else:
+                slots.append(slot)
+        assert pos == lens[b], f"sequence {b}: covered to {pos} of {lens[b]}"
+        if len(mine) > 1:
+            assert (np.diff(mine[:, 4]) == 1).all(), "a sequence's slots are consecutive"
+    assert len(set(slots)) == len(slots) and all(0 <= s < grid + batch for s in slots)
 
 
-@pytest.mark.parametrize("grid", [1, 7, 148, 296])
-def test_plan_covers_balances_and_fits_the_slots(grid):
+@pytest.mark.parametrize("grid", [1, 7, 148, 256])
+def test_device_plan_covers_balances_and_fits_the_slots(lib, grid):
     rng = np.random.default_rng(grid)
     for _ in range(150):
         batch = int(rng.integers(1, 300))
@@ -68,16 +106,21 @@ def test_plan_covers_balances_and_fits_the_slots(grid):
         elif kind == 2:  # mostly short, a few long
             lens = [int(x) if rng.random() < 0.9 else int(x) * 200
                     for x in rng.integers(1, 300, batch)]
-        else:            # with rejected (zero-length) sequences
+        else:            # with rejected sequences: length 0, or beyond a smaller capacity
             lens = [int(x) if rng.random() < 0.8 else 0 for x in rng.integers(1, 5000, batch)]
-        _check(lens, grid)
+            caps = [max(1, L) if rng.random() < 0.9 else max(1, L // 2) for L in lens]
+            _check(lib, lens, grid, caps)
+            continue
+        _check(lib, lens, grid)
 
 
-def test_plan_edge_cases():
-    _check([1], 148)                      # one tile: one CTA
-    _check([0, 0, 0], 148)                # all rejected: no work
-    _check([65536], 148)                  # one sequence over every CTA
-    _check([128] * 148, 148)              # one tile per CTA, no split
-    _check([129] * 148, 148)              # two tiles per sequence over 148 CTAs
-    _check([1] * 1024, 148)               # the largest batch
-    _check([65536] * 16, 148)
+def test_device_plan_edge_cases(lib):
+    _check(lib, [1], 148)                      # one tile: one CTA
+    _check(lib, [0, 0, 0], 148)                # all rejected: no work
+    _check(lib, [65536], 148)                  # one sequence over every CTA
+    _check(lib, [128] * 148, 148)              # one tile per CTA, no split
+    _check(lib, [129] * 148, 148)              # two tiles per sequence over 148 CTAs
+    _check(lib, [1] * 1024, 148)               # the largest batch
+    _check(lib, [65536] * 16, 148)
+    _check(lib, [4096] * 32, 148)              # the 4K workload: 6.92 tiles per CTA
+    _check(lib, [300, 0, 65536, 2], 148, caps=[300, 10, 65536, 1])  # 2 > capacity 1
