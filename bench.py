@@ -62,6 +62,12 @@ def parse_args():
                         "scale per 128 x 128 block; the layer uses bf16(code * scale))")
     p.add_argument("--page-order", choices=["shuffled", "sequential"], default="shuffled",
                    help="with --page-size: pages handed out in random or in sequence order")
+    p.add_argument("--passes", type=int, default=0,
+                   help="timed passes of --steps steps each (default: enough for about "
+                        "0.25 s of timed work, at least 5); the value is the median pass")
+    p.add_argument("--no-extra-workloads", action="store_true",
+                   help="time the chosen workload only (by default a single-GPU run of the "
+                        "default workload also times the 8K, FP8 and ragged workloads)")
     p.add_argument("--layers", type=int, default=0,
                    help="time the attention side of a whole decode step instead: this many "
                         "layers, each the MFA decode step plus its output projection")
@@ -237,7 +243,40 @@ def kv_bytes(inp) -> int:
     return 2 * row * int(inp.seq_lens.sum())
 
 
-def run_ours(args, wl, rank, world, local):
+def timed_passes(run_pass, passes, world, dev):
+    """Run `passes` timed passes. Each pass is bracketed by a barrier and a synchronize on
+    both sides; run_pass records its own CUDA events on the stream(s) it launches on and
+    returns the elapsed device time (ms). Per pass, the slowest rank's time."""
+    import torch
+    out = []
+    for _ in range(passes):
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        ms = run_pass()
+        if world > 1:
+            torch.distributed.barrier()
+        out.append(max_over_ranks(ms, world, dev))
+    return out
+
+
+def pick_passes(args, pass_ms_estimate: float) -> int:
+    """Passes of K steps: --passes if given, else enough for about 0.25 s of timed work (so
+    the clock samples cover a steady state), at least 5 and at most 300."""
+    if args.passes > 0:
+        return args.passes
+    return int(min(300, max(5, math.ceil(250.0 / max(pass_ms_estimate, 1e-3)))))
+
+
+def pass_summary(times):
+    return {"passes": len(times), "median_ms": statistics.median(times), "min_ms": min(times),
+            "max_ms": max(times)}
+
+
+def run_ours(args, wl, rank, world, local, headline=True):
+    """Measure one workload: the whole decode step (CUDA-graph replay, inputs resident in
+    HBM), the attention call alone, and (headline only) the end-to-end public call with
+    host copies and the CPU oracle baseline."""
     import torch
     from decode_attention_10_b200 import build, mfa
     from decode_attention_10_b200 import workloads as W
@@ -250,6 +289,7 @@ def run_ours(args, wl, rank, world, local):
     bsz = inp.batch
     step_bytes = (WEIGHT_BYTES // (2 if args.weights == "fp8" else 1)) + kv_bytes(inp)
     copies = max(2, math.ceil(3 * L2_BYTES / step_bytes))
+    K = args.steps
 
     class Copy:
         pass
@@ -285,15 +325,8 @@ def run_ours(args, wl, rank, world, local):
     for c in sets:
         c.step = mfa.DecodeStep(c.x, *c.w, c.cache, lens, c.q, c.out, ws)
 
-    def layer(c):
-        c.step()
-
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
     for i in range(args.warmup):
-        layer(sets[i % copies])
+        sets[i % copies].step()
     torch.cuda.synchronize()
     if mfa.get_error(ws) != 0:
         raise RuntimeError("device error flag set during warm-up")
@@ -305,7 +338,7 @@ def run_ours(args, wl, rank, world, local):
     n_host = 50
     h0 = time.perf_counter()
     for i in range(n_host):
-        layer(sets[i % copies])
+        sets[i % copies].step()
     host_us = (time.perf_counter() - h0) / n_host * 1e6
     torch.cuda.synchronize()
 
@@ -326,90 +359,39 @@ def run_ours(args, wl, rank, world, local):
         graphs[i % copies].replay()
     torch.cuda.synchronize()
 
-    # 1) the timed region: K whole decode steps (graph replays)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        e0.record()
-        for i in range(args.steps):
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def graph_pass():
+        ev[0].record()
+        for i in range(K):
             graphs[i % copies].replay()
-        e1.record()
+        ev[1].record()
         torch.cuda.synchronize()
-    barrier()
-    t_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    ms_per_step = t_ms / args.steps
-    value = whole_job_throughput(world, bsz, args.steps, t_ms)
+        return ev[0].elapsed_time(ev[1])
 
-    # 2) the attention launch alone: K launches back to back over the rotating copies, CUDA
-    #    events on the launching stream around the run (inter-launch gaps included)
-    for i in range(2):
-        c = sets[i % copies]
-        mfa.decode_attn(c.q, c.cache, lens, out=c.out, ws=ws)
-    torch.cuda.synchronize()
-    a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a0.record()
-    for i in range(args.steps):
-        c = sets[i % copies]
-        mfa.decode_attn(c.q, c.cache, lens, out=c.out, ws=ws)
-    a1.record()
-    torch.cuda.synchronize()
-    attn_ms = a0.elapsed_time(a1) / args.steps
+    def attn_pass():
+        ev[0].record()
+        for i in range(K):
+            c = sets[i % copies]
+            mfa.decode_attn(c.q, c.cache, lens, out=c.out, ws=ws)
+        ev[1].record()
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1])
 
-    # 3) end to end through the public call with host buffers: every step copies its x and
-    #    seq_lens in from pinned host memory and reads its output back, as a serving loop
-    #    does. A copy stream moves step i+1's inputs and step i's output while steps i and
-    #    i+1 compute (two buffer sets; events keep every buffer's writes and reads ordered).
-    x_host = [inp.x.pin_memory() for _ in range(copies)]
-    out_host = [torch.empty(bsz, 64, 256, dtype=torch.bfloat16).pin_memory()
-                for _ in range(copies)]
-    lens_host = inp.seq_lens.pin_memory()
-    comp, copy_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    for c in sets:
-        c.lens_e = torch.empty_like(lens)
-        c.step_e = mfa.DecodeStep(c.x, *c.w, c.cache, c.lens_e, c.q, c.out, ws, stream=comp)
-    h_evt = [torch.cuda.Event() for _ in range(copies)]
-    c_evt = [torch.cuda.Event() for _ in range(copies)]
-    d_evt = [torch.cuda.Event() for _ in range(copies)]
+    # 1) the timed region: passes of exactly K whole decode steps (graph replays); the
+    #    value is the median pass, the clocks are sampled across all passes
+    passes = pick_passes(args, max_over_ranks(graph_pass(), world, dev))  # same on every rank
+    with ClockSampler(local) as clk:
+        step_times = timed_passes(graph_pass, passes, world, dev)
+    t_ms = statistics.median(step_times)
+    ms_per_step = t_ms / K
+    value = whole_job_throughput(world, bsz, K, t_ms)
 
-    def h2d(i):  # on copy_s: step i's inputs, once step i - copies no longer reads the set
-        k = i % copies
-        if i >= copies:
-            copy_s.wait_event(c_evt[k])
-        sets[k].x.copy_(x_host[k], non_blocking=True)
-        sets[k].lens_e.copy_(lens_host, non_blocking=True)
-        h_evt[k].record(copy_s)
-
-    barrier()
-    torch.cuda.synchronize()
-    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(copy_s):
-        e2.record(copy_s)
-        h2d(0)
-    for i in range(args.steps):
-        k = i % copies
-        with torch.cuda.stream(copy_s):
-            if i + 1 < args.steps:
-                h2d(i + 1)
-        comp.wait_event(h_evt[k])
-        if i >= copies:
-            comp.wait_event(d_evt[k])  # step i - copies' output has been read back
-        sets[k].step_e()
-        c_evt[k].record(comp)
-        with torch.cuda.stream(copy_s):
-            copy_s.wait_event(c_evt[k])
-            out_host[k].copy_(sets[k].out, non_blocking=True)
-            d_evt[k].record(copy_s)
-    with torch.cuda.stream(copy_s):
-        e3.record(copy_s)
-    torch.cuda.synchronize()
-    barrier()
-    # each set computes the same inputs every step: what was read back must be its output
-    for k in range(min(copies, args.steps)):
-        if not torch.equal(out_host[k], sets[k].out.cpu()):
-            raise RuntimeError("e2e: an output read back differs from the step's result")
-    t_e2e = max_over_ranks(e2.elapsed_time(e3), world, dev)
-    e2e_value = whole_job_throughput(world, bsz, args.steps, t_e2e)
+    # 2) the attention launch alone: K calls back to back over the rotating copies, CUDA
+    #    events on the launching stream around each pass (inter-launch gaps included)
+    attn_pass()
+    attn_times = timed_passes(attn_pass, max(5, passes // 2), world, dev)
+    attn_ms = statistics.median(attn_times) / K
 
     peak, peak_kind = measured_peaks()
     a_bytes = attention_bytes(inp)
@@ -417,7 +399,7 @@ def run_ours(args, wl, rank, world, local):
     traffic = None if args.page_size else profiled_traffic(wl.name)
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if inp.kv_dtype == "bf16" else "bf16+fp8kv", "data": "synthetic",
         "config": {"workload": wl.name, "batch_per_gpu": bsz, "global_batch": bsz * world,
@@ -444,16 +426,94 @@ def run_ours(args, wl, rank, world, local):
                                                      else 2),
                                          ms_per_step / 1e3, peak, measured_tensor_peak()),
         "clocks": clk.summary(),
-        "e2e": {"value": e2e_value, "unit": UNIT,
-                "h2d_bytes_per_step": bsz * 7168 * 2 + bsz * 4,
-                "d2h_bytes_per_step": bsz * 64 * 256 * 2},
-        "gpu_launches": LAUNCHES_PER_LAYER * args.steps,
+        "step_passes": pass_summary(step_times),
+        "attn_passes": pass_summary(attn_times),
+        "gpu_launches": LAUNCHES_PER_LAYER * K,
         "host_us_per_call": host_us,
-        "timing": "value: CUDA-graph replay of the whole step; e2e: one public-API call "
-                  "per step plus the copies of each step's inputs in and output back, on a "
-                  "copy stream overlapping the neighbouring steps' compute; attn: "
-                  "back-to-back launches",
     }
+    if not headline:
+        return result
+
+    # 3) end to end through the public call with host buffers: every step copies its x and
+    #    seq_lens in from pinned host memory (one copy: x and seq_lens are adjacent in one
+    #    device buffer) and reads its output back, as a serving loop does. Inputs go in on
+    #    one copy stream and outputs come back on another, so the two directions use both
+    #    copy engines and overlap the neighbouring steps' compute (events keep every buffer's
+    #    writes and reads ordered; each set of buffers is reused every `copies` steps).
+    x_bytes = bsz * 7168 * 2
+    in_bytes = x_bytes + 4 * bsz
+    host_in = []
+    for c in sets:
+        buf = torch.empty(in_bytes + 256, dtype=torch.uint8, device=dev)
+        c.xe = buf[:x_bytes].view(torch.bfloat16).view(bsz, 7168)
+        c.lens_e = buf[x_bytes:in_bytes].view(torch.int32)
+        c.in_dev = buf[:in_bytes]
+        hb = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
+        hb[:x_bytes].view(torch.bfloat16).view(bsz, 7168).copy_(inp.x)
+        hb[x_bytes:].view(torch.int32).copy_(inp.seq_lens)
+        host_in.append(hb)
+    out_host = [torch.empty(bsz, 64, 256, dtype=torch.bfloat16).pin_memory()
+                for _ in range(copies)]
+    comp = torch.cuda.Stream(dev)
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    for c in sets:
+        c.step_e = mfa.DecodeStep(c.xe, *c.w, c.cache, c.lens_e, c.q, c.out, ws, stream=comp)
+    h_evt = [torch.cuda.Event() for _ in range(copies)]
+    c_evt = [torch.cuda.Event() for _ in range(copies)]
+    d_evt = [torch.cuda.Event() for _ in range(copies)]
+    e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def h2d(i):  # on h2d_s: step i's inputs, once step i - copies no longer reads the set
+        k = i % copies
+        if i >= copies:
+            h2d_s.wait_event(c_evt[k])
+        sets[k].in_dev.copy_(host_in[k], non_blocking=True)
+        h_evt[k].record(h2d_s)
+
+    def e2e_pass():
+        comp.wait_stream(torch.cuda.current_stream())
+        h2d_s.wait_stream(comp)
+        d2h_s.wait_stream(comp)
+        with torch.cuda.stream(h2d_s):
+            e2e_ev[0].record(h2d_s)
+            h2d(0)
+        for i in range(K):
+            k = i % copies
+            with torch.cuda.stream(h2d_s):
+                if i + 1 < K:
+                    h2d(i + 1)
+            comp.wait_event(h_evt[k])
+            if i >= copies:
+                comp.wait_event(d_evt[k])  # step i - copies' output has been read back
+            sets[k].step_e()
+            c_evt[k].record(comp)
+            with torch.cuda.stream(d2h_s):
+                d2h_s.wait_event(c_evt[k])
+                out_host[k].copy_(sets[k].out, non_blocking=True)
+                d_evt[k].record(d2h_s)
+        with torch.cuda.stream(d2h_s):
+            d2h_s.wait_stream(comp)
+            d2h_s.wait_stream(h2d_s)
+            e2e_ev[1].record(d2h_s)
+        torch.cuda.synchronize()
+        return e2e_ev[0].elapsed_time(e2e_ev[1])
+
+    e2e_pass()
+    e2e_times = timed_passes(e2e_pass, max(5, min(passes, 20)), world, dev)
+    # each set computes the same inputs every step: what was read back must be its output
+    for k in range(min(copies, K)):
+        if not torch.equal(out_host[k], sets[k].out.cpu()):
+            raise RuntimeError("e2e: an output read back differs from the step's result")
+    t_e2e = statistics.median(e2e_times)
+    result["e2e"] = {"value": whole_job_throughput(world, bsz, K, t_e2e), "unit": UNIT,
+                     "h2d_bytes_per_step": in_bytes,
+                     "d2h_bytes_per_step": bsz * 64 * 256 * 2,
+                     "passes": pass_summary(e2e_times)}
+    result["timing"] = ("value: median of passes of K CUDA-graph replays of the whole step; "
+                        "e2e: median of passes of K public-API calls, each step's inputs "
+                        "copied in and its output copied back on two copy streams that "
+                        "overlap the neighbouring steps' compute; attn: median of passes of "
+                        "K back-to-back mfa_decode_attn calls")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # whole decode steps of the first n_seq sequences, repeated until about 10 s of CPU
         # work (at most 20 repetitions)
@@ -467,6 +527,34 @@ def run_ours(args, wl, rank, world, local):
                                   "sample": f"{reps} whole decode steps of {n_seq} of the "
                                             f"{bsz} sequences (float64 numpy), {total:.1f} s"}
     return result
+
+
+def run_extra_workloads(args, rank, world, local):
+    """The other full-size workloads, measured the same way as the headline (whole step and
+    attention call; no host copies, no CPU baseline), each with its own clocks."""
+    import gc
+
+    import torch
+    from decode_attention_10_b200 import workloads as W
+    out = {}
+    gc.collect()
+    torch.cuda.empty_cache()
+    for name in EXTRA_WORKLOADS:
+        r = run_ours(args, W.workload(name), rank, world, local, headline=False)
+        out[name] = {k: r[k] for k in ("value", "ms_per_step", "attn_ms", "kv_gbs", "roofline",
+                                       "layer_roofline", "clocks", "step_passes",
+                                       "attn_passes")}
+        out[name]["config"] = {k: r["config"][k] for k in ("batch_per_gpu", "context",
+                                                           "kv_dtype", "kv_layout")}
+        gc.collect()
+        torch.cuda.empty_cache()
+    return out
+
+
+# The workloads timed after the headline in a default run: the 8K point of the metric, the
+# FP8 cache at 4K, and the ragged long-context batch.
+EXTRA_WORKLOADS = ("mfa_decode_b64_l8192_bf16", "mfa_decode_b128_l4096_fp8",
+                   "mfa_decode_b16_ragged64k_bf16")
 
 
 LAUNCHES_PER_LAYER = 5  # x-projection, split-K finish (+RMSNorm, append, split plan), q_up,
@@ -657,6 +745,9 @@ def main():
             res = run_stack(args, wl, rank, world, local)
         else:
             res = run_ours(args, wl, rank, world, local)
+            if (world == 1 and wl.name == DEFAULT_WORKLOAD and not args.no_extra_workloads
+                    and not args.page_size and args.weights == "bf16"):
+                res["workloads"] = run_extra_workloads(args, rank, world, local)
     finally:
         if world > 1:
             import torch

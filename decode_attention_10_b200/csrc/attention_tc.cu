@@ -1146,9 +1146,10 @@ size_t attention_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
 template <bool kFp8, bool kPaged>
 static cudaError_t launch_tc(const CUtensorMap& q_map, const AttnArgs& a, cudaStream_t s) {
   const size_t smem = attention_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attention_tc_kernel<kFp8, kPaged>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static std::atomic<uint64_t> smem_set{0};
+  if (!set_smem_limit_once(reinterpret_cast<const void*>(attention_tc_kernel<kFp8, kPaged>),
+                           (int)smem, &smem_set))
+    return cudaErrorInvalidValue;
   return launch_pdl(attention_tc_kernel<kFp8, kPaged>, dim3(a.grid), dim3(Cfg<kFp8>::kThreads), smem, s,
                     q_map, a);
 }

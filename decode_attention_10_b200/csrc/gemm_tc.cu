@@ -423,9 +423,11 @@ cudaError_t launch_wgemm_t(const CUtensorMap* w, const CUtensorMap& xmap, WGemmA
   }
   p.tmem_cols = cols;
   const size_t smem = 1024 + (size_t)stages * stage_bytes + sizeof(GemmCtl);
-  cudaError_t e = cudaFuncSetAttribute(wgemm_kernel<kW8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  // the limit is set once per device to the most any launch asks for
+  static std::atomic<uint64_t> smem_set{0};
+  if (smem > (size_t)kMaxSmem ||
+      !set_smem_limit_once(reinterpret_cast<const void*>(wgemm_kernel<kW8>), kMaxSmem, &smem_set))
+    return cudaErrorInvalidValue;
   const int rows = kW8 ? kMaxW8Rows : 256;
   dim3 grid(m_tiles, splits, (p.batch + rows - 1) / rows);
   return launch_pdl(wgemm_kernel<kW8>, grid, dim3(kThreads), smem, s, w[0], w[1], w[2], xmap,

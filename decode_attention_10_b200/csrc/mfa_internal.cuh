@@ -3,6 +3,8 @@
 
 #include <cuda.h>  // CUtensorMap (type only; the driver is reached through the runtime)
 #include <cuda_runtime.h>
+
+#include <atomic>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -239,6 +241,19 @@ size_t attention_tc_smem_bytes();
 // dependent.
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s);
 
+// One CTA whose bounded wait on a barrier that nothing completes gives up after limit_us
+// and sets kErrTimeout in *err (selftest.cu).
+cudaError_t launch_wait_selftest(uint32_t* err, uint32_t limit_us, cudaStream_t s);
+
+// The status a set of device error bits reports (the most specific bit wins).
+inline mfa_status status_of_error_bits(uint32_t bits) {
+  if (bits == 0) return MFA_OK;
+  if (bits & kErrCapacity) return MFA_ERR_CAPACITY;
+  if (bits & kErrEmpty) return MFA_ERR_EMPTY;
+  if (bits & kErrLayout) return MFA_ERR_INVALID_ARG;
+  return MFA_ERR_TIMEOUT;
+}
+
 // A projection weight: bf16 stored [in, out] (scales null), or block-FP8 e4m3 codes stored
 // [out, in] with one float32 scale per 128 x 128 block ([out / 128, in / 128]).
 struct WRef {
@@ -258,9 +273,13 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn encode_tiled_fn();
 // 2-D bf16/uint8 tensor map over a row-major [rows, cols] matrix, box [box_cols, box_rows],
-// 128-byte swizzle. Returns false if the driver rejects it.
+// 128-byte swizzle. Returns false if the driver rejects it. Maps already encoded on this
+// host thread (same address, shape and box) are copied from a small per-thread cache.
 bool encode_2d(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, int elem_bytes,
                uint32_t box_cols, uint32_t box_rows);
+// Raise `kernel`'s dynamic shared memory limit to `bytes` (the most any launch of it asks
+// for) on the current device, once per device; `done` is the kernel's per-device record.
+bool set_smem_limit_once(const void* kernel, int bytes, std::atomic<uint64_t>* done);
 // 3-D map over a page pool [pages, page_rows, 256] (elem_bytes each), box
 // [128 bytes of a row x box_rows x 1 page], 128-byte swizzle.
 bool encode_pool(CUtensorMap* m, const void* base, uint64_t pages, uint64_t page_rows,

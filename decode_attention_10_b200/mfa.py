@@ -56,6 +56,9 @@ _SIGNATURES = {
     "mfa_query_proj_noalloc": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_float, _P,
                                               ctypes.c_int32, _P]),
     "mfa_wait_selftest": (ctypes.c_int, [_P, ctypes.c_size_t, ctypes.c_uint32, _P]),
+    "mfa_query_proj_noalloc_get_error": (ctypes.c_int, [_P]),
+    "mfa_split_plan": (ctypes.c_int, [_P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
+    "mfa_query_proj_noalloc_wait_selftest": (ctypes.c_int, [ctypes.c_uint32, _P]),
 }
 NOALLOC_MAX_BATCH = 32
 
@@ -338,6 +341,26 @@ def query_proj_noalloc(x, w_qdown, gamma, w_qup, eps: float = 1e-6, q_out=None, 
                                       float(eps), _ptr(q_out), bsz, _stream(stream)),
            "mfa_query_proj_noalloc")
     return q_out
+
+
+def split_plan(cache, seq_lens: torch.Tensor, grid: int, stream=None):
+    """The attention's split plan as the device builds it (mfa_split_plan): returns
+    (G, NT, items) with items an int tensor [n, 7] of (cta, sequence, tok0, tok1, slot,
+    nsplit, split)."""
+    n_max = int(grid) + cache.batch
+    buf = torch.zeros(3 + 8 * n_max, dtype=torch.int32, device=seq_lens.device)
+    _check(load().mfa_split_plan(ctypes.byref(cache.desc), _ptr(seq_lens), int(grid),
+                                 _ptr(buf), buf.numel() * 4, _stream(stream)),
+           "mfa_split_plan")
+    host = buf.cpu()
+    n = int(host[2])
+    return int(host[0]), int(host[1]), host[3:3 + 8 * n].view(n, 8)[:, :7]
+
+
+def noalloc_get_error(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status of the calls of
+    query_proj_noalloc on the current device."""
+    return load().mfa_query_proj_noalloc_get_error(_stream(stream))
 
 
 def wait_selftest(ws: Workspace, limit_us: int = 1000, stream=None) -> None:

@@ -278,14 +278,29 @@ MFA_API mfa_status mfa_o_proj(const void* out, const void* w_o, void* y, int32_t
  *     small for it); batch < 1, eps <= 0 or a null/misaligned pointer return
  *     MFA_ERR_INVALID_ARG. Nothing is enqueued in either case.
  *   - The first call on a device looks up the array's device address on that device (it
- *     must be the current device); make that first call before any stream capture.
+ *     must be the current device) and keeps it for the rest of the process; make that first
+ *     call before any stream capture. A device reset (cudaDeviceReset) unloads the array, so
+ *     this call must not be used on that device again afterwards.
  *   - Every call on a device uses the same array, which keeps the last call's contents.
  *     Calls that can run at the same time on the GPU (unordered streams, several host
  *     threads) race on it and corrupt each other's results: order them on one stream.
- *   - The device-side error word is cleared at the start of each call and not reported. */
+ *   - Device-side errors (a bounded wait that expired) set bits in the array's error word,
+ *     which stays set across calls until mfa_query_proj_noalloc_get_error reads it. */
 MFA_API mfa_status mfa_query_proj_noalloc(const void* x, const void* w_qdown, const void* gamma,
                                           const void* w_qup, float eps, void* q_out,
                                           int32_t batch, void* stream);
+
+/* The device-side status of mfa_query_proj_noalloc on the current device: synchronizes
+ * `stream`, then returns and clears the error word of the built-in scratch (MFA_OK,
+ * or MFA_ERR_TIMEOUT if a bounded wait expired in a call since the last read). It allocates
+ * nothing. Like the calls it reports on, it must not overlap them on another stream. */
+MFA_API mfa_status mfa_query_proj_noalloc_get_error(void* stream);
+
+/* Diagnostic for mfa_query_proj_noalloc_get_error (no counterpart on the Step-3 pages):
+ * enqueues the kernel of mfa_wait_selftest on the built-in scratch's error word, so that
+ * the next mfa_query_proj_noalloc_get_error returns MFA_ERR_TIMEOUT. limit_us as for
+ * mfa_wait_selftest (1 .. 1,000,000; otherwise MFA_ERR_INVALID_ARG, nothing enqueued). */
+MFA_API mfa_status mfa_query_proj_noalloc_wait_selftest(uint32_t limit_us, void* stream);
 
 /* ---------------------------------------------------------------------------------------
  * Diagnostics
@@ -304,6 +319,24 @@ MFA_API mfa_status mfa_query_proj_noalloc(const void* x, const void* w_qdown, co
  *   of range (nothing enqueued), MFA_ERR_CUDA if the launch fails. */
 MFA_API mfa_status mfa_wait_selftest(void* ws, size_t ws_bytes, uint32_t limit_us,
                                      void* stream);
+
+/* The length-aware split plan of the decode attention (the scheduler that balances the K/V
+ * stream over the persistent grid; see mfa_decode_attn), as the device builds it for the
+ * lengths in `seq_lens` (device int32 [kv->batch]) and the capacities in kv's table, for a
+ * grid of `grid` CTAs (1 .. 256; the attention itself uses one CTA per SM). The plan cuts
+ * every accepted sequence (1 <= length <= capacity) into tiles of 128 positions, lays them
+ * end to end and gives CTA g the tiles [g NT / G, (g + 1) NT / G), G = min(grid, NT); the part
+ * of a sequence inside one CTA's range is a work item. Rejected sequences have no items.
+ *   out: device int32 buffer of at least 3 + 8 (grid + batch) entries, written as
+ *     out[0] = G, out[1] = NT, out[2] = n (work items), then item i at out[3 + 8 i]:
+ *     (cta, sequence, first position, one past the last, partial slot or -1 when the
+ *     sequence is finished by this item alone, CTAs sharing the sequence, this item's index
+ *     among them, 0). Items are listed CTA by CTA, each CTA's in the order it streams them.
+ *   Returns MFA_ERR_INVALID_ARG (null or misaligned pointer, batch or grid out of range),
+ *   MFA_ERR_WORKSPACE (out too small), MFA_ERR_CUDA (launch failure); asynchronous on
+ *   `stream` otherwise. */
+MFA_API mfa_status mfa_split_plan(const mfa_kv_cache* kv, const int32_t* seq_lens,
+                                  int32_t grid, int32_t* out, size_t out_bytes, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */
