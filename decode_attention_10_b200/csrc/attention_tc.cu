@@ -119,6 +119,8 @@ struct __align__(1024) TcSmem {
   uint8_t p[kPBytes];
   PlanSmem plan;
   float m_used[kHeads];
+  float m_thr[kHeads];  // m_used + the rescale threshold: a score above it needs a rescale
+  float m_p[kHeads];    // m_used - the P exponent offset: P = 2^(s - m_p)
   float alpha[kHeads];
   float red[4][kHeads];
   float lsum[kHeads];
@@ -196,13 +198,6 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
-}
-
-__device__ __forceinline__ float f16_lo(uint32_t w) {
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)));
-}
-__device__ __forceinline__ float f16_hi(uint32_t w) {
-  return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -632,19 +627,11 @@ __device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
 // A pair of values (f16x2, |v| <= 256) as e4m3 hi and lo parts: hi = e4m3(v), lo =
-// e4m3(v - hi); returns hi + lo (f16x2, exact: both parts and their sum fit f16).
-__device__ __forceinline__ uint32_t split_e4m3x2(uint32_t v, uint16_t& hi, uint16_t& lo) {
+// e4m3(v - hi) (v - hi is exact in f16).
+__device__ __forceinline__ void split_e4m3x2(uint32_t v, uint16_t& hi, uint16_t& lo) {
   hi = f16x2_to_e4m3x2(v);
-  const uint32_t hf = e4m3x2_to_f16x2(hi);
-  lo = f16x2_to_e4m3x2(hsub2_u32(v, hf));
-  return hadd2_u32(hf, e4m3x2_to_f16x2(lo));
+  lo = f16x2_to_e4m3x2(hsub2_u32(v, e4m3x2_to_f16x2(hi)));
 }
 
 // Q of work item `item` (bf16, four TMA boxes of [64 heads x 64 dims]) -> in place, two
@@ -758,7 +745,9 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
 
   plan_for_each_item(S.plan, a.batch, g, [&](const WorkItem& it) {
     const int n = num_tiles(it);
-    float lsum_w = 0.f;  // this warp's running row sum of head h0 + sum_head
+    // this thread's running sums of P over the positions it has held, per head of its group
+    // (taken across the 128 positions only once, at the end of the item)
+    float lacc[GH];
     float s_mul = s_mul0;
     if constexpr (kFp8) {
       // Q split into e4m3 hi and lo parts scaled by 2^-e, so the scores carry 2^e
@@ -772,6 +761,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       const uint32_t tile = gt + t, j = tile & 1, k = tile >> 1;
       const int pos = y + row;
       const bool valid = pos >= a0 && pos < e0;
+      const bool full = y >= a0 && y + kTile <= e0;  // every position of the window is used
 
       mbar_wait(&S.s_full[j], k & 1, abort);
       tc_fence_after();
@@ -783,30 +773,32 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
         tmem_wait_ld();
 #pragma unroll
         for (int h = 0; h < GH; ++h) s[h] = __uint_as_float(sr[h]);
-        if constexpr (kFp8) {  // plus the lo parts' scores, 64 columns on
-          tmem_ld_cols<GH>(sa + 64, sr);
-          tmem_wait_ld();
+        if constexpr (kFp8) {  // plus the lo parts' scores, 64 columns on (16 at a time)
 #pragma unroll
-          for (int h = 0; h < GH; ++h) s[h] += __uint_as_float(sr[h]);
+          for (int q = 0; q < GH / 16; ++q) {
+            uint32_t lr[16];
+            tmem_ld_cols<16>(sa + 64 + 16 * q, lr);
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < 16; ++h) s[16 * q + h] += __uint_as_float(lr[h]);
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.s_free[j]);
 
-#pragma unroll
-      for (int h = 0; h < GH; ++h) s[h] = valid ? s[h] * s_mul : -INFINITY;
-
+      // s holds the raw products; the scaled score of head h is s[h] * s_mul (log2 units)
       bool need = (t == 0);
-      if (!need) {
+      if (!need && valid) {
 #pragma unroll
-        for (int h = 0; h < GH; ++h) need |= s[h] > S.m_used[h0 + h] + C::kRescaleThreshold;
+        for (int h = 0; h < GH; ++h) need |= fmaf(s[h], s_mul, -S.m_thr[h0 + h]) > 0.f;
       }
       if (named_bar_or(gbar, kGroupThreads, need)) {
         // exact per-head max of this tile across the 128 positions
 #pragma unroll
         for (int h = 0; h < GH; ++h) {
-          const float r = warp_max_f32(s[h]);
+          const float r = warp_max_f32(valid ? s[h] * s_mul : -INFINITY);
           if (lane == 0) S.red[quad][h0 + h] = r;
         }
         named_bar_sync(gbar, kGroupThreads);
@@ -817,70 +809,90 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
           const float mn = fmaxf(mo, mt);
           S.alpha[hh] = exp2f(mo - mn);
           S.m_used[hh] = mn;
+          S.m_thr[hh] = mn + C::kRescaleThreshold;
+          S.m_p[hh] = mn - C::kPExp;
         }
         named_bar_sync(gbar, kGroupThreads);
-        if (t > 0) {
-          lsum_w *= S.alpha[h0 + sum_head];
+        if (t == 0) {
+#pragma unroll
+          for (int h = 0; h < GH; ++h) lacc[h] = 0.f;
+        } else {
+#pragma unroll
+          for (int h = 0; h < GH; ++h) lacc[h] *= S.alpha[h0 + h];
           // O must hold PV(t-1) before it is rescaled
           mbar_wait(&S.p_free, (tile - 1) & 1, abort);
           tc_fence_after();
           // each O^T half (FP8: its hi and its lo columns)
 #pragma unroll 1
-          for (int hp = 0; hp < (kFp8 ? 4 : 2); ++hp) {
-            uint32_t o[GH];
-            const uint32_t addr =
-                tmem + lane_addr + C::kTmemO + C::kSCols * (hp & 1) + 64 * (hp >> 1) + h0;
-            tmem_ld_cols<GH>(addr, o);
+          // (16 columns at a time: the scores and running sums are live here too)
+          for (int hp = 0; hp < (kFp8 ? 4 : 2) * (GH / 16); ++hp) {
+            uint32_t o[16];
+            const int q = hp % (GH / 16), hq = hp / (GH / 16);
+            const uint32_t addr = tmem + lane_addr + C::kTmemO + C::kSCols * (hq & 1) +
+                                  64 * (hq >> 1) + h0 + 16 * q;
+            tmem_ld_cols<16>(addr, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int h = 0; h < GH; ++h)
-              o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h0 + h]);
-            tmem_st_cols<GH>(addr, o);
+            for (int h = 0; h < 16; ++h)
+              o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h0 + 16 * q + h]);
+            tmem_st_cols<16>(addr, o);
           }
           tmem_wait_st();
         }
       }
 
       // probabilities, rounded to what the tensor core reads (bf16; for FP8 caches e4m3 hi
-      // and lo parts), this group's share of the P^T row, and the row sums of the rounded
-      // values
-      uint32_t pk[GH / 2];  // bf16: GH values; FP8: GH hi codes, then GH lo codes
-#pragma unroll
-      for (int h = 0; h < GH; h += 2) {
-        const float p0 = ex2(s[h] - (S.m_used[h0 + h] - C::kPExp));
-        const float p1 = ex2(s[h + 1] - (S.m_used[h0 + h + 1] - C::kPExp));
-        if constexpr (kFp8) {
-          uint16_t hi, lo;
-          const uint32_t w = split_e4m3x2(pack_f16x2(p0, p1), hi, lo);
-          if ((h & 2) == 0) {
-            pk[h / 4] = hi;
-            pk[GH / 4 + h / 4] = lo;
-          } else {
-            pk[h / 4] |= static_cast<uint32_t>(hi) << 16;
-            pk[GH / 4 + h / 4] |= static_cast<uint32_t>(lo) << 16;
-          }
-          s[h] = f16_lo(w);
-          s[h + 1] = f16_hi(w);
-        } else {
-          const uint32_t w = pack_bf16x2(p0, p1);
-          pk[h / 2] = w;
-          s[h] = __uint_as_float(w << 16);
-          s[h + 1] = __uint_as_float(w & 0xFFFF0000u);
-        }
-      }
-      lsum_w += warp_transpose_sum<GH>(s, lane);
-      // the P^T buffer is free once PV(t-1) has read it
+      // and lo parts), this group's share of the P^T row, and the running sums: of the bf16
+      // values, or for FP8 caches of the float32 probabilities (the pair is within 2^-8 of
+      // each, and taking it apart again costs the softmax warps, which pace the FP8 tile)
+      // The P^T buffer is free once PV(t-1) has read it. Each 16-byte piece of this thread's
+      // 128-byte P^T row (positions are rows, 128-byte swizzle) is stored as soon as it is
+      // complete: bf16, heads 8 c .. 8 c + 7 in logical piece c; FP8, the hi codes of heads
+      // 16 c .. 16 c + 15 in piece c < 4 and their lo codes in piece 4 + c.
       if (tile >= 1) mbar_wait(&S.p_free, (tile - 1) & 1, abort);
-      // logical 16-byte pieces of the 128-byte row: bf16, heads 8 c .. 8 c + 7 in piece c;
-      // FP8, the hi codes of heads 16 c .. 16 c + 15 in piece c < 4, their lo codes in 4 + c
-      constexpr int kPieces = GH / 8;  // of this group
+      auto prob = [&](int h) {
+        const float p = ex2(fmaf(s[h], s_mul, -S.m_p[h0 + h]));
+        return (!full && !valid) ? 0.f : p;  // outside the item (also any NaN read there)
+      };
+      auto store_piece = [&](int cl, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+        *reinterpret_cast<uint4*>(p_row + ((cl ^ (row & 7)) << 4)) = make_uint4(w0, w1, w2, w3);
+      };
+      if constexpr (kFp8) {
 #pragma unroll
-      for (int c = 0; c < kPieces; ++c) {
-        const int cl = kFp8 ? (c < kPieces / 2 ? group * (kPieces / 2) + c
-                                               : 4 + group * (kPieces / 2) + (c - kPieces / 2))
-                            : group * kPieces + c;
-        uint4 v = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        *reinterpret_cast<uint4*>(p_row + ((cl ^ (row & 7)) << 4)) = v;
+        for (int c = 0; c < GH / 16; ++c) {
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int h = 16 * c + 2 * i;
+            const float p0 = prob(h), p1 = prob(h + 1);
+            uint16_t hi, lo;
+            split_e4m3x2(pack_f16x2(p0, p1), hi, lo);
+            if ((i & 1) == 0) {
+              hw[i / 2] = hi;
+              lw[i / 2] = lo;
+            } else {
+              hw[i / 2] |= static_cast<uint32_t>(hi) << 16;
+              lw[i / 2] |= static_cast<uint32_t>(lo) << 16;
+            }
+            lacc[h] += p0;
+            lacc[h + 1] += p1;
+          }
+          store_piece(group * (GH / 16) + c, hw[0], hw[1], hw[2], hw[3]);
+          store_piece(4 + group * (GH / 16) + c, lw[0], lw[1], lw[2], lw[3]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < GH / 8; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int h = 8 * c + 2 * i;
+            w[i] = pack_bf16x2(prob(h), prob(h + 1));
+            lacc[h] += __uint_as_float(w[i] << 16);
+            lacc[h + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+          }
+          store_piece(group * (GH / 8) + c, w[0], w[1], w[2], w[3]);
+        }
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -895,6 +907,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
     }
 
     // ---- epilogue of the item (each group for its heads) ----
+    const float lsum_w = warp_transpose_sum<GH>(lacc, lane);  // this warp's positions
     if (sum_owner) S.red[quad][h0 + sum_head] = lsum_w;
     named_bar_sync(gbar, kGroupThreads);
     if (gt_id < GH) {
@@ -914,13 +927,16 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
       const uint32_t oa = tmem + lane_addr + C::kTmemO + C::kSCols * hf + h0;
       tmem_ld_cols<GH>(oa, o);
       tmem_wait_ld();
-      if constexpr (kFp8) {  // O = (V . P_hi) + (V . P_lo)
-        uint32_t ol[GH];
-        tmem_ld_cols<GH>(oa + 64, ol);
-        tmem_wait_ld();
+      if constexpr (kFp8) {  // O = (V . P_hi) + (V . P_lo), the lo columns 16 at a time
 #pragma unroll
-        for (int h = 0; h < GH; ++h)
-          o[h] = __float_as_uint(__uint_as_float(o[h]) + __uint_as_float(ol[h]));
+        for (int q = 0; q < GH / 16; ++q) {
+          uint32_t ol[16];
+          tmem_ld_cols<16>(oa + 64 + 16 * q, ol);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 16; ++h)
+            o[16 * q + h] = __float_as_uint(__uint_as_float(o[16 * q + h]) + __uint_as_float(ol[h]));
+        }
       }
       const int d = hf * 128 + row;
       if (ok) {
