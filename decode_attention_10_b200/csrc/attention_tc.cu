@@ -1049,17 +1049,32 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// combine: one block per (sequence, group of 4 heads); thread t owns dims 2t and 2t + 1.
+// combine: one block per (sequence, group of 4 heads); each thread owns kHT of the 4 heads
+// and two dims, so a block has 4 / kHT * 128 threads.
 //   M[h] = max_i m_i[h],  L[h] = sum_i l_i[h] 2^(m_i[h] - M[h]),
 //   out[h][d] = v_mul / L[h] * sum_i 2^(m_i[h] - M[h]) acc_i[h][d].
-// Sequences finished by a single work item were written by the attention kernel; rejected
-// sequences (no split) get a zero output here.
+// Up to kOnePass(kHT) splits, every split's m, l and accumulators are loaded at once (one
+// round trip to L2); beyond that the weights go through shared memory first. Two shapes:
+// kHT = 2 (256 threads) for batches of few long sequences, which split many ways and need
+// their merge in one round trip; kHT = 4 (128 threads, fewer registers per block) for large
+// batches, whose many blocks must fit the SMs at once. Sequences finished by a single work
+// item were written by the attention kernel; rejected sequences (no split) get a zero
+// output here.
 // ---------------------------------------------------------------------------------------
 constexpr int kCombineHeads = 4;
-constexpr int kCombineOnePass = 8;      // up to this many splits: the one-pass merge
 constexpr int kCombineMaxSplits = kMaxAttnGrid;  // a sequence has at most grid splits
 
-__global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
+template <int kHT>
+struct CombineCfg {
+  static constexpr int kThreads = kCombineHeads / kHT * 128;
+  static constexpr int kOnePass = kHT == 2 ? 6 : 3;
+  static constexpr int kMinBlocks = kHT == 2 ? 4 : 8;
+};
+
+template <int kHT>
+__global__ void __launch_bounds__(CombineCfg<kHT>::kThreads, CombineCfg<kHT>::kMinBlocks)
+    attention_combine_kernel(AttnArgs a) {
+  using C = CombineCfg<kHT>;
   pdl_wait();
   pdl_launch_dependents();
   const int b = blockIdx.x, h0 = blockIdx.y * kCombineHeads, tid = threadIdx.x;
@@ -1067,94 +1082,109 @@ __global__ void __launch_bounds__(128) attention_combine_kernel(AttnArgs a) {
   const int base = info.x, ns = info.y;
   uint32_t* out = reinterpret_cast<uint32_t*>(a.out + (size_t)b * kQWidth + h0 * kHeadDim);
   if (ns == 0) {
-    for (int i = tid; i < kCombineHeads * kHeadDim / 2; i += 128) out[i] = 0u;
+    for (int i = tid; i < kCombineHeads * kHeadDim / 2; i += C::kThreads) out[i] = 0u;
     return;
   }
   if (ns == 1) return;
   const float v_mul = a.kv_dtype == MFA_KV_FP8_E4M3 ? a.v_scale : 1.f;
-  if (ns > kCombineOnePass && ns <= kCombineMaxSplits) {
-    // Many splits (long sequences): a pass with a running max would chain the splits' L2
-    // round trips. Instead: (1) every (split, head) pair's m and l in one round trip; (2)
-    // the weights v_mul 2^(m_i - M) / L per head, one warp per head; (3) the accumulators,
-    // whose loads no longer depend on any arithmetic, so many splits stay in flight.
-    __shared__ float sm[kCombineHeads][kCombineMaxSplits];
-    __shared__ float sl[kCombineHeads][kCombineMaxSplits];
-    for (int t = tid; t < kCombineHeads * ns; t += 128) {
-      const int i = t >> 2, h = t & 3;
-      sm[h][i] = __ldcg(partial_m(a.partials, base + i) + h0 + h);
-      sl[h][i] = __ldcg(partial_l(a.partials, base + i) + h0 + h);
-    }
-    __syncthreads();
-    {
-      const int h = tid >> 5, lane = tid & 31;  // warp h: head h0 + h
-      float mx = -INFINITY;
-      for (int i = lane; i < ns; i += 32) mx = fmaxf(mx, sm[h][i]);
-      mx = warp_max_f32(mx);
-      float ls = 0.f;
-      for (int i = lane; i < ns; i += 32) ls = fmaf(sl[h][i], exp2f(sm[h][i] - mx), ls);
+  const int hg = tid >> 7, hl = h0 + kHT * hg;  // this thread's first head
+  const int d2 = tid & 127;                     // dims 2 d2, 2 d2 + 1
+  uint32_t* o_out = out + (kHT * hg) * kHeadDim / 2 + d2;
+  auto head_of = [](const float4& v, int h) { return h == 0 ? v.x : h == 1 ? v.y : h == 2 ? v.z : v.w; };
+  auto ld_heads = [&](const float* p) {  // kHT consecutive floats from head hl on
+    if constexpr (kHT == 4) return __ldcg(reinterpret_cast<const float4*>(p + hl));
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p + hl));
+    return make_float4(v.x, v.y, 0.f, 0.f);
+  };
+  if (ns <= C::kOnePass) {
+    float4 mv[C::kOnePass], lv[C::kOnePass];
+    float2 xv[C::kOnePass][kHT];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
-      __syncwarp();
-      const float sc = v_mul / ls;
-      for (int i = lane; i < ns; i += 32) sl[h][i] = sc * exp2f(sm[h][i] - mx);  // weights
-    }
-    __syncthreads();
-    float2 o[kCombineHeads];
+    for (int i = 0; i < C::kOnePass; ++i) {
+      if (i < ns) {
+        mv[i] = ld_heads(partial_m(a.partials, base + i));
+        lv[i] = ld_heads(partial_l(a.partials, base + i));
+        const float* acc = partial_acc(a.partials, base + i) + hl * kHeadDim + 2 * d2;
 #pragma unroll
-    for (int h = 0; h < kCombineHeads; ++h) o[h] = make_float2(0.f, 0.f);
-#pragma unroll 8
-    for (int i = 0; i < ns; ++i) {
-      const float* acc = partial_acc(a.partials, base + i) + h0 * kHeadDim + 2 * tid;
-#pragma unroll
-      for (int h = 0; h < kCombineHeads; ++h) {
-        const float2 x = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
-        const float w = sl[h][i];
-        o[h].x = fmaf(w, x.x, o[h].x);
-        o[h].y = fmaf(w, x.y, o[h].y);
+        for (int h = 0; h < kHT; ++h)
+          xv[i][h] = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
       }
     }
 #pragma unroll
-    for (int h = 0; h < kCombineHeads; ++h) out[h * kHeadDim / 2 + tid] = pack_bf16x2(o[h].x, o[h].y);
+    for (int h = 0; h < kHT; ++h) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < C::kOnePass; ++i)
+        if (i < ns) M = fmaxf(M, head_of(mv[i], h));
+      float L = 0.f;
+      float2 o = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < C::kOnePass; ++i) {
+        if (i < ns) {
+          const float w = exp2f(head_of(mv[i], h) - M);
+          L = fmaf(head_of(lv[i], h), w, L);
+          o.x = fmaf(w, xv[i][h].x, o.x);
+          o.y = fmaf(w, xv[i][h].y, o.y);
+        }
+      }
+      const float inv = v_mul / L;
+      o_out[h * kHeadDim / 2] = pack_bf16x2(o.x * inv, o.y * inv);
+    }
     return;
   }
-  // few splits: one pass with a running max per head; every split's loads are independent
-  // of the arithmetic, so all splits' worth stay in flight
-  float M[kCombineHeads], L[kCombineHeads];
-  float2 o[kCombineHeads];
+  // More splits: (1) every (split, head) pair's m and l in one round trip; (2) the weights
+  // v_mul 2^(m_i - M) / L per head, one warp per head; (3) the accumulators, whose loads
+  // no longer depend on any arithmetic, so many splits stay in flight.
+  __shared__ float sm[kCombineHeads][kCombineMaxSplits];
+  __shared__ float sl[kCombineHeads][kCombineMaxSplits];
+  for (int t = tid; t < kCombineHeads * ns; t += C::kThreads) {
+    const int i = t >> 2, h = t & 3;
+    sm[h][i] = __ldcg(partial_m(a.partials, base + i) + h0 + h);
+    sl[h][i] = __ldcg(partial_l(a.partials, base + i) + h0 + h);
+  }
+  __syncthreads();
+  if (tid < 32 * kCombineHeads) {
+    const int h = tid >> 5, lane = tid & 31;  // warp h: head h0 + h
+    float mx = -INFINITY;
+    for (int i = lane; i < ns; i += 32) mx = fmaxf(mx, sm[h][i]);
+    mx = warp_max_f32(mx);
+    float ls = 0.f;
+    for (int i = lane; i < ns; i += 32) ls = fmaf(sl[h][i], exp2f(sm[h][i] - mx), ls);
 #pragma unroll
-  for (int h = 0; h < kCombineHeads; ++h) M[h] = -INFINITY, L[h] = 0.f, o[h] = make_float2(0.f, 0.f);
-#pragma unroll 4
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    __syncwarp();
+    const float sc = v_mul / ls;
+    for (int i = lane; i < ns; i += 32) sl[h][i] = sc * exp2f(sm[h][i] - mx);  // weights
+  }
+  __syncthreads();
+  float2 o[kHT];
+#pragma unroll
+  for (int h = 0; h < kHT; ++h) o[h] = make_float2(0.f, 0.f);
+#pragma unroll 8
   for (int i = 0; i < ns; ++i) {
-    const float4 m = __ldcg(reinterpret_cast<const float4*>(partial_m(a.partials, base + i) + h0));
-    const float4 l = __ldcg(reinterpret_cast<const float4*>(partial_l(a.partials, base + i) + h0));
-    const float* acc = partial_acc(a.partials, base + i) + h0 * kHeadDim + 2 * tid;
-    float2 x[kCombineHeads];
+    const float* acc = partial_acc(a.partials, base + i) + hl * kHeadDim + 2 * d2;
 #pragma unroll
-    for (int h = 0; h < kCombineHeads; ++h)
-      x[h] = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
-    const float mm[4] = {m.x, m.y, m.z, m.w}, ll[4] = {l.x, l.y, l.z, l.w};
-#pragma unroll
-    for (int h = 0; h < kCombineHeads; ++h) {
-      const float mn = fmaxf(M[h], mm[h]);
-      const float so = exp2f(M[h] - mn), si = exp2f(mm[h] - mn);
-      L[h] = fmaf(L[h], so, ll[h] * si);
-      o[h].x = fmaf(o[h].x, so, x[h].x * si);
-      o[h].y = fmaf(o[h].y, so, x[h].y * si);
-      M[h] = mn;
+    for (int h = 0; h < kHT; ++h) {
+      const float2 x = __ldcg(reinterpret_cast<const float2*>(acc + h * kHeadDim));
+      const float w = sl[kHT * hg + h][i];
+      o[h].x = fmaf(w, x.x, o[h].x);
+      o[h].y = fmaf(w, x.y, o[h].y);
     }
   }
 #pragma unroll
-  for (int h = 0; h < kCombineHeads; ++h) {
-    const float inv = v_mul / L[h];
-    out[h * kHeadDim / 2 + tid] = pack_bf16x2(o[h].x * inv, o[h].y * inv);
-  }
+  for (int h = 0; h < kHT; ++h) o_out[h * kHeadDim / 2] = pack_bf16x2(o[h].x, o[h].y);
 }
 
 }  // namespace
 
 cudaError_t launch_attention_combine(const AttnArgs& a, cudaStream_t s) {
-  return launch_pdl(attention_combine_kernel, dim3(a.batch, kHeads / kCombineHeads, 1), dim3(128),
-                    0, s, a);
+  // large batches split each sequence a few ways over the grid: many small merges, blocks
+  // with fewer registers so they all fit at once; small batches: few long sequences split
+  // many ways, each merge in one round trip
+  const dim3 grid(a.batch, kHeads / kCombineHeads, 1);
+  if (a.batch >= 64)
+    return launch_pdl(attention_combine_kernel<4>, grid, dim3(CombineCfg<4>::kThreads), 0, s, a);
+  return launch_pdl(attention_combine_kernel<2>, grid, dim3(CombineCfg<2>::kThreads), 0, s, a);
 }
 
 size_t attention_tc_smem_bytes() { return sizeof(TcSmem) + 1024; }
