@@ -428,7 +428,7 @@ def run_ours(args, wl, rank, world, local, headline=True):
         "clocks": clk.summary(),
         "step_passes": pass_summary(step_times),
         "attn_passes": pass_summary(attn_times),
-        "gpu_launches": LAUNCHES_PER_LAYER * K,
+        "gpu_launches": (LAUNCHES_PER_LAYER if args.weights == "bf16" else LAUNCHES_PER_LAYER_W8) * K,
         "host_us_per_call": host_us,
     }
     if not headline:
@@ -559,6 +559,7 @@ EXTRA_WORKLOADS = ("mfa_decode_b64_l8192_bf16", "mfa_decode_b128_l4096_fp8",
 
 LAUNCHES_PER_LAYER = 5  # x-projection, split-K finish (+RMSNorm, append, split plan), q_up,
 #                         attention, split combine
+LAUNCHES_PER_LAYER_W8 = 6  # FP8 weights: the same plus the quantization of x
 
 
 # The pages' per-stage budgets of a 50 ms TPOT pipeline, summed over the 61 layers (bud-325

@@ -56,6 +56,17 @@ struct alignas(128) KvSeq {
 };
 static_assert(sizeof(KvSeq) == 384, "KvSeq layout");
 
+// The element row, in its K or V buffer (or pool), of cache row `row` of sequence s: the
+// sequence's own row, or for a paged cache row % page_size of page pages[row / page_size].
+// -1 if the row is outside the sequence's capacity or its page outside the pool.
+__device__ inline long long kv_row_index(const KvSeq& s, int row) {
+  if (row < 0 || row >= s.capacity) return -1;
+  if (s.page_size == 0) return row;
+  const int page = s.pages[row / s.page_size];
+  if (page < 0 || page >= s.num_pages) return -1;
+  return static_cast<long long>(page) * s.page_size + row % s.page_size;
+}
+
 // Paged caches: rows per TMA box (a 128-position window is 128 / box rows boxes, each
 // inside one page).
 __host__ __device__ inline int paged_box_rows(int page_size) {

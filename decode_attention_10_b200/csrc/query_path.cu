@@ -122,20 +122,10 @@ __global__ void __launch_bounds__(kFinishThreads) xproj_finish_kernel(FinishArgs
   if (!do_kv) return;
   const int row = a.pos[b] - (a.pos_from_len ? 1 : 0);
   const KvSeq* s = a.kv + b;
-  if (row < 0 || row >= s->capacity) {
+  const long long at = kv_row_index(*s, row);  // -1: past the capacity or outside the pool
+  if (at < 0) {
     if (tid == 0) atomicOr(a.err, kErrCapacity);
     return;
-  }
-  // the row's index in the buffer: the sequence's own rows, or for a paged cache row
-  // row % page_size of page pages[row / page_size] of the pool
-  size_t at = (size_t)row;
-  if (s->page_size != 0) {
-    const int page = s->pages[row / s->page_size];
-    if (page < 0 || page >= s->num_pages) {
-      if (tid == 0) atomicOr(a.err, kErrCapacity);
-      return;
-    }
-    at = (size_t)page * s->page_size + row % s->page_size;
   }
   const bool is_v = tid >= kHeadDim;
   const int j = is_v ? tid - kHeadDim : tid;

@@ -187,6 +187,32 @@ def test_attention_long_sequence_split_over_many_ctas(kv_dtype):
     assert_close(out, ref, kv_dtype, "mixed long")
 
 
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+@pytest.mark.parametrize("shape", ["few_sequences", "large_batch"])
+def test_attention_every_combine_path(kv_dtype, shape):
+    # The combine merges a split sequence in one of four ways: batches under 64 sequences with
+    # 2 heads per thread, in one round trip up to 6 splits and through shared-memory weights
+    # beyond; batches of 64 and more with 4 heads per thread, one round trip up to 3 splits.
+    # Each case below reaches both ways of its shape (checked on the device's own plan).
+    from decode_attention_10_b200 import mfa
+    if shape == "few_sequences":
+        lens = [20000, 6000, 1500, 700, 520, 129, 64, 3]
+        one_pass_max = 6
+    else:
+        rng = np.random.default_rng(71)
+        lens = [30000, 8000, 2000] + rng.integers(250, 700, 45).tolist() + [1, 2] * 8
+        one_pass_max = 3
+    out, ref, cache = _attn_case(lens, kv_dtype, seed=70 if shape == "few_sequences" else 71)
+    _, _, items = mfa.split_plan(cache, torch.tensor(lens, dtype=torch.int32, device="cuda"),
+                                 torch.cuda.get_device_properties(0).multi_processor_count)
+    ns = {int(b): int(n) for b, n in zip(items[:, 1], items[:, 5])}
+    splits = set(ns.values())
+    assert any(2 <= n <= one_pass_max for n in splits), splits  # one round trip
+    assert any(n > one_pass_max for n in splits), splits        # two phases
+    assert 1 in splits                                          # finished in place
+    assert_close(out, ref, kv_dtype, f"combine paths ({shape})")
+
+
 def test_attention_one_workspace_across_differently_split_calls():
     # One workspace across calls whose sequences split differently (2 to 148 CTAs per
     # sequence, sequences finished by one CTA alone, lengths of 1 and 5). Each call rewrites
