@@ -23,10 +23,11 @@ and cache, the whole stack one CUDA graph; its line compares the time of 61 such
 the pages' per-stage budgets of a 50 ms TPOT pipeline.
 
 `--impl reference` times the float64 CPU oracle on this host's cores on a bounded sample
-of the same workload (the baseline of this build; there is no runnable reference code).
+of the same workload (the oracle is the baseline: the pages ship no runnable code).
 """
 
 import argparse
+import itertools
 import json
 import math
 import os
@@ -34,6 +35,7 @@ import statistics
 import sys
 import threading
 import time
+import types
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
@@ -342,8 +344,12 @@ def run_ours(args, wl, rank, world, local, headline=True):
     host_us = (time.perf_counter() - h0) / n_host * 1e6
     torch.cuda.synchronize()
 
-    # each copy's whole decode step captured once as a CUDA graph (the kernels, their
-    # arguments and tensor maps are recorded; replay re-runs exactly those launches)
+    # The K steps of a pass captured once as one CUDA graph over the rotating copies (the
+    # kernels, their arguments and tensor maps are recorded; replay re-runs exactly those
+    # launches). Inside it each step's first kernel is a programmatic dependent of the previous
+    # step's last, as consecutive layers are on a serving stream: it streams its first weight
+    # stages while the previous combine runs and reads x only once that step has completed.
+    # Each copy's step is also captured alone, for the isolated-step figure.
     graphs = []
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
@@ -354,14 +360,26 @@ def run_ours(args, wl, rank, world, local, headline=True):
             with torch.cuda.graph(g, stream=side):
                 c.gstep()
             graphs.append(g)
+        pass_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pass_graph, stream=side):
+            for i in range(K):
+                sets[i % copies].gstep()
     torch.cuda.current_stream().wait_stream(side)
     for i in range(max(args.warmup, 2)):
         graphs[i % copies].replay()
+    pass_graph.replay()
     torch.cuda.synchronize()
 
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
     def graph_pass():
+        ev[0].record()
+        pass_graph.replay()
+        ev[1].record()
+        torch.cuda.synchronize()
+        return ev[0].elapsed_time(ev[1])
+
+    def isolated_pass():
         ev[0].record()
         for i in range(K):
             graphs[i % copies].replay()
@@ -386,6 +404,10 @@ def run_ours(args, wl, rank, world, local, headline=True):
     t_ms = statistics.median(step_times)
     ms_per_step = t_ms / K
     value = whole_job_throughput(world, bsz, K, t_ms)
+
+    # the same K steps as K separate graph replays: no step overlaps its neighbours
+    isolated_pass()
+    iso_times = timed_passes(isolated_pass, max(5, passes // 2), world, dev)
 
     # 2) the attention launch alone: K calls back to back over the rotating copies, CUDA
     #    events on the launching stream around each pass (inter-launch gaps included)
@@ -427,6 +449,7 @@ def run_ours(args, wl, rank, world, local, headline=True):
                                          ms_per_step / 1e3, peak, measured_tensor_peak()),
         "clocks": clk.summary(),
         "step_passes": pass_summary(step_times),
+        "ms_per_step_isolated": statistics.median(iso_times) / K,
         "attn_passes": pass_summary(attn_times),
         "gpu_launches": (LAUNCHES_PER_LAYER if args.weights == "bf16" else LAUNCHES_PER_LAYER_W8) * K,
         "host_us_per_call": host_us,
@@ -436,39 +459,55 @@ def run_ours(args, wl, rank, world, local, headline=True):
 
     # 3) end to end through the public call with host buffers: every step copies its x and
     #    seq_lens in from pinned host memory (one copy: x and seq_lens are adjacent in one
-    #    device buffer) and reads its output back, as a serving loop does. Inputs go in on
-    #    one copy stream and outputs come back on another, so the two directions use both
-    #    copy engines and overlap the neighbouring steps' compute (events keep every buffer's
-    #    writes and reads ordered; each set of buffers is reused every `copies` steps).
+    #    device buffer) and reads its output back, inputs on one copy stream and outputs on
+    #    another. Each step's output goes back as soon as that step is done (an event record
+    #    on the compute stream, which does not hold the next step back); inputs go in by
+    #    groups of steps (1, then 4, then E2E_GROUP at a time, as the layers of a token step
+    #    run between its copies), and the compute stream waits for a group's inputs only
+    #    before the group, so inside a group each step chains to the previous one as in the
+    #    device-timed passes. Step i uses buffer i % n_buf; events order every reuse.
     x_bytes = bsz * 7168 * 2
     in_bytes = x_bytes + 4 * bsz
-    host_in = []
-    for c in sets:
+    n_buf = 2 * E2E_GROUP
+    comp = torch.cuda.Stream(dev)
+    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    bufs = []
+    for j in range(n_buf):
         buf = torch.empty(in_bytes + 256, dtype=torch.uint8, device=dev)
-        c.xe = buf[:x_bytes].view(torch.bfloat16).view(bsz, 7168)
-        c.lens_e = buf[x_bytes:in_bytes].view(torch.int32)
-        c.in_dev = buf[:in_bytes]
+        xe = buf[:x_bytes].view(torch.bfloat16).view(bsz, 7168)
+        lens_e = buf[x_bytes:in_bytes].view(torch.int32)
+        out_e = torch.empty(bsz, 64, 256, dtype=torch.bfloat16, device=dev)
         hb = torch.empty(in_bytes, dtype=torch.uint8).pin_memory()
         hb[:x_bytes].view(torch.bfloat16).view(bsz, 7168).copy_(inp.x)
         hb[x_bytes:].view(torch.int32).copy_(inp.seq_lens)
-        host_in.append(hb)
-    out_host = [torch.empty(bsz, 64, 256, dtype=torch.bfloat16).pin_memory()
-                for _ in range(copies)]
-    comp = torch.cuda.Stream(dev)
-    h2d_s, d2h_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    for c in sets:
-        c.step_e = mfa.DecodeStep(c.xe, *c.w, c.cache, c.lens_e, c.q, c.out, ws, stream=comp)
-    h_evt = [torch.cuda.Event() for _ in range(copies)]
-    c_evt = [torch.cuda.Event() for _ in range(copies)]
-    d_evt = [torch.cuda.Event() for _ in range(copies)]
+        bufs.append(types.SimpleNamespace(
+            in_dev=buf[:in_bytes], host_in=hb, out=out_e,
+            out_host=torch.empty(bsz, 64, 256, dtype=torch.bfloat16).pin_memory(),
+            # step i runs weight set i % copies on buffer i % n_buf: one bound call per set
+            step={k: mfa.DecodeStep(xe, *sets[k].w, sets[k].cache, lens_e, sets[k].q, out_e,
+                                    ws, stream=comp) for k in range(copies)},
+            c_evt=torch.cuda.Event(),  # its step computed (inputs consumed)
+            d_evt=torch.cuda.Event()))  # its output read back
+    groups, g0 = [], 0
+    for size in itertools.chain((1, 4), itertools.repeat(E2E_GROUP)):
+        if g0 >= K:
+            break
+        groups.append(range(g0, min(g0 + min(size, E2E_GROUP), K)))
+        g0 = groups[-1].stop
+    # two consecutive groups never hold more than n_buf steps, so the copies of group g + 1,
+    # enqueued before group g's calls, wait only for steps of groups before g, whose events
+    # are recorded (and not yet recorded again) by then
+    assert all(len(a) + len(b) <= n_buf for a, b in zip(groups, groups[1:]))
+    h_evt = [torch.cuda.Event() for _ in range(2)]  # inputs of group g in (by g % 2)
     e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
-    def h2d(i):  # on h2d_s: step i's inputs, once step i - copies no longer reads the set
-        k = i % copies
-        if i >= copies:
-            h2d_s.wait_event(c_evt[k])
-        sets[k].in_dev.copy_(host_in[k], non_blocking=True)
-        h_evt[k].record(h2d_s)
+    def h2d(gi):  # on h2d_s: group gi's inputs, each once its buffer's previous step is done
+        for i in groups[gi]:
+            b = bufs[i % n_buf]
+            if i >= n_buf:
+                h2d_s.wait_event(b.c_evt)
+            b.in_dev.copy_(b.host_in, non_blocking=True)
+        h_evt[gi % 2].record(h2d_s)
 
     def e2e_pass():
         comp.wait_stream(torch.cuda.current_stream())
@@ -477,20 +516,23 @@ def run_ours(args, wl, rank, world, local, headline=True):
         with torch.cuda.stream(h2d_s):
             e2e_ev[0].record(h2d_s)
             h2d(0)
-        for i in range(K):
-            k = i % copies
+        for gi, grp in enumerate(groups):
+            # the next group's inputs go in while this group computes; enqueued before this
+            # group's read-backs, which would otherwise hold them back in the copy queue
             with torch.cuda.stream(h2d_s):
-                if i + 1 < K:
-                    h2d(i + 1)
-            comp.wait_event(h_evt[k])
-            if i >= copies:
-                comp.wait_event(d_evt[k])  # step i - copies' output has been read back
-            sets[k].step_e()
-            c_evt[k].record(comp)
-            with torch.cuda.stream(d2h_s):
-                d2h_s.wait_event(c_evt[k])
-                out_host[k].copy_(sets[k].out, non_blocking=True)
-                d_evt[k].record(d2h_s)
+                if gi + 1 < len(groups):
+                    h2d(gi + 1)
+            comp.wait_event(h_evt[gi % 2])
+            if grp[-1] >= n_buf:  # the group's buffers' previous outputs have been read back
+                comp.wait_event(bufs[grp[-1] % n_buf].d_evt)
+            for i in grp:
+                b = bufs[i % n_buf]
+                b.step[i % copies]()
+                b.c_evt.record(comp)
+                with torch.cuda.stream(d2h_s):
+                    d2h_s.wait_event(b.c_evt)
+                    b.out_host.copy_(b.out, non_blocking=True)
+                    b.d_evt.record(d2h_s)
         with torch.cuda.stream(d2h_s):
             d2h_s.wait_stream(comp)
             d2h_s.wait_stream(h2d_s)
@@ -500,19 +542,25 @@ def run_ours(args, wl, rank, world, local, headline=True):
 
     e2e_pass()
     e2e_times = timed_passes(e2e_pass, max(5, min(passes, 20)), world, dev)
-    # each set computes the same inputs every step: what was read back must be its output
-    for k in range(min(copies, K)):
-        if not torch.equal(out_host[k], sets[k].out.cpu()):
+    # every step computes the same inputs on its weight set: what each buffer read back last
+    # must be that set's output of the device-timed steps
+    for i in range(max(0, K - n_buf), K):
+        b = bufs[i % n_buf]
+        if not torch.equal(b.out_host, sets[i % copies].out.cpu()):
             raise RuntimeError("e2e: an output read back differs from the step's result")
     t_e2e = statistics.median(e2e_times)
     result["e2e"] = {"value": whole_job_throughput(world, bsz, K, t_e2e), "unit": UNIT,
                      "h2d_bytes_per_step": in_bytes,
                      "d2h_bytes_per_step": bsz * 64 * 256 * 2,
-                     "passes": pass_summary(e2e_times)}
-    result["timing"] = ("value: median of passes of K CUDA-graph replays of the whole step; "
+                     "group": E2E_GROUP, "passes": pass_summary(e2e_times)}
+    result["timing"] = ("value: median of passes of one CUDA-graph replay of K whole steps "
+                        "(each step chained to the previous one by programmatic dependent "
+                        "launch); ms_per_step_isolated: the same steps as K separate graph "
+                        "replays; "
                         "e2e: median of passes of K public-API calls, each step's inputs "
-                        "copied in and its output copied back on two copy streams that "
-                        "overlap the neighbouring steps' compute; attn: median of passes of "
+                        "copied in (by groups of 1, 4, then E2E_GROUP steps) and its output "
+                        "copied back, on two copy streams that overlap the compute; "
+                        "attn: median of passes of "
                         "K back-to-back mfa_decode_attn calls")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         # whole decode steps of the first n_seq sequences, repeated until about 10 s of CPU
@@ -541,7 +589,8 @@ def run_extra_workloads(args, rank, world, local):
     torch.cuda.empty_cache()
     for name in EXTRA_WORKLOADS:
         r = run_ours(args, W.workload(name), rank, world, local, headline=False)
-        out[name] = {k: r[k] for k in ("value", "ms_per_step", "attn_ms", "kv_gbs", "roofline",
+        out[name] = {k: r[k] for k in ("value", "ms_per_step", "ms_per_step_isolated",
+                                       "attn_ms", "kv_gbs", "roofline",
                                        "layer_roofline", "clocks", "step_passes",
                                        "attn_passes")}
         out[name]["config"] = {k: r["config"][k] for k in ("batch_per_gpu", "context",
@@ -549,6 +598,11 @@ def run_extra_workloads(args, rank, world, local):
         gc.collect()
         torch.cuda.empty_cache()
     return out
+
+
+# Largest group of steps whose inputs the end-to-end passes copy in together: the calls of a
+# group run back to back on the compute stream (a few layers of one token step of a model).
+E2E_GROUP = 8
 
 
 # The workloads timed after the headline in a default run: the 8K point of the metric, the
