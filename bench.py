@@ -335,13 +335,32 @@ def run_ours(args, wl, rank, world, local, headline=True):
     if not torch.isfinite(sets[0].out.float()).all():
         raise RuntimeError("non-finite output")
 
-    # host cost of one call of the public API (enqueue only, no device work waited for)
+    # host cost of one call of the public API: the median time to enqueue one call into an
+    # idle stream (no device work waited for, no queue back-pressure); the same for a replay
+    # of the step captured by the library (mfa_decode_layer_graph); and the mean over 50
+    # calls back to back, whose later calls can wait for room in the launch queue
+    def enqueue_us(call, reps=200):
+        times = []
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            h0 = time.perf_counter()
+            call()
+            times.append((time.perf_counter() - h0) * 1e6)
+        torch.cuda.synchronize()
+        return statistics.median(times)
+
+    host_us = enqueue_us(sets[0].step)
+    captured = mfa.StepGraph(sets[0].x, *sets[0].w, sets[0].cache, lens, sets[0].q,
+                             sets[0].out, ws)
+    captured()
+    host_us_graph = enqueue_us(captured)
+    captured.close()
     torch.cuda.synchronize()
     n_host = 50
     h0 = time.perf_counter()
     for i in range(n_host):
         sets[i % copies].step()
-    host_us = (time.perf_counter() - h0) / n_host * 1e6
+    host_us_queued = (time.perf_counter() - h0) / n_host * 1e6
     torch.cuda.synchronize()
 
     # The K steps of a pass captured once as one CUDA graph over the rotating copies (the
@@ -453,6 +472,8 @@ def run_ours(args, wl, rank, world, local, headline=True):
         "attn_passes": pass_summary(attn_times),
         "gpu_launches": (LAUNCHES_PER_LAYER if args.weights == "bf16" else LAUNCHES_PER_LAYER_W8) * K,
         "host_us_per_call": host_us,
+        "host_us_per_call_graph": host_us_graph,
+        "host_us_per_call_queued": host_us_queued,
     }
     if not headline:
         return result

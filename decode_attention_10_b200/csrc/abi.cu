@@ -5,9 +5,17 @@
 
 #include <atomic>
 #include <cstring>
+#include <new>
 #include <vector>
 
 #include "mfa_internal.cuh"
+
+// A captured decode step (include/mfa.h): the instantiated graph and the device it was
+// captured on.
+struct mfa_step_graph {
+  cudaGraphExec_t exec;
+  int device;
+};
 
 namespace mfa {
 namespace {
@@ -615,20 +623,70 @@ mfa_status decode_layer_impl(const void* x, WRef w_qdown, const void* gamma, WRe
 }  // namespace
 }  // namespace mfa
 
+namespace mfa {
+namespace {
+
+// The checks of one decode step (direct or captured), in this order: the KV description, eps
+// and scale, the pointers (non-null, 16-byte aligned), the FP8 weights (weights_ok), then the
+// workspace, whose layout goes to *L.
+mfa_status check_layer(const void* const* ptrs, size_t n, bool weights_ok, float eps,
+                       float scale, const mfa_kv_cache* kv, void* ws, size_t ws_bytes,
+                       WsLayout* L) {
+  mfa_status st = check_kv(kv);
+  if (st != MFA_OK) return st;
+  if (!(eps > 0.f) || !(scale > 0.f)) return MFA_ERR_INVALID_ARG;
+  for (size_t i = 0; i < n; ++i)
+    if (ptrs[i] == nullptr || !aligned16(ptrs[i])) return MFA_ERR_INVALID_ARG;
+  if (!weights_ok) return MFA_ERR_INVALID_ARG;
+  return check_ws(ws, ws_bytes, kv->batch, L);
+}
+
+bool valid_w8_all(const mfa_w8& a, const mfa_w8& b, const mfa_w8& c, const mfa_w8& d) {
+  return valid_w8(a) && valid_w8(b) && valid_w8(c) && valid_w8(d);
+}
+
+// Records launch(stream) on a stream of the library's own (thread-local capture, so other
+// threads' work is not affected) and instantiates the graph for the current device.
+template <class F>
+mfa_status capture_step(F&& launch, mfa_step_graph** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MFA_ERR_CUDA;
+  cudaStream_t cs = nullptr;
+  if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return MFA_ERR_CUDA;
+  mfa_status st = MFA_ERR_CUDA;
+  cudaGraph_t graph = nullptr;
+  if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) == cudaSuccess) {
+    st = launch(cs);
+    // the capture always ends, whatever the launches returned
+    if (cudaStreamEndCapture(cs, &graph) != cudaSuccess && st == MFA_OK) st = MFA_ERR_CUDA;
+  }
+  cudaGraphExec_t exec = nullptr;
+  if (st == MFA_OK && (graph == nullptr || cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess))
+    st = MFA_ERR_CUDA;
+  if (graph != nullptr) cudaGraphDestroy(graph);
+  cudaStreamDestroy(cs);
+  if (st != MFA_OK) return st;
+  mfa_step_graph* g = new (std::nothrow) mfa_step_graph{exec, dev};
+  if (g == nullptr) {
+    cudaGraphExecDestroy(exec);
+    return MFA_ERR_CUDA;
+  }
+  *out = g;
+  return MFA_OK;
+}
+
+}  // namespace
+}  // namespace mfa
+
 extern "C" {
 
 mfa_status mfa_decode_layer(const void* x, const void* w_qdown, const void* gamma,
                             const void* w_qup, const void* w_k, const void* w_v, float eps,
                             const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
                             void* q_out, void* out, void* ws, size_t ws_bytes, void* stream) {
-  mfa_status st = check_kv(kv);
-  if (st != MFA_OK) return st;
-  if (!(eps > 0.f) || !(scale > 0.f)) return MFA_ERR_INVALID_ARG;
   const void* ptrs[] = {x, w_qdown, gamma, w_qup, w_k, w_v, seq_lens, q_out, out};
-  for (const void* p : ptrs)
-    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
   WsLayout L;
-  st = check_ws(ws, ws_bytes, kv->batch, &L);
+  const mfa_status st = check_layer(ptrs, 9, true, eps, scale, kv, ws, ws_bytes, &L);
   if (st != MFA_OK) return st;
   return decode_layer_impl(x, WRef{w_qdown, nullptr}, gamma, WRef{w_qup, nullptr},
                            WRef{w_k, nullptr}, WRef{w_v, nullptr}, eps, kv, seq_lens, scale,
@@ -639,21 +697,68 @@ mfa_status mfa_decode_layer_w8(const void* x, mfa_w8 w_qdown, const void* gamma,
                                mfa_w8 w_k, mfa_w8 w_v, float eps, const mfa_kv_cache* kv,
                                const int32_t* seq_lens, float scale, void* q_out, void* out,
                                void* ws, size_t ws_bytes, void* stream) {
-  mfa_status st = check_kv(kv);
-  if (st != MFA_OK) return st;
-  if (!(eps > 0.f) || !(scale > 0.f)) return MFA_ERR_INVALID_ARG;
   const void* ptrs[] = {x, gamma, seq_lens, q_out, out};
-  for (const void* p : ptrs)
-    if (p == nullptr || !aligned16(p)) return MFA_ERR_INVALID_ARG;
-  if (!valid_w8(w_qdown) || !valid_w8(w_qup) || !valid_w8(w_k) || !valid_w8(w_v))
-    return MFA_ERR_INVALID_ARG;
   WsLayout L;
-  st = check_ws(ws, ws_bytes, kv->batch, &L);
+  const bool w_ok = valid_w8_all(w_qdown, w_qup, w_k, w_v);
+  const mfa_status st = check_layer(ptrs, 5, w_ok, eps, scale, kv, ws, ws_bytes, &L);
   if (st != MFA_OK) return st;
   return decode_layer_impl(x, WRef{w_qdown.codes, w_qdown.scales}, gamma,
                            WRef{w_qup.codes, w_qup.scales}, WRef{w_k.codes, w_k.scales},
                            WRef{w_v.codes, w_v.scales}, eps, kv, seq_lens, scale, q_out, out,
                            ws, L, static_cast<cudaStream_t>(stream));
+}
+
+mfa_status mfa_decode_layer_graph(const void* x, const void* w_qdown, const void* gamma,
+                                  const void* w_qup, const void* w_k, const void* w_v, float eps,
+                                  const mfa_kv_cache* kv, const int32_t* seq_lens, float scale,
+                                  void* q_out, void* out, void* ws, size_t ws_bytes,
+                                  mfa_step_graph** graph) {
+  if (graph == nullptr) return MFA_ERR_INVALID_ARG;
+  *graph = nullptr;
+  const void* ptrs[] = {x, w_qdown, gamma, w_qup, w_k, w_v, seq_lens, q_out, out};
+  WsLayout L;
+  const mfa_status st = check_layer(ptrs, 9, true, eps, scale, kv, ws, ws_bytes, &L);
+  if (st != MFA_OK) return st;
+  return capture_step(
+      [&](cudaStream_t cs) {
+        return decode_layer_impl(x, WRef{w_qdown, nullptr}, gamma, WRef{w_qup, nullptr},
+                                 WRef{w_k, nullptr}, WRef{w_v, nullptr}, eps, kv, seq_lens,
+                                 scale, q_out, out, ws, L, cs);
+      },
+      graph);
+}
+
+mfa_status mfa_decode_layer_w8_graph(const void* x, mfa_w8 w_qdown, const void* gamma,
+                                     mfa_w8 w_qup, mfa_w8 w_k, mfa_w8 w_v, float eps,
+                                     const mfa_kv_cache* kv, const int32_t* seq_lens,
+                                     float scale, void* q_out, void* out, void* ws,
+                                     size_t ws_bytes, mfa_step_graph** graph) {
+  if (graph == nullptr) return MFA_ERR_INVALID_ARG;
+  *graph = nullptr;
+  const void* ptrs[] = {x, gamma, seq_lens, q_out, out};
+  WsLayout L;
+  const bool w_ok = valid_w8_all(w_qdown, w_qup, w_k, w_v);
+  const mfa_status st = check_layer(ptrs, 5, w_ok, eps, scale, kv, ws, ws_bytes, &L);
+  if (st != MFA_OK) return st;
+  return capture_step(
+      [&](cudaStream_t cs) {
+        return decode_layer_impl(x, WRef{w_qdown.codes, w_qdown.scales}, gamma,
+                                 WRef{w_qup.codes, w_qup.scales}, WRef{w_k.codes, w_k.scales},
+                                 WRef{w_v.codes, w_v.scales}, eps, kv, seq_lens, scale, q_out,
+                                 out, ws, L, cs);
+      },
+      graph);
+}
+
+mfa_status mfa_step_graph_launch(const mfa_step_graph* graph, void* stream) {
+  if (graph == nullptr) return MFA_ERR_INVALID_ARG;
+  return cuda_status(cudaGraphLaunch(graph->exec, static_cast<cudaStream_t>(stream)));
+}
+
+void mfa_step_graph_destroy(mfa_step_graph* graph) {
+  if (graph == nullptr) return;
+  cudaGraphExecDestroy(graph->exec);
+  delete graph;
 }
 
 }  // extern "C"

@@ -59,6 +59,15 @@ _SIGNATURES = {
     "mfa_query_proj_noalloc_get_error": (ctypes.c_int, [_P]),
     "mfa_split_plan": (ctypes.c_int, [_P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "mfa_query_proj_noalloc_wait_selftest": (ctypes.c_int, [ctypes.c_uint32, _P]),
+    "mfa_decode_layer_graph": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _P,
+                                              ctypes.c_float, _P, _P, _P, ctypes.c_size_t,
+                                              ctypes.POINTER(ctypes.c_void_p)]),
+    "mfa_decode_layer_w8_graph": (ctypes.c_int, [_P, W8, _P, W8, W8, W8, ctypes.c_float, _P,
+                                                 _P, ctypes.c_float, _P, _P, _P,
+                                                 ctypes.c_size_t,
+                                                 ctypes.POINTER(ctypes.c_void_p)]),
+    "mfa_step_graph_launch": (ctypes.c_int, [_P, _P]),
+    "mfa_step_graph_destroy": (None, [_P]),
 }
 NOALLOC_MAX_BATCH = 32
 
@@ -394,3 +403,44 @@ class DecodeStep:
         st = self._fn(*self._args)
         if st != 0:
             raise MfaError(st, "mfa_decode_layer_w8" if self._w8 else "mfa_decode_layer")
+
+
+class StepGraph:
+    """A decode step captured once by the library (mfa_decode_layer_graph): each call replays
+    it with one graph launch (mfa_step_graph_launch) instead of the step's kernel launches,
+    with results bit-identical to mfa_decode_layer's. Buffers as for DecodeStep: addresses
+    fixed for the handle's life, contents free to change between calls. A replay does not
+    overlap the kernel before it on the stream, so DecodeStep is the faster choice when the
+    GPU, not the host, paces the loop. Captured on the current CUDA device."""
+
+    def __init__(self, x, w_qdown, gamma, w_qup, w_k, w_v, cache: KVCache, seq_lens,
+                 q_out, out, ws: Workspace, eps: float = 1e-6, scale: float = 1.0 / 16.0,
+                 stream=None):
+        self._lib = load()
+        self._h = ctypes.c_void_p()
+        self._keep = (x, w_qdown, gamma, w_qup, w_k, w_v, cache, seq_lens, q_out, out, ws)
+        w8 = isinstance(w_qdown, BlockFP8Weight)
+        wa = (lambda w: w.struct) if w8 else (lambda w: _P(_ptr(w)))
+        fn = self._lib.mfa_decode_layer_w8_graph if w8 else self._lib.mfa_decode_layer_graph
+        _check(fn(_P(_ptr(x)), wa(w_qdown), _P(_ptr(gamma)), wa(w_qup), wa(w_k), wa(w_v),
+                  ctypes.c_float(eps), ctypes.byref(cache.desc), _P(_ptr(seq_lens)),
+                  ctypes.c_float(scale), _P(_ptr(q_out)), _P(_ptr(out)), _P(ws.ptr),
+                  ctypes.c_size_t(ws.nbytes), ctypes.byref(self._h)),
+               "mfa_decode_layer_w8_graph" if w8 else "mfa_decode_layer_graph")
+        self._stream = _P(_stream(stream))
+
+    def __call__(self):
+        st = self._lib.mfa_step_graph_launch(self._h, self._stream)
+        if st != 0:
+            raise MfaError(st, "mfa_step_graph_launch")
+
+    def close(self):
+        if self._h is not None and self._h.value is not None:
+            self._lib.mfa_step_graph_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -338,6 +338,46 @@ MFA_API mfa_status mfa_wait_selftest(void* ws, size_t ws_bytes, uint32_t limit_u
 MFA_API mfa_status mfa_split_plan(const mfa_kv_cache* kv, const int32_t* seq_lens,
                                   int32_t grid, int32_t* out, size_t out_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------------------
+ * Captured decode steps (no counterpart in the pages: a host-cost option of this library)
+ * ------------------------------------------------------------------------------------- */
+
+/* One decode step captured once as a CUDA graph on the current device, for callers whose
+ * host thread, not the GPU, paces the loop: replaying it costs one graph launch instead of
+ * the step's five or six kernel launches. A replay runs exactly the launches that
+ * mfa_decode_layer (w8: mfa_decode_layer_w8) would make with these arguments, so its results
+ * are bit-identical to that call's. The arguments are read once, at capture: the addresses
+ * and the mfa_kv_cache fields must stay valid and unchanged for the handle's life, while the
+ * buffers' contents (x, seq_lens, the weights, the cache rows, the KV table's entries) may
+ * change between replays. A replay begins only after the stream's earlier work has
+ * completed (no programmatic overlap with the kernel before it), so back-to-back direct
+ * calls, which do overlap, are the faster choice whenever the GPU paces the loop.
+ *   *out receives the handle (NULL on error). Errors as mfa_decode_layer, plus
+ *   MFA_ERR_CUDA if the capture or the graph instantiation fails. The capture runs on a
+ *   stream of the library's own and does not touch the caller's streams. */
+typedef struct mfa_step_graph mfa_step_graph;
+
+MFA_API mfa_status mfa_decode_layer_graph(const void* x, const void* w_qdown, const void* gamma,
+                                          const void* w_qup, const void* w_k, const void* w_v,
+                                          float eps, const mfa_kv_cache* kv,
+                                          const int32_t* seq_lens, float scale, void* q_out,
+                                          void* out, void* ws, size_t ws_bytes,
+                                          mfa_step_graph** graph);
+
+MFA_API mfa_status mfa_decode_layer_w8_graph(const void* x, mfa_w8 w_qdown, const void* gamma,
+                                             mfa_w8 w_qup, mfa_w8 w_k, mfa_w8 w_v, float eps,
+                                             const mfa_kv_cache* kv, const int32_t* seq_lens,
+                                             float scale, void* q_out, void* out, void* ws,
+                                             size_t ws_bytes, mfa_step_graph** graph);
+
+/* Replay a captured step on `stream` (a stream of the device it was captured on).
+ * MFA_ERR_INVALID_ARG for a NULL handle, MFA_ERR_CUDA if the launch fails. */
+MFA_API mfa_status mfa_step_graph_launch(const mfa_step_graph* graph, void* stream);
+
+/* Release a handle (NULL is ignored). Replays already enqueued still run: the graph is
+ * freed once they complete. */
+MFA_API void mfa_step_graph_destroy(mfa_step_graph* graph);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

@@ -131,6 +131,33 @@ def test_invalid_arguments_are_rejected_before_any_device_work(lib):
     assert lib.mfa_get_error(None, None) == 1
 
 
+def test_captured_step_arguments_are_rejected_before_any_device_work(lib):
+    P = ctypes.c_void_p
+    fake = P(4096)
+    kv = mfa.KvCacheDesc(4, 0, 1.0, 1.0, 4096)
+    h = ctypes.c_void_p(1234)
+    # no place for the handle
+    assert lib.mfa_decode_layer_graph(fake, fake, fake, fake, fake, fake, 1e-6,
+                                      ctypes.byref(kv), fake, 0.0625, fake, fake, fake,
+                                      1 << 30, None) == 1
+    # a rejected argument leaves a NULL handle (scale, a misaligned x, a bad cache)
+    for scale, x, desc in ((-1.0, fake, kv), (0.0625, P(4098), kv),
+                           (0.0625, fake, mfa.KvCacheDesc(0, 0, 1.0, 1.0, 4096))):
+        assert lib.mfa_decode_layer_graph(x, fake, fake, fake, fake, fake, 1e-6,
+                                          ctypes.byref(desc), fake, scale, fake, fake, fake,
+                                          1 << 30, ctypes.byref(h)) == 1
+        assert h.value is None
+        h = ctypes.c_void_p(1234)
+    w = mfa.W8(4096, 4096)
+    bad_w = mfa.W8(4096, None)  # FP8 weights need their scales
+    assert lib.mfa_decode_layer_w8_graph(fake, w, fake, w, bad_w, w, 1e-6, ctypes.byref(kv),
+                                         fake, 0.0625, fake, fake, fake, 1 << 30,
+                                         ctypes.byref(h)) == 1
+    assert h.value is None
+    assert lib.mfa_step_graph_launch(None, None) == 1
+    lib.mfa_step_graph_destroy(None)
+
+
 def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(mfa, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
