@@ -509,12 +509,7 @@ def run_ours(args, wl, rank, world, local, headline=True):
                                     ws, stream=comp) for k in range(copies)},
             c_evt=torch.cuda.Event(),  # its step computed (inputs consumed)
             d_evt=torch.cuda.Event()))  # its output read back
-    groups, g0 = [], 0
-    for size in itertools.chain((1, 4), itertools.repeat(E2E_GROUP)):
-        if g0 >= K:
-            break
-        groups.append(range(g0, min(g0 + min(size, E2E_GROUP), K)))
-        g0 = groups[-1].stop
+    groups = e2e_groups(K, E2E_GROUP)
     # two consecutive groups never hold more than n_buf steps, so the copies of group g + 1,
     # enqueued before group g's calls, wait only for steps of groups before g, whose events
     # are recorded (and not yet recorded again) by then
@@ -619,6 +614,19 @@ def run_extra_workloads(args, rank, world, local):
         gc.collect()
         torch.cuda.empty_cache()
     return out
+
+
+def e2e_groups(steps: int, largest: int):
+    """The end-to-end passes' groups of consecutive steps: 1, then 4, then `largest` at a time
+    (the first group small so that the first call waits for one input copy only), the last
+    group what is left. Returns ranges that cover 0 .. steps - 1 in order."""
+    groups, g0 = [], 0
+    for size in itertools.chain((1, 4), itertools.repeat(largest)):
+        if g0 >= steps:
+            break
+        groups.append(range(g0, min(g0 + min(size, largest), steps)))
+        g0 = groups[-1].stop
+    return groups
 
 
 # Largest group of steps whose inputs the end-to-end passes copy in together: the calls of a

@@ -52,3 +52,15 @@ def test_paged_layout_holds_every_sequence_row_in_its_listed_pages():
                 rows = torch.cat([raw[int(pt[b, p])] for p in range(need[b])])[:t.shape[0]]
                 want = t.view(torch.uint8) if t.element_size() == 1 else t.view(torch.int16)
                 assert torch.equal(rows, want)
+
+
+def test_e2e_groups_cover_the_steps_in_order_within_the_buffer_ring():
+    import bench
+    for largest in (1, 4, 8):
+        for steps in range(1, 60):
+            groups = bench.e2e_groups(steps, largest)
+            flat = [i for g in groups for i in g]
+            assert flat == list(range(steps))
+            assert len(groups[0]) == 1 and all(1 <= len(g) <= largest for g in groups)
+            # the e2e loop reuses a ring of 2 * largest buffers: two consecutive groups fit it
+            assert all(len(a) + len(b) <= 2 * largest for a, b in zip(groups, groups[1:]))
