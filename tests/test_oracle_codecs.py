@@ -10,7 +10,9 @@ from oracle import codecs
 
 
 def _f32_from_bf16_bits(bits):
-    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    # (NaN patterns widen to NaN; numpy warns about the cast of signalling ones)
+    with np.errstate(invalid="ignore"):
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def test_bf16_decode_all_patterns_match_binary32_upper_half():
