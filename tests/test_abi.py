@@ -162,3 +162,44 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(mfa, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         mfa.load(str(tmp_path / "nope.so"))
+
+
+def test_header_compiles_as_c99_and_the_library_links_from_c(lib, tmp_path):
+    # the boundary needs no Python and no torch: a C99 program includes the header, links
+    # libmfa.so and gets the documented statuses for calls rejected before any device work
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi_check.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "mfa.h"
+int main(void) {
+  void* fake = (void*)4096;
+  mfa_kv_cache kv = {4, MFA_KV_BF16, 1.0f, 1.0f, fake, 0};
+  mfa_step_graph* g = (mfa_step_graph*)fake;
+  int bad = 0;
+  bad |= mfa_version() < 100;
+  bad |= mfa_query_proj(fake, fake, fake, fake, 0.0f, fake, 4, fake, 1u << 30, 0) !=
+         MFA_ERR_INVALID_ARG;
+  bad |= mfa_decode_attn(fake, 0, fake, 0.0625f, fake, fake, 1u << 30, 0) !=
+         MFA_ERR_INVALID_ARG;
+  bad |= mfa_decode_layer_graph(fake, fake, fake, fake, fake, fake, 1e-6f, &kv, fake, -1.0f,
+                                fake, fake, fake, 1u << 30, &g) != MFA_ERR_INVALID_ARG;
+  bad |= g != 0;
+  bad |= mfa_step_graph_launch(0, 0) != MFA_ERR_INVALID_ARG;
+  mfa_step_graph_destroy(0);
+  printf("%s %s\n", bad ? "FAIL" : "OK", mfa_status_str(MFA_ERR_WORKSPACE));
+  return bad;
+}
+""")
+    libdir = os.path.join(ROOT, "decode_attention_10_b200")
+    exe = tmp_path / "abi_check"
+    subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lmfa",
+                    "-Wl,-rpath," + libdir], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.split() == ["OK", "MFA_ERR_WORKSPACE"]
