@@ -511,8 +511,8 @@ def run_ours(args, wl, rank, world, local, headline=True):
             d_evt=torch.cuda.Event()))  # its output read back
     groups = e2e_groups(K, E2E_GROUP)
     # two consecutive groups never hold more than n_buf steps, so the copies of group g + 1,
-    # enqueued before group g's calls, wait only for steps of groups before g, whose events
-    # are recorded (and not yet recorded again) by then
+    # enqueued after group g's first call, wait only for steps of groups before g, whose
+    # events are recorded (and not yet recorded again by group g, whose buffers differ)
     assert all(len(a) + len(b) <= n_buf for a, b in zip(groups, groups[1:]))
     h_evt = [torch.cuda.Event() for _ in range(2)]  # inputs of group g in (by g % 2)
     e2e_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
@@ -533,11 +533,6 @@ def run_ours(args, wl, rank, world, local, headline=True):
             e2e_ev[0].record(h2d_s)
             h2d(0)
         for gi, grp in enumerate(groups):
-            # the next group's inputs go in while this group computes; enqueued before this
-            # group's read-backs, which would otherwise hold them back in the copy queue
-            with torch.cuda.stream(h2d_s):
-                if gi + 1 < len(groups):
-                    h2d(gi + 1)
             comp.wait_event(h_evt[gi % 2])
             if grp[-1] >= n_buf:  # the group's buffers' previous outputs have been read back
                 comp.wait_event(bufs[grp[-1] % n_buf].d_evt)
@@ -545,6 +540,13 @@ def run_ours(args, wl, rank, world, local, headline=True):
                 b = bufs[i % n_buf]
                 b.step[i % copies]()
                 b.c_evt.record(comp)
+                if i == grp[0] and gi + 1 < len(groups):
+                    # the next group's inputs go in while this group computes: enqueued once
+                    # the group's first call is (so the GPU does not wait for the host to
+                    # issue them), and before any of the group's read-backs, which would
+                    # otherwise hold them back in the copy queue
+                    with torch.cuda.stream(h2d_s):
+                        h2d(gi + 1)
                 with torch.cuda.stream(d2h_s):
                     d2h_s.wait_event(b.c_evt)
                     b.out_host.copy_(b.out, non_blocking=True)
