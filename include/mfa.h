@@ -27,7 +27,9 @@
  *     be 16-byte aligned; rows are dense (no padding) unless stated.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Compute calls only
  *     enqueue work on it: they neither allocate nor synchronize, and may be captured in
- *     a CUDA graph. Setup calls (mfa_kv_table_init, mfa_workspace_init) may synchronize.
+ *     a CUDA graph. Setup calls (mfa_kv_table_init, mfa_workspace_init, and the capture
+ *     calls mfa_decode_layer_graph / _w8_graph, which create a stream and a CUDA graph of
+ *     their own) may synchronize.
  *   - Problems visible on the host (null pointer, bad size, misalignment, workspace too
  *     small, unsupported dtype) return an error status before anything is enqueued.
  *     Problems visible only on the device (a length above a sequence's capacity, an empty
