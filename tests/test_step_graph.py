@@ -140,3 +140,67 @@ def test_capture_rejects_bad_arguments_and_leaves_no_handle():
     torch.cuda.synchronize()
     assert mfa.get_error(step.ws) == 0
     lib.mfa_step_graph_destroy(h)
+
+
+@pytest.mark.parametrize("kv_dtype", [W.KV_BF16, W.KV_FP8])
+def test_chained_steps_on_one_workspace_match_isolated_steps(kv_dtype):
+    # Consecutive steps on a stream overlap through programmatic dependent launch (each
+    # step's first kernel streams weights while the previous step's combine runs) and share
+    # the workspace. Two input sets with different x and lengths (so different split plans),
+    # run A, B, A, B back to back -- direct calls and one CUDA graph of the four calls --
+    # must leave exactly the outputs of isolated calls.
+    from decode_attention_10_b200 import mfa
+    sets = []
+    ws = None
+    for lens, seed in (([1, 130, 300, 129], 150), ([257, 64, 1000, 5], 151)):
+        inp = W.generate(lens, kv_dtype, seed=seed)
+        st = GpuStep(inp)
+        if ws is None:
+            ws = st.ws
+        q = torch.empty(len(lens), 64, 256, dtype=torch.bfloat16, device="cuda")
+        out = torch.empty_like(q)
+        st.call = mfa.DecodeStep(st.x, st.w_qdown, st.gamma, st.w_qup, st.w_k, st.w_v,
+                                 st.cache, st.seq_lens, q, out, ws)
+        st.q_buf, st.out_buf = q, out
+        sets.append(st)
+    ref = []
+    for st in sets:  # isolated: each call alone on an idle stream (the append is idempotent)
+        torch.cuda.synchronize()
+        st.call()
+        torch.cuda.synchronize()
+        ref.append((st.q_buf.clone(), st.out_buf.clone()))
+    assert mfa.get_error(ws) == 0
+
+    def check(where):
+        torch.cuda.synchronize()
+        for st, (q0, o0) in zip(sets, ref):
+            assert torch.equal(st.q_buf, q0), f"{where}: q differs from the isolated call"
+            assert torch.equal(st.out_buf, o0), f"{where}: output differs from the isolated call"
+        assert mfa.get_error(ws) == 0
+
+    for st in sets:
+        st.q_buf.zero_()
+        st.out_buf.zero_()
+    for st in sets + sets:  # direct calls, back to back
+        st.call()
+    check("direct chain")
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        for st in sets:
+            st.gcall = mfa.DecodeStep(st.x, st.w_qdown, st.gamma, st.w_qup, st.w_k, st.w_v,
+                                      st.cache, st.seq_lens, st.q_buf, st.out_buf, ws,
+                                      stream=side)
+        with torch.cuda.graph(g, stream=side):
+            for st in sets + sets:
+                st.gcall()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for st in sets:
+        st.q_buf.zero_()
+        st.out_buf.zero_()
+    g.replay()
+    check("graph of four chained steps")
+    del g
