@@ -85,11 +85,22 @@ template <bool kFp8>
 struct Cfg {
   static constexpr int kGroups = 2;
   static constexpr int kSoftmaxWarps = 4 * kGroups;     // warps 2 .. 2 + kSoftmaxWarps - 1
-  static constexpr int kThreads = 64 + 32 * kSoftmaxWarps;
+  // FP8: S and PV are issued by two warps (warp 1 and warp kPvWarp), so that a PV is never
+  // held back behind the issue of the next S (an issuing thread waits while the tensor core's
+  // queue is full); K and V boxes then sit in rings of their own, each read by one warp
+  static constexpr bool kSplitIssue = kFp8;
+  static constexpr int kPvWarp = 2 + kSoftmaxWarps;
+  static constexpr int kMmaWarps = kSplitIssue ? 2 : 1;
+  static constexpr int kThreads = 64 + 32 * kSoftmaxWarps + (kSplitIssue ? 32 : 0);
+  // the launch bound: at most three warps share an SM sub-partition, so 168 registers a thread
+  // is the ceiling either way (384 threads cap the compiler at it)
+  static constexpr int kBoundThreads = kSplitIssue ? 384 : kThreads;
   static constexpr int kGroupHeads = kHeads / kGroups;  // heads per group
   static constexpr uint32_t kBarAll = 1 + kGroups;      // named barrier of all softmax warps
-  // bf16 ring: even, so a V half-tile's 2 chunks are adjacent
+  // bf16 ring: even, so a V half-tile's 2 chunks are adjacent. FP8: K boxes in slots
+  // [0, kKSlots), V boxes in [kKSlots, kSlots)
   static constexpr int kSlots = kFp8 ? 8 : 6;
+  static constexpr int kKSlots = kSplitIssue ? 4 : kSlots;
   static constexpr int kTileBoxes = kFp8 ? 2 : 4;   // ring boxes per K (or V) tile
   static constexpr int kBoxDims = kFp8 ? 128 : 64;  // head dims per box
   static constexpr int kMmaK = kFp8 ? 32 : 16;      // K of one MMA instruction
@@ -105,6 +116,11 @@ struct Cfg {
   static constexpr uint32_t kIdescPV = idesc_f16(128, kSCols, !kFp8, true, true);   // V^T x P^T
 };
 static_assert(Cfg<true>::kSlots <= kMaxSlots && Cfg<false>::kSlots <= kMaxSlots, "ring");
+static_assert(!Cfg<true>::kSplitIssue ||
+                  (Cfg<true>::kPvWarp * 32 + 32 == Cfg<true>::kThreads &&
+                   Cfg<true>::kThreads <= Cfg<true>::kBoundThreads && Cfg<true>::kKSlots % 2 == 0),
+              "FP8: the PV warp is the last warp; K and V rings of whole tiles");
+static_assert(Cfg<false>::kPvWarp * 32 == Cfg<false>::kThreads, "bf16: no PV warp");
 static_assert(2 * kQ8ChunkBytes == 4 * kQChunkBytes, "FP8 Q is split in place");
 static_assert(Cfg<true>::kSoftmaxWarps <= kMaxSoftmaxWarps &&
                   Cfg<false>::kSoftmaxWarps <= kMaxSoftmaxWarps,
@@ -264,7 +280,10 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   const int page_shift = 31 - __clz(page_size);         // page sizes are powers of two
   const int box_rows = kPaged ? paged_box_rows(page_size) : kTile;
   constexpr int kC = C::kTileBoxes;
-  uint32_t chunk = 0, issued = 0;  // ring boxes
+  uint32_t chunk = 0, issued = 0;  // ring boxes (FP8: the K ring's)
+  uint32_t vchunk = 0, vissued = 0;  // FP8: the V ring's
+  constexpr uint32_t kKN = C::kKSlots;
+  constexpr uint32_t kVN = kN > C::kKSlots ? kN - C::kKSlots : 1;  // (unused with one ring)
   int item = 0, q_issued = 0;
   if (leader) prefetch_tensormap(q_map);
   // every K/V byte is read once: keep it from evicting q and the split partials from L2
@@ -330,12 +349,9 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
       }
     }
   };
-  auto issue_box = [&](const WorkItem& w, int j) {
-    const KvSeq* seq = a.kv + w.b;
-    int y, a0, e0;
+  // box j of an item: K or V, of tile t, column box c
+  auto classify = [&](const WorkItem& w, int j, bool& is_v, int& t, int& c) {
     const int n = num_tiles(w);
-    bool is_v;
-    int t, c;
     if (j < kC) {
       is_v = false, t = 0, c = j;
     } else {
@@ -345,15 +361,32 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
       else
         is_v = true, t = n - 1, c = rr;
     }
+  };
+  auto issue_box = [&](const WorkItem& w, int j) {
+    const KvSeq* seq = a.kv + w.b;
+    int y, a0, e0;
+    bool is_v;
+    int t, c;
+    classify(w, j, is_v, t, c);
     tile_window(w, t, paged, y, a0, e0);
-    const uint32_t slot = chunk % kN, use = chunk / kN;
+    // the box's slot and the use of that slot it is (one ring, or FP8's K and V rings)
+    uint32_t slot, use;
+    uint32_t* rc = &chunk;
+    if constexpr (C::kSplitIssue) {
+      if (is_v) rc = &vchunk;
+      slot = is_v ? kKN + *rc % kVN : *rc % kKN;
+      use = is_v ? *rc / kVN : *rc / kKN;
+    } else {
+      slot = chunk % kN;
+      use = chunk / kN;
+    }
     if (use > 0) mbar_wait(&S.kv_empty[slot], (use - 1) & 1, abort);
     const bool ok = !*abort;
     if (leader && ok) mbar_arrive_expect_tx(&S.kv_full[slot], kChunkBytes);
     load_rows(ring_chunk(S, slot), is_v ? &seq->tmap_v : &seq->tmap_k, C::kBoxDims * c, w, y,
               &S.kv_full[slot], evict_first, ok);
-    if (ok) issued = chunk + 1;
-    ++chunk;
+    if (ok) *(rc == &vchunk ? &vissued : &issued) = *rc + 1;
+    ++*rc;
   };
   // Q of work item `item` into its buffer (after the previous user of the buffer is done).
   auto issue_q = [&](int item_no, const WorkItem& w) {
@@ -385,10 +418,23 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
     }
   }
   if (has) {
+    // the boxes that find their slot free: the first kN, or with two rings the leading boxes
+    // that are the first use of their ring's slots
     const int total = kBoxesPerTile * num_tiles(it);
-    const int pre = static_cast<int>(kN);
-    first_done = total < pre ? total : pre;
-    for (int j = 0; j < first_done; ++j) issue_box(it, j);
+    if constexpr (C::kSplitIssue) {
+      int nk = 0, nv = 0;
+      while (first_done < total) {
+        bool is_v;
+        int t, c;
+        classify(it, first_done, is_v, t, c);
+        if (is_v ? nv >= static_cast<int>(kVN) : nk >= static_cast<int>(kKN)) break;
+        (is_v ? nv : nk) += 1;
+        issue_box(it, first_done++);
+      }
+    } else {
+      first_done = total < static_cast<int>(kN) ? total : static_cast<int>(kN);
+      for (int j = 0; j < first_done; ++j) issue_box(it, j);
+    }
   }
   pdl_wait();
   while (has) {
@@ -412,20 +458,29 @@ __device__ void run_producer(TcSmem& S, const CUtensorMap* q_map, const AttnArgs
   }
   // Before the CTA may exit, every copy it started must have landed.
   if (*abort) {
-    for (uint32_t c = (issued > kN ? issued - kN : 0); c < issued; ++c)
-      mbar_wait_drain(&S.kv_full[c % kN], (c / kN) & 1);
+    for (uint32_t c = (issued > kKN ? issued - kKN : 0); c < issued; ++c)
+      mbar_wait_drain(&S.kv_full[c % kKN], (c / kKN) & 1);
+    if constexpr (C::kSplitIssue) {
+      for (uint32_t c = (vissued > kVN ? vissued - kVN : 0); c < vissued; ++c)
+        mbar_wait_drain(&S.kv_full[kKN + c % kVN], (c / kVN) & 1);
+    }
     for (int i = (q_issued > C::kQBufs ? q_issued - C::kQBufs : 0); i < q_issued; ++i)
       mbar_wait_drain(&S.q_full[i % C::kQBufs], (i / C::kQBufs) & 1);
   }
 }
 
 // ---------------------------------------------------------------------------------------
-// warp 1 (one elected lane issues): MMA
+// MMA issue (one elected lane issues; the warp runs its loop converged). kRole 0: S and PV
+// from one warp (bf16); FP8: kRole 1, the S products (warp 1, K ring), and kRole 2, the PV
+// products (warp kPvWarp, V ring).
 // ---------------------------------------------------------------------------------------
-template <bool kFp8, bool kPaged>
+template <bool kFp8, bool kPaged, int kRole>
 __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool leader) {
   using C = Cfg<kFp8>;
+  static_assert((kRole == 0) == !C::kSplitIssue, "one issuing warp for bf16, two for FP8");
   constexpr uint32_t kSlots = C::kSlots;
+  // FP8 rings: K boxes in slots [0, kKS), V boxes in [kKS, kSlots); each role counts its own
+  constexpr uint32_t kKS = C::kKSlots, kVS = kSlots > kKS ? kSlots - kKS : 1;
   constexpr int kC = C::kTileBoxes;
   volatile int* abort = &S.abort_flag;
   const int lane = threadIdx.x & 31;
@@ -442,8 +497,8 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       return window_rows_kept(paged, y, e0);
     };
     const int qb = item % C::kQBufs, qu = item / C::kQBufs;
-    // FP8: q_ready completes once per item (the split of its Q)
-    mbar_wait(kFp8 ? &S.q_ready : &S.q_full[qb], (kFp8 ? item : qu) & 1, abort);
+    // FP8: q_ready completes once per item (the split of its Q); the PV role needs no Q
+    if (kRole != 2) mbar_wait(kFp8 ? &S.q_ready : &S.q_full[qb], (kFp8 ? item : qu) & 1, abort);
     tc_fence_after();
     const uint32_t q_base = smem_u32(q_buf<kFp8>(S, qb));
 
@@ -469,9 +524,9 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
         // K(tile): both boxes, then the 8 MMAs back to back. FP8 tiles are consumed slower
         // than they stream, so the ring runs ahead and the boxes have landed; a wait or a
         // commit between MMAs would stall the issue stream.
-        const uint32_t s0 = chunk % kSlots, s1 = (chunk + 1) % kSlots;
-        mbar_wait(&S.kv_full[s0], (chunk / kSlots) & 1, abort);
-        mbar_wait(&S.kv_full[s1], ((chunk + 1) / kSlots) & 1, abort);
+        const uint32_t s0 = chunk % kKS, s1 = (chunk + 1) % kKS;
+        mbar_wait(&S.kv_full[s0], (chunk / kKS) & 1, abort);
+        mbar_wait(&S.kv_full[s1], ((chunk + 1) / kKS) & 1, abort);
         tc_fence_after();
         if (!*abort && leader) {
 #pragma unroll
@@ -519,9 +574,9 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       if constexpr (kFp8) {
         // V(tile): both boxes (one per half of V^T: 128 dims, one M=128 product each), then
         // the 8 MMAs back to back, as for S
-        const uint32_t s0 = chunk % kSlots, s1 = (chunk + 1) % kSlots;
-        mbar_wait(&S.kv_full[s0], (chunk / kSlots) & 1, abort);
-        mbar_wait(&S.kv_full[s1], ((chunk + 1) / kSlots) & 1, abort);
+        const uint32_t s0 = kKS + chunk % kVS, s1 = kKS + (chunk + 1) % kVS;
+        mbar_wait(&S.kv_full[s0], (chunk / kVS) & 1, abort);
+        mbar_wait(&S.kv_full[s1], ((chunk + 1) / kVS) & 1, abort);
         tc_fence_after();
         if (kPaged && keep < kTile && __shfl_sync(0xffffffffu, *abort, 0) == 0) {
           // paged cache, the sequence's last window: V rows past its end are zeroed (see
@@ -589,12 +644,19 @@ __device__ void run_mma(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem, bool
       }
     };
 
-    for (int t = 0; t < n; ++t) {
-      issue_s(gt + t);
-      if (t >= 1) issue_pv(gt + t - 1, t - 1 == 0, rows_kept(t - 1));
+    if constexpr (kRole == 0) {
+      for (int t = 0; t < n; ++t) {
+        issue_s(gt + t);
+        if (t >= 1) issue_pv(gt + t - 1, t - 1 == 0, rows_kept(t - 1));
+      }
+      if (!*abort && leader) umma_commit(&S.q_empty[qb]);
+      issue_pv(gt + n - 1, n == 1, rows_kept(n - 1));
+    } else if constexpr (kRole == 1) {
+      for (int t = 0; t < n; ++t) issue_s(gt + t);
+      if (!*abort && leader) umma_commit(&S.q_empty[qb]);
+    } else {
+      for (int t = 0; t < n; ++t) issue_pv(gt + t, t == 0, rows_kept(t));
     }
-    if (!*abort && leader) umma_commit(&S.q_empty[qb]);
-    issue_pv(gt + n - 1, n == 1, rows_kept(n - 1));
     gt += n;
     ++item;
   });
@@ -966,7 +1028,7 @@ __device__ void run_softmax(TcSmem& S, const AttnArgs& a, int g, uint32_t tmem) 
 }
 
 template <bool kFp8, bool kPaged>
-__global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<kFp8>::kBoundThreads, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap q_map, AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   TcSmem& S = *reinterpret_cast<TcSmem*>(
@@ -991,7 +1053,7 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
     mbar_init(&S.p_full, Cfg<kFp8>::kSoftmaxWarps);
     mbar_init(&S.p_free, 1);
     mbar_init(&S.o_free, Cfg<kFp8>::kSoftmaxWarps);
-    mbar_init(&S.mma_done, 1);
+    mbar_init(&S.mma_done, Cfg<kFp8>::kMmaWarps);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -1033,9 +1095,16 @@ __global__ void __launch_bounds__(Cfg<kFp8>::kThreads, 1)
   if (warp == 0) {
     run_producer<kFp8, kPaged>(S, &q_map, a, g, lane == 0);
   } else if (warp == 1) {
-    run_mma<kFp8, kPaged>(S, a, g, tmem, lane == 0);
+    run_mma<kFp8, kPaged, Cfg<kFp8>::kSplitIssue ? 1 : 0>(S, a, g, tmem, lane == 0);
   } else {
-    run_softmax<kFp8, kPaged>(S, a, g, tmem);
+    bool pv_warp = false;
+    if constexpr (Cfg<kFp8>::kSplitIssue) {
+      if (warp == Cfg<kFp8>::kPvWarp) {
+        run_mma<kFp8, kPaged, 2>(S, a, g, tmem, lane == 0);
+        pv_warp = true;
+      }
+    }
+    if (!pv_warp) run_softmax<kFp8, kPaged>(S, a, g, tmem);
   }
 
   tc_fence_before();
