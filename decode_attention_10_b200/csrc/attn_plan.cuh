@@ -26,13 +26,22 @@ struct PlanSmem {
   int32_t page_size;  // the KV table's layout: 0 contiguous, else rows per page
 };
 
+// The products below stay under 2^27 (NT <= kMaxBatch * kMaxTilesPerSeq = 2^19 tiles, G <=
+// kMaxAttnGrid = 2^8), so 32-bit unsigned arithmetic computes them exactly (a 64-bit division
+// is a long software routine on the GPU, and the plan is on the critical path of every call).
+constexpr uint32_t kMaxTilesPerSeq = (MFA_MAX_CONTEXT + kTile - 1) / kTile;
+static_assert(static_cast<uint64_t>(kMaxBatch) * kMaxTilesPerSeq * kMaxAttnGrid < (1ull << 32),
+              "plan arithmetic fits 32 bits");
+
 __device__ __forceinline__ int plan_bound(int g, int G, int NT) {
-  return static_cast<int>(static_cast<int64_t>(g) * NT / G);
+  return static_cast<int>(static_cast<uint32_t>(g) * static_cast<uint32_t>(NT) /
+                          static_cast<uint32_t>(G));
 }
 
 // CTA owning tile t: the largest g with plan_bound(g) <= t.
 __device__ __forceinline__ int plan_cta_of(int t, int G, int NT) {
-  return static_cast<int>((static_cast<int64_t>(t + 1) * G - 1) / NT);
+  return static_cast<int>((static_cast<uint32_t>(t + 1) * static_cast<uint32_t>(G) - 1u) /
+                          static_cast<uint32_t>(NT));
 }
 
 // Inclusive sum over the lanes of a warp (lane l gets the sum of lanes 0..l).
