@@ -7,7 +7,7 @@
 // Because every head reads the same K/V rows, one pass over a sequence's cache serves all
 // 64 heads: each cached byte is read from HBM once and used 64 times on chip.
 //
-// Design (one persistent CTA per SM, warp-specialized, 320 threads):
+// Design (one persistent CTA per SM, warp-specialized, 320 threads; 352 for FP8 caches):
 //   warp 0      TMA producer: Q of each work item (4 boxes of [64 heads x 64 dims]; two Q
 //               buffers, so the next item's Q loads while this one streams), then K and V
 //               tiles of 128 positions as 16 KB boxes of [128 positions x 64 dims] into a
@@ -31,8 +31,11 @@
 // FP8 caches: the e4m3 codes go to the tensor cores as they are (tcgen05 kind::f8f6f4; e4m3
 // values times the power-of-two scales below are exact, and so are the products). The ring
 // holds raw boxes of [128 positions x 128 dims] (128 bytes a row, the same swizzle), two per
-// K or V tile, eight in flight; each S and each PV is issued as 8 MMAs back to back once
-// both of its boxes have landed (at this byte rate the ring runs ahead of the tensor core). The other operand must be e4m3 too, so Q and P each become a
+// K or V tile: a 4-box K ring read by warp 1, which issues the S products, and a 4-box V ring
+// read by warp 10, which issues the PV products (an issuing thread waits while the tensor
+// core's queue is full, so with one issuing warp a PV whose P was ready waited behind the
+// issue of the next S). Each S and each PV is issued as 8 MMAs back to back once both of its
+// boxes have landed. The other operand must be e4m3 too, so Q and P each become a
 // pair of e4m3 matrices with one common scale, a high part and the rounded remainder (hi +
 // lo keeps 7 to 8 significant bits, about what bf16 keeps), stacked along N:
 //   S^T(t)[128 pos x 128] = K(t) . [Q_hi ; Q_lo]^T        (M=128, N=128: hi heads, lo heads)
